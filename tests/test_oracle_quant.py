@@ -1,0 +1,145 @@
+"""Pins for the oracle's quantizers and packing (CPU only).
+
+Brute force (argmin over all 16 codes), round-trip bounds, the packing golden
+examples and the special cases (zero rows, one-hot rows, constant KV vectors).
+"""
+
+import numpy as np
+import pytest
+
+from oracle import formats, hadamard, quant
+
+
+def _int4_bruteforce(x, s):
+    codes = np.arange(-8, 8)
+    d = np.abs(x[..., None] - codes * s)
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    # ties: choose the even integer (round half to even)
+    even = (codes % 2) == 0
+    pick = np.where((cand & even).any(axis=-1), np.argmax(cand & even, axis=-1), np.argmax(cand, axis=-1))
+    return codes[pick]
+
+
+def test_int4_bruteforce_and_bound():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((64, 256))
+    x[:, 3] *= 40
+    q, s, tie = quant.int4_sym_rows(x)
+    assert q.min() >= -7 and q.max() <= 7         # -8 never produced (s = amax / 7)
+    for r in range(x.shape[0]):
+        bf = _int4_bruteforce(x[r], float(s[r]))
+        ok = (bf == q[r]) | tie[r]
+        assert ok.all()
+    err = np.abs(x - quant.int4_dequant(q, s))
+    assert np.all(err <= s.astype(np.float64)[:, None] * (0.5 + 1e-6))
+    # the extreme element of every row maps to +-7
+    arg = np.abs(x).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(64), arg]) == 7)
+
+
+def test_int4_scale_is_fp32_amax_over_7():
+    x = np.array([[0.0, -3.5, 1.0, 7.0 / 3.0]])
+    q, s, _ = quant.int4_sym_rows(x)
+    assert s.dtype == np.float32
+    assert s[0] == np.float32(3.5) / np.float32(7.0)
+    assert list(q[0]) == [0, -7, 2, 5]          # 1/0.5 = 2 ; (7/3)/0.5 = 4.67 -> 5
+
+
+def test_int4_zero_row():
+    q, s, tie = quant.int4_sym_rows(np.zeros((2, 16)))
+    assert np.all(q == 0) and np.all(s == 0) and not tie.any()
+
+
+def test_int4_half_even_ties():
+    # scale = 1: values k + 0.5 round to the even neighbour
+    x = np.array([[7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5]])
+    q, s, tie = quant.int4_sym_rows(x)
+    assert s[0] == 1.0
+    assert list(q[0]) == [7, 0, 2, 2, 0, -2, -2, 4]
+    assert list(tie[0]) == [False] + [True] * 7
+
+
+def test_packing_golden(golden):
+    for line in golden("int4_packing.txt"):
+        codes, packed = line.split(";")
+        c = np.array([int(t) for t in codes.split()])
+        p = np.array([int(t, 16) for t in packed.split()], dtype=np.uint8)
+        assert np.array_equal(quant.pack_nibbles(c), p)
+        assert np.array_equal(quant.unpack_nibbles(p, signed=True), c)
+
+
+def _nvfp4_bruteforce(x, sdec, g):
+    vals = np.array([formats.e2m1_decode(c) for c in range(16)]) * sdec * g
+    d = np.abs(x[:, None] - vals[None, :])
+    return vals[np.argmin(d, axis=1)]
+
+
+def test_nvfp4_bruteforce_and_structure():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((16, 256))
+    x[:, 7] *= 30
+    g = quant.nvfp4_global_scale(x)
+    assert g == np.float32(np.float32(np.abs(x).max()) / np.float32(2688.0))
+    e, sc, tie_e, tie_s = quant.nvfp4_rows(x, g)
+    assert sc.shape == (16, 16) and sc.max() <= 0x7E
+    xh = quant.nvfp4_dequant(e, sc, g)
+    sdec = formats.e4m3_values(sc)
+    for r in range(16):
+        for b in range(16):
+            sl = slice(16 * b, 16 * b + 16)
+            if sdec[r, b] == 0:
+                assert np.all(e[r, sl] == 0)
+                continue
+            bf = _nvfp4_bruteforce(x[r, sl], sdec[r, b], np.float64(g))
+            ok = (np.abs(bf - xh[r, sl]) == 0) | tie_e[r, sl]
+            assert ok.all()
+    # the global amax element lands on +-6 * S * g with S = 448 (up to E4M3 rounding)
+    r, c = np.unravel_index(np.abs(x).argmax(), x.shape)
+    assert sc[r, c // 16] == 0x7E
+    assert abs(formats.e2m1_decode(e[r, c])) == 6.0
+
+
+def test_nvfp4_static_scale_saturates():
+    x = np.full((1, 16), 100.0)
+    e, sc, _, _ = quant.nvfp4_rows(x, np.float32(0.001))     # far too small a g
+    assert sc[0, 0] == 0x7E and np.all(e == 7)
+
+
+def test_nvfp4_zero_block():
+    x = np.zeros((2, 32))
+    x[0, 20] = 1.0
+    g = quant.nvfp4_global_scale(x)
+    e, sc, _, _ = quant.nvfp4_rows(x, g)
+    assert sc[0, 0] == 0 and np.all(e[0, :16] == 0) and np.all(sc[1] == 0)
+
+
+def test_kv4_bruteforce_and_bound():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((3, 5, 128))
+    xr = hadamard.rotate(x.reshape(-1, 128), rng.choice([-1, 1], size=128), 128).reshape(x.shape)
+    q, s_h, z_h, tie, _ = quant.kv4_vectors(xr)
+    assert q.min() >= 0 and q.max() <= 15
+    codes = np.arange(16)
+    recon = codes[None, None, None, :] * s_h[..., None, None] + z_h[..., None, None]
+    bf = np.argmin(np.abs(xr[..., None] - recon), axis=-1)
+    assert np.all((bf == q) | tie)
+    lo, hi = xr.min(-1), xr.max(-1)
+    s = (hi - lo) / 15
+    bound = s_h / 2 + np.abs(lo - z_h) + 15 * np.abs(s - s_h)
+    assert np.all(np.abs(xr - quant.kv4_dequant(q, s_h, z_h)) <= bound[..., None] * (1 + 1e-9))
+    # scale and zero are fp16 values
+    assert np.array_equal(formats.to_fp16(s_h), s_h) and np.array_equal(formats.to_fp16(z_h), z_h)
+
+
+def test_kv4_constant_vector():
+    x = np.full((1, 128), 3.0)
+    q, s_h, z_h, _, _ = quant.kv4_vectors(x)
+    assert np.all(q == 0) and s_h[0] == 0 and z_h[0] == 3.0
+
+
+@pytest.mark.parametrize("k", [16, 512])
+def test_unpack_roundtrip_unsigned(k):
+    rng = np.random.default_rng(k)
+    c = rng.integers(0, 16, size=(3, k))
+    assert np.array_equal(quant.unpack_nibbles(quant.pack_nibbles(c), signed=False), c)
