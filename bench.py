@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the rotation-based W4A4 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the online path over one batch of synthetic input:
+  rq_rotate_quantize(X)   randomized Hadamard + quantize + pack (HBM-bound)
+  rq_w4a4_gemm(Xq, Wq)    quantized GEMM on tcgen05 tensor cores
+with the weights rotated and quantized once beforehand (the offline side).
+For the KV workload a step is rq_kv_rotate_quantize on K and on V.
+
+The metric is the pair "fused Hadamard+quant GB/s vs HBM peak; W4A4 GEMM TOPS
+vs tensor peak": `value` is the fused rotate+quantize throughput in GB/s
+(algorithmic bytes / device time), and the `gemm` object carries the GEMM's
+TOPS.  Times are CUDA events on the launching stream, L2 is flushed between
+steps, and for N > 1 each rank runs its own batch (weak scaling, no data-path
+collective) and the time is the max over ranks.
+"""
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from rotation_w4a4_quantization_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "fused Hadamard+quant GB/s vs HBM peak; W4A4 GEMM TOPS vs tensor peak"
+L2_FLUSH_BYTES = 256 << 20
+DEFAULT_WORKLOAD = "q_proj_int4"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--y-dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+# --------------------------------------------------------------------------- workload
+class Workload:
+    """Device-resident inputs and the step function for one workload."""
+
+    def __init__(self, name, rq, device, seed_offset, y_dtype):
+        self.name = name
+        self.rq = rq
+        self.cfg = syn.WORKLOADS[name]
+        self.y_dtype = y_dtype
+        self.kv = name == "kv4"
+        if self.kv:
+            c = self.cfg
+            self.k = syn.kv(device=device, which=0, seed_offset=seed_offset)
+            self.v = syn.kv(device=device, which=1, seed_offset=seed_offset)
+            self.signs = syn.workload_signs(name).to(device)
+            shape = (c["B"], c["H"], c["S"])
+            self.outs = [(torch.empty(shape + (64,), dtype=torch.uint8, device=device),
+                          torch.empty(shape, dtype=torch.float16, device=device),
+                          torch.empty(shape, dtype=torch.float16, device=device)) for _ in range(2)]
+            n_vec = 2 * c["B"] * c["H"] * c["S"]
+            self.quant_bytes = n_vec * (128 * 2 + 64 + 2 + 2)
+            self.gemm_ops = 0
+            self.h2d_bytes = 2 * self.k.numel() * 2
+        else:
+            c = self.cfg
+            self.fmt = c["fmt"]
+            self.block = c["block"]
+            self.x = syn.activations(name, device=device, seed_offset=seed_offset)
+            w = syn.weights(name, device=device)
+            self.signs = syn.workload_signs(name).to(device)
+            self.wq = rq.prepare_weights(w, self.signs, self.block, self.fmt)
+            del w
+            m, k, n = c["M"], c["K"], c["N"]
+            self.xq_out = rq._alloc_quant_outputs(m, k, rq._fmt(self.fmt), device)
+            self.gscale = torch.empty((1,), dtype=torch.float32, device=device)
+            self.ws = torch.empty((16,), dtype=torch.uint8, device=device)
+            self.y = torch.empty((m, n), dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32,
+                                 device=device)
+            scale_bytes = m * 4 if self.fmt == "int4" else m * (k // 16)
+            self.quant_bytes = m * k * 2 + m * k // 2 + scale_bytes
+            self.gemm_ops = 2 * m * n * k
+            self.h2d_bytes = self.x.numel() * 2
+        self.d2h_bytes = 0
+
+    def quant_launches(self):
+        if self.kv:
+            return 2
+        return 2 if self.fmt == "nvfp4" else 1
+
+    def gemm_launches(self):
+        return 0 if self.kv else 1
+
+    def quant(self):
+        rq = self.rq
+        if self.kv:
+            rq.kv_rotate_quantize(self.k, self.signs, out=self.outs[0])
+            rq.kv_rotate_quantize(self.v, self.signs, out=self.outs[1])
+            return None
+        return rq.rotate_quantize(self.x, self.signs, self.block, self.fmt, "dynamic", gscale=self.gscale,
+                                  out=self.xq_out, workspace=self.ws)
+
+    def gemm(self, xq):
+        if self.kv:
+            return None
+        return self.rq.w4a4_gemm(xq, self.wq, self.fmt, self.y_dtype, y=self.y)
+
+    def result(self):
+        return self.outs[0][0] if self.kv else self.y
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", "rq_clocks_%d_%d.csv" % (os.getpid(), index))
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [t.strip() for t in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    mhz.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not mhz:
+            return None
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(name, rows):
+    """Time the oracle (as it stands) on `rows` rows of the workload; returns (GB/s, TOPS, seconds, desc, threads)."""
+    from oracle import gemm as ogemm, hadamard as ohad, quant as oquant
+    c = syn.WORKLOADS[name]
+    if name == "kv4":
+        kv = syn.kv(batch=1, heads=4, seq=rows)
+        s = syn.workload_signs(name).numpy()
+        x = kv.to(torch.float64).numpy().reshape(-1, 128)
+        t0 = time.perf_counter()
+        xr = ohad.rotate(x, s, 128)
+        q, sh, zh, _, _ = oquant.kv4_vectors(xr)
+        oquant.pack_nibbles(q)
+        dt = time.perf_counter() - t0
+        nbytes = x.shape[0] * (128 * 2 + 64 + 4)
+        return nbytes / dt / 1e9, None, dt, "%d head_dim vectors (1 x 4 heads x %d tokens)" % (x.shape[0], rows)
+    x = syn.activations(name, rows=rows).to(torch.float64).numpy()
+    w = syn.weights(name).to(torch.float64).numpy()
+    s = syn.workload_signs(name).numpy()
+    k, n = c["K"], c["N"]
+    block = c["block"]
+    wr = ohad.rotate(w, s, block)
+    if c["fmt"] == "int4":
+        qw, sw, _ = oquant.int4_sym_rows(wr)
+    else:
+        gw = oquant.nvfp4_global_scale(wr)
+        ew, sfw, _, _ = oquant.nvfp4_rows(wr, gw)
+    t0 = time.perf_counter()
+    xr = ohad.rotate(x, s, block)
+    if c["fmt"] == "int4":
+        qx, sx, _ = oquant.int4_sym_rows(xr)
+        oquant.pack_nibbles(qx)
+    else:
+        gx = oquant.nvfp4_global_scale(xr)
+        ex, sfx, _, _ = oquant.nvfp4_rows(xr, gx)
+        oquant.pack_nibbles(ex)
+    t1 = time.perf_counter()
+    if c["fmt"] == "int4":
+        ogemm.int4_y(ogemm.int4_acc(qx, qw), sx, sw)
+    else:
+        ogemm.nvfp4_y(ex, sfx, gx, ew, sfw, gw)
+    t2 = time.perf_counter()
+    scale_bytes = rows * 4 if c["fmt"] == "int4" else rows * (k // 16)
+    nbytes = rows * k * 2 + rows * k // 2 + scale_bytes
+    return (nbytes / (t1 - t0) / 1e9, 2.0 * rows * n * k / (t2 - t1) / 1e12, t2 - t0,
+            "%d of %d rows of X with the full W" % (rows, c["M"]))
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def sample_rows(name):
+    return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096}[name]
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from rotation_w4a4_quantization_b200 import rq
+    rq.init(local)
+    wl = Workload(args.workload, rq, dev, seed_offset=rank, y_dtype=args.y_dtype)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        xq = wl.quant()
+        if ev is not None:
+            ev[1].record(stream)
+        wl.gemm(xq)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    rq.get_device_error()
+    torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()           # evict L2 (126 MB) between steps
+        step(events[i])
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    rq.get_device_error()
+
+    q_ms = np.array([e[0].elapsed_time(e[1]) for e in events])
+    g_ms = np.array([e[1].elapsed_time(e[2]) for e in events])
+    step_ms = q_ms + g_ms
+    tot = torch.tensor([step_ms.sum(), q_ms.sum(), g_ms.sum()], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    tot = tot.cpu().numpy()
+    K = args.steps
+    ms_step = tot[0] / K
+    q_mean_ms = tot[1] / K
+    g_mean_ms = tot[2] / K
+
+    # end to end through the public API: pinned host input -> device -> path -> host result
+    e2e = measure_e2e(wl, rq, dev, stream, K=min(K, 20))
+
+    peaks = load_peaks()
+    quant_gbs = wl.quant_bytes * world / (q_mean_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(quant_gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4" if args.workload != "q_proj_nvfp4" else "nvfp4",
+        "data": "synthetic (seeded, shaped like the article's Qwen3-8B layer inputs)",
+        "config": workload_config(args, wl),
+        "gpu_launches": K * (wl.quant_launches() + wl.gemm_launches()),
+    }
+    q_launch_ms = q_mean_ms / wl.quant_launches()
+    roof_q = {"bound": "hbm", "achieved": round(wl.quant_bytes / wl.quant_launches() / (q_launch_ms * 1e-3) / 1e9, 1),
+              "peak": peaks["hbm"], "unit": "GB/s", "traffic": None,
+              "kernel": "rotate_full_kernel" if (not wl.kv and wl.block == 0) else "rotate_block_kernel",
+              "peak_source": peaks["src"]}
+    roof_q["frac"] = round(roof_q["achieved"] / roof_q["peak"], 4)
+    if wl.gemm_launches():
+        ratio = 2.0  # INT8 and FP4 dense tensor peaks are 2x / 4x the bf16 one (nominal ratios)
+        if wl.fmt == "nvfp4":
+            ratio = 4.0
+        tops = wl.gemm_ops * world / (g_mean_ms * 1e-3) / 1e12
+        peak_t = peaks["bf16"] * ratio
+        roof_g = {"bound": "tensor", "achieved": round(wl.gemm_ops / (g_mean_ms * 1e-3) / 1e12, 1), "peak": peak_t,
+                  "unit": "TFLOP/s", "traffic": None,
+                  "kernel": "gemm_int4_kernel" if wl.fmt == "int4" else "gemm_nvfp4_kernel",
+                  "peak_source": "%s bf16 x %g (nominal %s/bf16 ratio)" % (peaks["src"], ratio,
+                                                                           "int8" if ratio == 2 else "fp4")}
+        roof_g["frac"] = round(roof_g["achieved"] / peak_t, 4)
+        out["gemm"] = {"value": round(tops, 2), "unit": "TOPS", "ms": round(g_mean_ms, 5),
+                       "frac_of_peak": roof_g["frac"]}
+        dominant = roof_g if g_mean_ms >= q_mean_ms else roof_q
+        out["roofline"] = dominant
+        out["roofline_hadamard_quant"] = roof_q
+        out["roofline_gemm"] = roof_g
+    else:
+        out["roofline"] = roof_q
+    out["hadamard_quant_ms"] = round(q_mean_ms, 5)
+    out["e2e"] = e2e
+    out["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, tops_cpu, secs, desc = oracle_sample(args.workload, sample_rows(args.workload))
+        out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                               "sample": desc, "seconds": round(secs, 2), "host_cpus": os.cpu_count()}
+        if tops_cpu is not None:
+            out["cpu_baseline"]["gemm_tops"] = round(tops_cpu, 5)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_e2e(wl, rq, dev, stream, K):
+    """Same metric through the public API with host buffers: the timed region holds,
+    per step, the pinned host -> device copy of the step's input, the path, and the
+    device -> host copy of its result."""
+    if wl.kv:
+        host_in = [wl.k.cpu().pin_memory(), wl.v.cpu().pin_memory()]
+        dev_in = [wl.k, wl.v]
+    else:
+        host_in = [wl.x.cpu().pin_memory()]
+        dev_in = [wl.x]
+    res = wl.result()
+    host_out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(K + 2):
+        if i == 2:
+            ev0.record(stream)
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        xq = wl.quant()
+        wl.gemm(xq)
+        host_out.copy_(wl.result(), non_blocking=True)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / K
+    return {"value": round(wl.quant_bytes / (ms * 1e-3) / 1e9, 3), "unit": "GB/s", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def workload_config(args, wl):
+    c = dict(syn.WORKLOADS[args.workload])
+    c.pop("index", None)
+    cfg = {"workload": args.workload}
+    cfg.update(c)
+    if not wl.kv:
+        cfg["block"] = "full" if wl.block == 0 else wl.block
+        cfg["y_dtype"] = args.y_dtype
+        cfg["weights"] = "rotated+quantized once before timing (offline side)"
+    cfg["l2"] = "flushed between steps (256 MiB memset, outside the kernel events)"
+    return cfg
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    K = args.steps
+    rows = sample_rows(args.workload)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample(args.workload, max(8, rows // 8))
+    vals, secs = [], 0.0
+    for _ in range(K):
+        gbs, tops, s, desc = oracle_sample(args.workload, rows)
+        vals.append(gbs)
+        secs += s
+    v = float(np.mean(vals))
+    out = {
+        "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / K, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+        "config": {"workload": args.workload, "sample_rows": rows},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * rq.h -- C ABI of librq: the online hot path of rotation-based W4A4
+ * quantization (QuaRot / SpinQuant style) on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Rotations for 4-Bit Activations: QuaRot, SpinQuant, and
+ * Friends", section "A rotation changes nothing, and that is the point"):
+ * a linear layer Y = X.W^T equals (X.Q).(W.Q)^T for any orthogonal Q, so X.Q
+ * and W.Q are quantized instead of X and W.  Q is a randomized Hadamard matrix
+ * scaled by 1/sqrt(n) -- a +-1 sign per channel followed by a Sylvester
+ * Hadamard -- either over all K channels or block-diagonal in 128-wide blocks
+ * (sections "The recipe" and "Gotchas"; QuaRot page, "Activation scheme").
+ *
+ *   Q = blockdiag_{K/B}( diag(s_blk) . H_B / sqrt(B) ),  B = 128 or B = K,
+ *   H_B[i][j] = (-1)^popcount(i & j).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are DEVICE pointers owned by the caller; the
+ *    library never allocates, frees or retains them.  Host arrays are named
+ *    *_host.  Matrices are row-major; leading dimensions are in elements.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and never synchronizes, except
+ *    rq_get_device_error and rq_init.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call returns a status other than RQ_OK and leaves every output
+ *    untouched.  RQ_ERR_CUDA reports a launch failure (cudaGetLastError).
+ *  - Kernels that wait on barriers give up after about one second, record
+ *    RQ_ERR_TIMEOUT in a device word and return; rq_get_device_error reads it.
+ *  - Codes are packed two per byte, element 2i in the low nibble (bits 0-3),
+ *    element 2i+1 in the high nibble.  INT4 codes are two's complement in
+ *    [-7, 7]; KV4 codes unsigned in [0, 15]; NVFP4 codes are E2M1 with the
+ *    sign in bit 3 (a value that rounds to zero is written as +0).
+ *  - Inputs must be finite and, for KV4, within the fp16 range; NaN or Inf
+ *    inputs give unspecified codes.
+ */
+#ifndef RQ_H_
+#define RQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RQ_API __attribute__((visibility("default")))
+#else
+#define RQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* rq_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  RQ_OK = 0,
+  RQ_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+  RQ_ERR_UNSUPPORTED_SHAPE = 2, /* K, block or head_dim outside what the kernels support */
+  RQ_ERR_ALIGNMENT = 3,         /* a pointer or leading dimension breaks the stated alignment */
+  RQ_ERR_UNSUPPORTED_DEVICE = 4,/* not a compute-capability 10.0 GPU, or the sm_100a image does not load */
+  RQ_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+  RQ_ERR_TIMEOUT = 6            /* a kernel gave up on a bounded wait (see rq_get_device_error) */
+} rq_status;
+
+typedef enum { RQ_INT4 = 0, RQ_NVFP4 = 1 } rq_format;
+
+typedef enum {
+  RQ_OUT_F32 = 0,     /* Y as fp32 */
+  RQ_OUT_BF16 = 1,    /* Y as bf16 (round to nearest even) */
+  RQ_OUT_I32_ACC = 2  /* INT4 only: the raw int32 accumulators sum_k qx*qw, no scales */
+} rq_out;
+
+typedef enum {
+  RQ_SCALE_DYNAMIC = 0, /* NVFP4 per-tensor scale from the rotated tensor's own max */
+  RQ_SCALE_STATIC = 1   /* NVFP4 per-tensor scale supplied by the caller */
+} rq_gscale;
+
+/* Checks that `device` is a compute-capability 10.0 GPU and that this
+ * library's sm_100a kernels load on it.  Synchronous.  Call once per device
+ * before the other entry points (they do not call it themselves). */
+RQ_API rq_status rq_init(int device);
+
+/* Static description of a status code.  Never NULL. */
+RQ_API const char* rq_status_string(rq_status status);
+
+/* Bytes of device workspace rq_rotate_quantize / rq_prepare_weights need:
+ * 16 for NVFP4 (the dynamic-scale max word), 0 for INT4.  The workspace must
+ * be 16-byte aligned; its contents need not be initialised. */
+RQ_API size_t rq_workspace_bytes(rq_format fmt);
+
+/*
+ * rq_rotate_quantize: X~ = X.Q, then quantize and pack (the online activation
+ * side; "What it buys in 4 bits, and what it doesn't": INT4 with one scale per
+ * token, or NVFP4 with an FP8 scale for every block of 16 values).
+ *
+ *  X_dev      bf16 [M, ldx]; rows 16-byte aligned (X_dev and ldx*2 multiples of 16).
+ *  M          rows (tokens), >= 0.  M = 0 is a no-op.
+ *  K          channels; a multiple of 128, at most 32768.
+ *  signs_dev  int8 [K], each +1 or -1 (the random sign diagonal; any other value
+ *             is read as +1 if positive and -1 otherwise).
+ *  block      128 for 128-wide blocks, or 0 for a full-width rotation (then K
+ *             must be a power of two in [256, 4096]; INT4 only).
+ *  fmt        RQ_INT4:
+ *               codes_dev  uint8 [M, K/2], scales_dev float [M]:
+ *               s = amax/7 (fp32, amax = max |x~| of the row); q = rint(x~/s).
+ *             RQ_NVFP4 (block must be 128):
+ *               codes_dev  uint8 [M, K/2] E2M1 codes,
+ *               scales_dev uint8 [M, K/16] E4M3 block scales,
+ *               gscale_dev float scalar g:
+ *                 RQ_SCALE_DYNAMIC: written, g = fp32(amax(X~)) / 2688;
+ *                 RQ_SCALE_STATIC : read.
+ *               S_b = E4M3_rn_satfinite(amax_b / (6 g));
+ *               e = E2M1_rn_satfinite(x~ / (S_b g)); S_b = 0 gives e = 0.
+ *  workspace_dev  rq_workspace_bytes(fmt) bytes (may be NULL when that is 0).
+ *  codes_dev and scales_dev 16-byte aligned (8 for NVFP4 scales).
+ * Values that sit within a few fp32 ulps of a rounding boundary may round
+ * either way (the rotation is computed in fp32).
+ */
+RQ_API rq_status rq_rotate_quantize(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev,
+                             int block, rq_format fmt, rq_gscale gmode, uint8_t* codes_dev, void* scales_dev,
+                             float* gscale_dev, void* workspace_dev, rq_stream_t stream);
+
+/*
+ * rq_prepare_weights: the offline side, W~ = W.Q then quantize and pack, with
+ * the same Q as the activations so (X.Q)(W.Q)^T = X.W^T ("Where the rotations
+ * go": offline rotations are folded into the weights).  A row of W is an
+ * output channel, so INT4 gives one scale per output channel.  Same arguments,
+ * layouts and errors as rq_rotate_quantize with X -> W [N, K]; NVFP4 always
+ * uses the dynamic per-tensor scale (gscale_dev is written).
+ */
+RQ_API rq_status rq_prepare_weights(const void* W_dev, int64_t N, int64_t K, int64_t ldw, const int8_t* signs_dev,
+                             int block, rq_format fmt, uint8_t* codes_dev, void* scales_dev, float* gscale_dev,
+                             void* workspace_dev, rq_stream_t stream);
+
+/*
+ * rq_w4a4_gemm: Y[M, N] = deq(X codes) . deq(W codes)^T, the quantized
+ * product of section "What it buys in 4 bits, and what it doesn't".
+ *  RQ_INT4 : xscales_dev float [M], wscales_dev float [N] (16-byte aligned);
+ *            acc = sum_k qx[m,k] qw[n,k] exactly in int32; Y = acc * sx[m] * sw[n].
+ *            xgscale_dev / wgscale_dev unused (may be NULL).
+ *  RQ_NVFP4: xscales_dev uint8 [M, K/16], wscales_dev uint8 [N, K/16] (E4M3, 16-byte aligned),
+ *            xgscale_dev / wgscale_dev float scalars;
+ *            Y = gx gw sum_b Sx[m,b] Sw[n,b] sum_{k in b} ex ew.
+ *  xcodes_dev uint8 [M, K/2], wcodes_dev uint8 [N, K/2], both 16-byte aligned.
+ *  K a multiple of 128 (INT4) or 256 (NVFP4), at most 65536; M, N >= 0.
+ *  Y_dev [M, ldy] of fp32, bf16 or int32 per `out`; ldy >= N; Y_dev aligned to
+ *  its element size (16-byte aligned rows are stored with vector stores).
+ */
+RQ_API rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev, const float* xgscale_dev,
+                       const uint8_t* wcodes_dev, const void* wscales_dev, const float* wgscale_dev, int64_t M,
+                       int64_t N, int64_t K, rq_format fmt, void* Y_dev, int64_t ldy, rq_out out,
+                       rq_stream_t stream);
+
+/*
+ * rq_kv_rotate_quantize: 4-bit KV cache entries ("QuaRot", "Activation
+ * scheme": the rotation is applied to the KV cache too; "SpinQuant",
+ * "Activation scheme": asymmetric INT4 for the KV cache).  Each head_dim
+ * vector v of K or V [B, H, S, D] (D = 128) becomes v~ = v.diag(s).H_128/sqrt(128),
+ * then z = min(v~), s = (max(v~) - min(v~))/15, stored as fp16 z_h, s_h, and
+ * q = clamp(rint((v~ - z_h)/s_h), 0, 15) (s_h = 0 gives q = 0).
+ *  KV_dev      bf16, element (b,h,t,d) at KV_dev + b*strides_host[0] + h*strides_host[1]
+ *              + t*strides_host[2] + d (strides in elements; d contiguous; each
+ *              vector 16-byte aligned).
+ *  signs_dev   int8 [D].
+ *  codes_dev   uint8 [B, H, S, D/2] contiguous, 16-byte aligned.
+ *  scale_dev, zero_dev  fp16 [B, H, S] contiguous.
+ */
+RQ_API rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H, int64_t S, int64_t D,
+                                const int64_t* strides_host, const int8_t* signs_dev, uint8_t* codes_dev,
+                                void* scale_dev, void* zero_dev, rq_stream_t stream);
+
+/*
+ * rq_rotate_f32: the rotation alone, X~ = X.Q as fp32 [M, ldo] (ldo a multiple
+ * of 4, out_dev 16-byte aligned).  Same X, K, signs and block rules as
+ * rq_rotate_quantize (block 0 allowed for K a power of two in [256, 4096]).
+ * Intended for checking the rotation against a reference.
+ */
+RQ_API rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev, int block,
+                        float* out_dev, int64_t ldo, rq_stream_t stream);
+
+/* Synchronizes `stream`, returns RQ_ERR_TIMEOUT if any kernel of this library
+ * recorded a device-side timeout since the last call (and clears the record),
+ * RQ_ERR_CUDA if the stream reports an error, else RQ_OK. */
+RQ_API rq_status rq_get_device_error(rq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQ_H_ */

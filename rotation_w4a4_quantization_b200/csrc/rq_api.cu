@@ -1,0 +1,322 @@
+// librq: the C ABI declared in include/rq.h.  Host-side argument checks,
+// kernel selection and launches.  All kernels live in the headers included
+// below (one translation unit, so the device error word is a single symbol).
+#include "../../include/rq.h"
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "rq_common.cuh"
+#include "rq_rotate.cuh"
+#include "rq_gemm.cuh"
+
+namespace {
+
+using namespace rq;
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxKBlock = 32768;
+constexpr size_t kSmemBudget = 220 * 1024;
+
+int num_sms_of_current_device() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+// Raise a kernel's dynamic shared memory limit once per (kernel, device).
+bool ensure_smem(const void* kernel) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, uint64_t>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = (dev < 64) ? (1ull << dev) : 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : done)
+    if (e.first == kernel && bit && (e.second & bit)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget + 7 * 1024) !=
+      cudaSuccess)
+    return false;
+  for (auto& e : done)
+    if (e.first == kernel) {
+      e.second |= bit;
+      return true;
+    }
+  done.emplace_back(kernel, bit);
+  return true;
+}
+
+rq_status last_launch_status() { return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+struct RotCfg {
+  int R, stages, threads;
+  size_t smem;
+};
+
+RotCfg block_config(int64_t K) {
+  const int nb = (int)(K / 128);
+  RotCfg c;
+  c.R = (256 % nb == 0) ? 256 / nb : (nb <= 384 ? 384 / nb : 1);
+  if (c.R < 1) c.R = 1;
+  c.threads = c.R * nb;
+  const size_t sb = RotSmemLayout::stage_bytes(c.R, (int)K);
+  const size_t fixed = RotSmemLayout::total(c.R, (int)K, 0);
+  int st = (int)((kSmemBudget - fixed) / sb);
+  c.stages = st > 4 ? 4 : st;
+  c.smem = RotSmemLayout::total(c.R, (int)K, c.stages);
+  return c;
+}
+
+RotCfg full_config(int64_t K) {
+  const int NB = (int)(K / 128);
+  RotCfg c;
+  c.R = 256 / NB;
+  c.threads = 256;
+  const size_t sb = RotSmemLayout::stage_bytes(c.R, (int)K);
+  const size_t fixed = RotSmemLayout::total(c.R, (int)K, 0);
+  int st = (int)((kSmemBudget - fixed) / sb);
+  c.stages = st > 3 ? 3 : st;
+  c.smem = RotSmemLayout::total(c.R, (int)K, c.stages);
+  return c;
+}
+
+template <int MODE>
+rq_status launch_block(RotParams p, cudaStream_t st) {
+  const RotCfg c = block_config(p.K);
+  if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
+  p.R = c.R;
+  p.stages = c.stages;
+  p.num_tiles = (p.rows + c.R - 1) / c.R;
+  const int64_t grid = p.num_tiles < num_sms_of_current_device() ? p.num_tiles : num_sms_of_current_device();
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_block_kernel<MODE>))) return RQ_ERR_CUDA;
+  rotate_block_kernel<MODE><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
+  return last_launch_status();
+}
+
+template <int MODE, int NB>
+rq_status launch_full_nb(RotParams p, cudaStream_t st) {
+  const RotCfg c = full_config(p.K);
+  if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
+  p.R = c.R;
+  p.stages = c.stages;
+  p.num_tiles = (p.rows + c.R - 1) / c.R;
+  const int64_t grid = p.num_tiles < num_sms_of_current_device() ? p.num_tiles : num_sms_of_current_device();
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_full_kernel<MODE, NB>))) return RQ_ERR_CUDA;
+  rotate_full_kernel<MODE, NB><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
+  return last_launch_status();
+}
+
+template <int MODE>
+rq_status launch_full(RotParams p, cudaStream_t st) {
+  switch (p.nb) {
+    case 2: return launch_full_nb<MODE, 2>(p, st);
+    case 4: return launch_full_nb<MODE, 4>(p, st);
+    case 8: return launch_full_nb<MODE, 8>(p, st);
+    case 16: return launch_full_nb<MODE, 16>(p, st);
+    case 32: return launch_full_nb<MODE, 32>(p, st);
+    default: return RQ_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
+// Common checks of the X / K / signs / block arguments.
+// Pointers are only required (and checked) when there is work: M = 0 is a no-op.
+rq_status check_rotation_args(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* signs, int block) {
+  if (M > 0 && (!X || !signs)) return RQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || ldx < K) return RQ_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K > kMaxKBlock) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (block != 0 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (block == 0 && !(is_pow2(K) && K >= 256 && K <= 4096)) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || (ldx * 2) % 16 != 0) return RQ_ERR_ALIGNMENT;
+  return RQ_OK;
+}
+
+RotParams matrix_params(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* signs) {
+  RotParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.x = static_cast<const uint8_t*>(X);
+  p.rows = M;
+  p.K = (int)K;
+  p.nb = (int)(K / 128);
+  p.S = M > 0 ? M : 1;
+  p.H = 1;
+  p.sS = ldx * 2;
+  p.sH = 0;
+  p.sB = 0;
+  p.signs = signs;
+  p.cfull = (float)(1.0 / std::sqrt((double)K));
+  return p;
+}
+
+rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* signs, int block,
+                               rq_format fmt, rq_gscale gmode, uint8_t* codes, void* scales, float* gscale,
+                               void* workspace, cudaStream_t st) {
+  rq_status s = check_rotation_args(X, M, K, ldx, signs, block);
+  if (s != RQ_OK) return s;
+  if (fmt != RQ_INT4 && fmt != RQ_NVFP4) return RQ_ERR_INVALID_ARG;
+  if (gmode != RQ_SCALE_DYNAMIC && gmode != RQ_SCALE_STATIC) return RQ_ERR_INVALID_ARG;
+  if (fmt == RQ_NVFP4 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return RQ_OK;
+  if (!codes || !scales) return RQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 16)) return RQ_ERR_ALIGNMENT;
+  if (fmt == RQ_NVFP4) {
+    if (!gscale) return RQ_ERR_INVALID_ARG;
+    if (gmode == RQ_SCALE_DYNAMIC && !workspace) return RQ_ERR_INVALID_ARG;
+    if (!aligned(scales, 8) || !aligned(gscale, 4)) return RQ_ERR_ALIGNMENT;
+    if (workspace && !aligned(workspace, 16)) return RQ_ERR_ALIGNMENT;
+  } else {
+    if (!aligned(scales, 4)) return RQ_ERR_ALIGNMENT;
+  }
+  if (M == 0) return RQ_OK;
+
+  RotParams p = matrix_params(X, M, K, ldx, signs);
+  p.codes = codes;
+  if (fmt == RQ_INT4) {
+    p.scales_f32 = static_cast<float*>(scales);
+    if (block == 0) return launch_full<kModeInt4>(p, st);
+    return launch_block<kModeInt4>(p, st);
+  }
+  p.scales_e4m3 = static_cast<uint8_t*>(scales);
+  if (gmode == RQ_SCALE_DYNAMIC) {
+    p.amax_word = static_cast<unsigned*>(workspace);
+    if (cudaMemsetAsync(workspace, 0, sizeof(unsigned), st) != cudaSuccess) return RQ_ERR_CUDA;
+    s = launch_block<kModeAmax>(p, st);
+    if (s != RQ_OK) return s;
+    p.nvfp4_dynamic = 1;
+    p.g_out = gscale;
+  } else {
+    p.nvfp4_dynamic = 0;
+    p.g_in = gscale;
+  }
+  return launch_block<kModeNvfp4>(p, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rq_status_string(rq_status status) {
+  switch (status) {
+    case RQ_OK: return "ok";
+    case RQ_ERR_INVALID_ARG: return "invalid argument";
+    case RQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case RQ_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case RQ_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0, sm_100a)";
+    case RQ_ERR_CUDA: return "CUDA error";
+    case RQ_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+rq_status rq_init(int device) {
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || device < 0 || device >= n) return RQ_ERR_UNSUPPORTED_DEVICE;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return RQ_ERR_UNSUPPORTED_DEVICE;
+  if (prop.major != 10 || prop.minor != 0) return RQ_ERR_UNSUPPORTED_DEVICE;
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess) return RQ_ERR_CUDA;
+  if (cudaSetDevice(device) != cudaSuccess) return RQ_ERR_CUDA;
+  cudaFuncAttributes attr;
+  const cudaError_t e = cudaFuncGetAttributes(&attr, rotate_block_kernel<kModeInt4>);
+  (void)cudaSetDevice(prev);
+  if (e != cudaSuccess) return RQ_ERR_UNSUPPORTED_DEVICE;
+  return RQ_OK;
+}
+
+size_t rq_workspace_bytes(rq_format fmt) { return fmt == RQ_NVFP4 ? 16 : 0; }
+
+rq_status rq_rotate_quantize(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev,
+                             int block, rq_format fmt, rq_gscale gmode, uint8_t* codes_dev, void* scales_dev,
+                             float* gscale_dev, void* workspace_dev, rq_stream_t stream) {
+  return rotate_quantize_impl(X_dev, M, K, ldx, signs_dev, block, fmt, gmode, codes_dev, scales_dev, gscale_dev,
+                              workspace_dev, static_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_prepare_weights(const void* W_dev, int64_t N, int64_t K, int64_t ldw, const int8_t* signs_dev,
+                             int block, rq_format fmt, uint8_t* codes_dev, void* scales_dev, float* gscale_dev,
+                             void* workspace_dev, rq_stream_t stream) {
+  return rotate_quantize_impl(W_dev, N, K, ldw, signs_dev, block, fmt, RQ_SCALE_DYNAMIC, codes_dev, scales_dev,
+                              gscale_dev, workspace_dev, static_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev, int block,
+                        float* out_dev, int64_t ldo, rq_stream_t stream) {
+  rq_status s = check_rotation_args(X_dev, M, K, ldx, signs_dev, block);
+  if (s != RQ_OK) return s;
+  if (ldo < K) return RQ_ERR_INVALID_ARG;
+  if (M == 0) return RQ_OK;
+  if (!out_dev) return RQ_ERR_INVALID_ARG;
+  if (!aligned(out_dev, 16) || ldo % 4 != 0) return RQ_ERR_ALIGNMENT;
+  RotParams p = matrix_params(X_dev, M, K, ldx, signs_dev);
+  p.out_f32 = out_dev;
+  p.ldo = ldo;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (block == 0) return launch_full<kModeF32>(p, st);
+  return launch_block<kModeF32>(p, st);
+}
+
+rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H, int64_t S, int64_t D,
+                                const int64_t* strides_host, const int8_t* signs_dev, uint8_t* codes_dev,
+                                void* scale_dev, void* zero_dev, rq_stream_t stream) {
+  if (B < 0 || H < 0 || S < 0) return RQ_ERR_INVALID_ARG;
+  if (D != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (B * H * S == 0) return RQ_OK;
+  if (!KV_dev || !strides_host || !signs_dev || !codes_dev || !scale_dev || !zero_dev) return RQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (strides_host[i] < 0) return RQ_ERR_INVALID_ARG;
+  if (!aligned(KV_dev, 16) || !aligned(codes_dev, 16) || !aligned(scale_dev, 2) || !aligned(zero_dev, 2))
+    return RQ_ERR_ALIGNMENT;
+  for (int i = 0; i < 3; ++i)
+    if ((strides_host[i] * 2) % 16 != 0) return RQ_ERR_ALIGNMENT;
+  const int64_t rows = B * H * S;
+  if (rows == 0) return RQ_OK;
+  RotParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.x = static_cast<const uint8_t*>(KV_dev);
+  p.rows = rows;
+  p.K = 128;
+  p.nb = 1;
+  p.S = S;
+  p.H = H;
+  p.sB = strides_host[0] * 2;
+  p.sH = strides_host[1] * 2;
+  p.sS = strides_host[2] * 2;
+  p.signs = signs_dev;
+  p.codes = codes_dev;
+  p.kv_scale = static_cast<__half*>(scale_dev);
+  p.kv_zero = static_cast<__half*>(zero_dev);
+  return launch_block<kModeKv4>(p, static_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev, const float* xgscale_dev,
+                       const uint8_t* wcodes_dev, const void* wscales_dev, const float* wgscale_dev, int64_t M,
+                       int64_t N, int64_t K, rq_format fmt, void* Y_dev, int64_t ldy, rq_out out,
+                       rq_stream_t stream) {
+  return rq::gemm_dispatch(xcodes_dev, xscales_dev, xgscale_dev, wcodes_dev, wscales_dev, wgscale_dev, M, N, K, fmt,
+                           Y_dev, ldy, out, static_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_get_device_error(rq_stream_t stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RQ_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, rq::g_device_error, sizeof(v)) != cudaSuccess) return RQ_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(rq::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return RQ_ERR_CUDA;
+  return v ? RQ_ERR_TIMEOUT : RQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,608 @@
+// W4A4 GEMM on the 5th-generation tensor cores (tcgen05), sm_100a.
+//
+// Y[M,N] = deq(X codes) . deq(W codes)^T -- the quantized product of
+// "Rotations for 4-Bit Activations: QuaRot, SpinQuant, and Friends", section
+// "What it buys in 4 bits, and what it doesn't".  Both operands were rotated
+// by the same Q, so this equals the layer output up to quantization error
+// (section "A rotation changes nothing, and that is the point").
+//
+// INT4 path (kind::i8).  Blackwell has no 4-bit x 4-bit integer MMA (the
+// SpinQuant and QuaRot pages make the same point about earlier hardware), so
+// the packed nibbles are widened to int8 in shared memory.  Each nibble q is
+// placed in the HIGH half of its byte (the byte is 16*q, exact in int8), which
+// needs only a mask and a byte permute per four codes; the MMA then
+// accumulates 256 * sum(qx*qw) exactly in int32 (|acc| <= 2^14 K < 2^31 for
+// K <= 65536) and the epilogue shifts right by 8.
+//
+// NVFP4 path (kind::mxf4nvf4, block16).  E2M1 codes go by TMA straight into
+// 128B-swizzled shared memory; the E4M3 block scales are written into tensor
+// memory with tcgen05.st in the layout the block-scaled MMA reads: for a
+// 64-wide K slice, row r's four scales sit in lane (r mod 32) of every lane
+// quadrant, column r/32.
+//
+// Both kernels are persistent (one CTA per SM) and warp-specialized:
+//   warp 0      TMA producer (one elected lane)
+//   warp 1      TMEM allocator + MMA issuer (one elected lane)
+//   warps 2-5   INT4: nibble -> int8 converters;  NVFP4: scale loaders
+//   warps 6-9   epilogue: TMEM -> registers -> scale -> global
+// CTA tile 128 x 256 (M x N), accumulators in TMEM (int32 or fp32).
+#pragma once
+
+#include <cuda.h>
+
+#include "rq_common.cuh"
+#include "rq_tc.cuh"
+
+namespace rq {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kGemmThreads = 320;
+
+struct GemmParams {
+  int M, N, K;
+  const void* xscale;   // INT4: float [M]; NVFP4: uint8 [M, K/16]
+  const void* wscale;   // INT4: float [N]; NVFP4: uint8 [N, K/16]
+  const float* xg;      // NVFP4 per-tensor scales
+  const float* wg;
+  void* y;
+  int64_t ldy;
+  int out;              // 0 f32, 1 bf16, 2 i32 accumulators
+  int vec_ok;           // 1: Y rows allow 16-byte vector stores
+  int tiles_m, tiles_n, num_tiles;
+};
+
+// Bounded wait used by every role; on timeout the role stops issuing work.
+__device__ __forceinline__ bool wait_or_fail(uint64_t* bar, unsigned parity, int* abort_flag) {
+  if (*((volatile int*)abort_flag)) return false;
+  if (!mbar_wait_bounded(bar, parity)) {
+    *((volatile int*)abort_flag) = 1;
+    return false;
+  }
+  return true;
+}
+
+// Epilogue for one 32-row x 256-column slab held by this warp's TMEM lanes.
+// acc_kind 0: int32 accumulators of 256*sum (INT4), 1: fp32 (NVFP4).
+template <int ACC_KIND>
+__device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tacc, int m0, int n0, int q, int lane,
+                                               float rowscale, const float* colscale, float gscale) {
+  const int row = m0 + 32 * q + lane;
+  const bool row_ok = row < p.M;
+#pragma unroll 1
+  for (int cc = 0; cc < kBN / 32; ++cc) {
+    uint32_t r[32];
+    __syncwarp();
+    tmem_ld32(tacc + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * cc), r);
+    tmem_wait_ld();
+    const int c0 = n0 + 32 * cc;
+    if (!row_ok || c0 >= p.N) continue;
+    const bool full = (c0 + 32 <= p.N) && p.vec_ok;
+    if (p.out == 2) {  // raw int32 accumulators (INT4 only)
+      int32_t* dst = reinterpret_cast<int32_t*>(p.y) + (int64_t)row * p.ldy + c0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<int4*>(dst + j) = make_int4((int)r[j] >> 8, (int)r[j + 1] >> 8, (int)r[j + 2] >> 8,
+                                                        (int)r[j + 3] >> 8);
+      } else {
+        for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = (int)r[j] >> 8;
+      }
+      continue;
+    }
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float a;
+      if (ACC_KIND == 0)
+        a = (float)((int)r[j] >> 8);
+      else
+        a = __uint_as_float(r[j]);
+      v[j] = a * rowscale;
+    }
+    if (ACC_KIND == 0) {
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 s = *reinterpret_cast<const float4*>(colscale + c0 + j);
+          v[j] *= s.x;
+          v[j + 1] *= s.y;
+          v[j + 2] *= s.z;
+          v[j + 3] *= s.w;
+        }
+      } else {
+        for (int j = 0; j < 32; ++j) v[j] *= (c0 + j < p.N) ? colscale[c0 + j] : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= gscale;
+    }
+    if (p.out == 0) {
+      float* dst = reinterpret_cast<float*>(p.y) + (int64_t)row * p.ldy + c0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      } else {
+        for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = v[j];
+      }
+    } else {
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + (int64_t)row * p.ldy + c0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 w;
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(v[j], v[j + 1]);
+          __nv_bfloat162 b1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
+          __nv_bfloat162 b3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
+          w.x = *reinterpret_cast<uint32_t*>(&b0);
+          w.y = *reinterpret_cast<uint32_t*>(&b1);
+          w.z = *reinterpret_cast<uint32_t*>(&b2);
+          w.w = *reinterpret_cast<uint32_t*>(&b3);
+          *reinterpret_cast<uint4*>(dst + j) = w;
+        }
+      } else {
+        for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// INT4 x INT4 -> int32 (kind::i8)
+// ---------------------------------------------------------------------------
+constexpr int kI4BK = 128;                 // K elements per k-tile (64 packed bytes per row)
+constexpr int kI4Stg = 4;                  // packed staging stages
+constexpr int kI4Ops = 2;                  // widened operand stages
+constexpr int kI4StgA = kBM * 64, kI4StgB = kBN * 64;
+constexpr int kI4OpA = kBM * 128, kI4OpB = kBN * 128;
+constexpr size_t kI4Smem = 1024 + (size_t)kI4Stg * (kI4StgA + kI4StgB) + (size_t)kI4Ops * (kI4OpA + kI4OpB) + 256;
+
+// Widen 16 packed bytes (32 INT4 codes, element 2i in the low nibble) to 32
+// bytes of int8 holding 16*q.
+__device__ __forceinline__ void widen16(const uint4 in, uint4& o0, uint4& o1) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t lo = (w[i] << 4) & 0xF0F0F0F0u;  // elements 0,2,4,6 (x16)
+    const uint32_t hi = w[i] & 0xF0F0F0F0u;         // elements 1,3,5,7 (x16)
+    o[2 * i] = __byte_perm(lo, hi, 0x5140);
+    o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);
+  }
+  o0 = make_uint4(o[0], o[1], o[2], o[3]);
+  o1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Convert one packed row (64 B, 64B-swizzled staging) into a 128B-swizzled int8 row.
+__device__ __forceinline__ void convert_row(const uint8_t* stg, uint8_t* op, int r) {
+  const int sw_in = (r >> 1) & 3;
+  const int sw_out = r & 7;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (j ^ sw_in));
+    uint4 o0, o1;
+    widen16(in, o0, o1);
+    *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j) ^ sw_out)) = o0;
+    *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j + 1) ^ sw_out)) = o1;
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_int4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                     const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* op = base;                                            // [kI4Ops][A 16K | B 32K]
+  uint8_t* stg = op + (size_t)kI4Ops * (kI4OpA + kI4OpB);        // [kI4Stg][A 8K | B 16K]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (size_t)kI4Stg * (kI4StgA + kI4StgB));
+  uint64_t* stg_full = bars;
+  uint64_t* stg_empty = stg_full + kI4Stg;
+  uint64_t* op_full = stg_empty + kI4Stg;
+  uint64_t* op_empty = op_full + kI4Ops;
+  uint64_t* acc_full = op_empty + kI4Ops;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KT = p.K / kI4BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kI4Stg; ++i) {
+      mbar_init(&stg_full[i], 1);
+      mbar_init(&stg_empty[i], 4);
+    }
+    for (int i = 0; i < kI4Ops; ++i) {
+      mbar_init(&op_full[i], 4);
+      mbar_init(&op_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      unsigned ph = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&stg_empty[s], ph ^ 1, abort_flag)) goto done;
+          uint8_t* sa = stg + (size_t)s * (kI4StgA + kI4StgB);
+          mbar_arrive_expect_tx(&stg_full[s], kI4StgA + kI4StgB);
+          tma_load_2d(sa, &tmap_x, kt * 64, m0, &stg_full[s]);
+          tma_load_2d(sa + kI4StgA, &tmap_w, kt * 64, n0, &stg_full[s]);
+          if (++s == kI4Stg) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_i8(kBM, kBN);
+      int o = 0;
+      unsigned oph = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const unsigned aph = (unsigned)((it >> 1) & 1);
+        if (!wait_or_fail(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(ab * kBN);
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&op_full[o], oph, abort_flag)) goto done;
+          tc_fence_after();
+          const uint8_t* a = op + (size_t)o * (kI4OpA + kI4OpB);
+          const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kI4OpA);
+#pragma unroll
+          for (int j = 0; j < kI4BK / 32; ++j)
+            mma_i8(d, ad + 2 * j, bd + 2 * j, idesc, (kt | j) != 0);
+          tc_commit(&op_empty[o]);
+          if (++o == kI4Ops) { o = 0; oph ^= 1; }
+        }
+        tc_commit(&acc_full[ab]);
+      }
+    }
+  } else if (warp < 6) {
+    // converters: thread t widens A row t and B rows t, t+128 of each k-tile
+    const int t = threadIdx.x - 64;
+    int s = 0, o = 0;
+    unsigned ph = 0, oph = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!wait_or_fail(&stg_full[s], ph, abort_flag)) goto done;
+        if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
+        const uint8_t* sa = stg + (size_t)s * (kI4StgA + kI4StgB);
+        uint8_t* oa = op + (size_t)o * (kI4OpA + kI4OpB);
+        convert_row(sa, oa, t);
+        convert_row(sa + kI4StgA, oa + kI4OpA, t);
+        convert_row(sa + kI4StgA, oa + kI4OpA, t + 128);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&op_full[o]);
+          mbar_arrive(&stg_empty[s]);
+        }
+        if (++s == kI4Stg) { s = 0; ph ^= 1; }
+        if (++o == kI4Ops) { o = 0; oph ^= 1; }
+      }
+    }
+  } else {
+    // epilogue
+    const int q = warp & 3;
+    const float* xs = static_cast<const float*>(p.xscale);
+    const float* ws = static_cast<const float*>(p.wscale);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+      const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
+      const int ab = it & 1;
+      const unsigned aph = (unsigned)((it >> 1) & 1);
+      if (!wait_or_fail(&acc_full[ab], aph, abort_flag)) goto done;
+      tc_fence_after();
+      const int row = m0 + 32 * q + lane;
+      const float sx = (row < p.M) ? xs[row] : 0.f;
+      epilogue_store<0>(p, tmem + (uint32_t)(ab * kBN), m0, n0, q, lane, sx, ws, 1.0f);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 x NVFP4 -> fp32 (kind::mxf4nvf4, block16 E4M3 scales)
+// ---------------------------------------------------------------------------
+constexpr int kF4BK = 256;                 // K elements per k-tile (128 packed bytes per row)
+constexpr int kF4St = 4;
+constexpr int kF4OpA = kBM * 128, kF4OpB = kBN * 128;
+constexpr size_t kF4Smem = 1024 + (size_t)kF4St * (kF4OpA + kF4OpB) + 256;
+constexpr uint32_t kF4SfCol0 = 256;        // TMEM columns [256, 256 + 48*stages) hold the scales
+constexpr uint32_t kF4SfCols = 48;         // per stage: SFA 16 columns, SFB 32 columns
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                      const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* op = base;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(op + (size_t)kF4St * (kF4OpA + kF4OpB));
+  uint64_t* op_full = bars;
+  uint64_t* op_empty = op_full + kF4St;
+  uint64_t* sf_full = op_empty + kF4St;
+  uint64_t* acc_full = sf_full + kF4St;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KT = p.K / kF4BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kF4St; ++i) {
+      mbar_init(&op_full[i], 1);
+      mbar_init(&op_empty[i], 1);
+      mbar_init(&sf_full[i], 4);
+    }
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_empty[0], 4);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      unsigned ph = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&op_empty[s], ph ^ 1, abort_flag)) goto done;
+          uint8_t* sa = op + (size_t)s * (kF4OpA + kF4OpB);
+          mbar_arrive_expect_tx(&op_full[s], kF4OpA + kF4OpB);
+          tma_load_2d(sa, &tmap_x, kt * 128, m0, &op_full[s]);
+          tma_load_2d(sa + kF4OpA, &tmap_w, kt * 128, n0, &op_full[s]);
+          if (++s == kF4St) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_nvf4(kBM, kBN);
+      int s = 0;
+      unsigned ph = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+        if (!wait_or_fail(&acc_empty[0], (unsigned)(it & 1) ^ 1, abort_flag)) goto done;
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&op_full[s], ph, abort_flag)) goto done;
+          if (!wait_or_fail(&sf_full[s], ph, abort_flag)) goto done;
+          tc_fence_after();
+          const uint8_t* a = op + (size_t)s * (kF4OpA + kF4OpB);
+          const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kF4OpA);
+          const uint32_t sf = tmem + kF4SfCol0 + (uint32_t)s * kF4SfCols;
+#pragma unroll
+          for (int j = 0; j < kF4BK / 64; ++j)
+            mma_nvf4(tmem, ad + 2 * j, bd + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (kt | j) != 0);
+          tc_commit(&op_empty[s]);
+          if (++s == kF4St) { s = 0; ph ^= 1; }
+        }
+        tc_commit(&acc_full[0]);
+      }
+    }
+  } else if (warp < 6) {
+    // scale loaders: warp covers TMEM lane quadrant q; lane = row within the quadrant
+    const int q = warp & 3;
+    const uint8_t* sxa = static_cast<const uint8_t*>(p.xscale);
+    const uint8_t* swa = static_cast<const uint8_t*>(p.wscale);
+    const int64_t sld = p.K / 16;
+    int s = 0;
+    unsigned ph = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
+      for (int kt = 0; kt < KT; ++kt) {
+        uint4 ua[4], ub[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = m0 + lane + 32 * i;
+          ua[i] = r < p.M ? *reinterpret_cast<const uint4*>(sxa + (int64_t)r * sld + kt * 16) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = n0 + lane + 32 * i;
+          ub[i] = r < p.N ? *reinterpret_cast<const uint4*>(swa + (int64_t)r * sld + kt * 16) : make_uint4(0, 0, 0, 0);
+        }
+        if (!wait_or_fail(&op_empty[s], ph ^ 1, abort_flag)) goto done;
+        tc_fence_after();
+        uint32_t da[16], db0[16], db1[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&ua[i]);
+            da[4 * j + i] = w[j];
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&ub[i]);
+            const int c = 8 * j + i;
+            if (c < 16)
+              db0[c] = w[j];
+            else
+              db1[c - 16] = w[j];
+          }
+        }
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + kF4SfCol0 + (uint32_t)s * kF4SfCols;
+        tmem_st16(tq, da);
+        tmem_st16(tq + 16, db0);
+        tmem_st16(tq + 32, db1);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[s]);
+        if (++s == kF4St) { s = 0; ph ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const float g = (*p.xg) * (*p.wg);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+      const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
+      if (!wait_or_fail(&acc_full[0], (unsigned)(it & 1), abort_flag)) goto done;
+      tc_fence_after();
+      epilogue_store<1>(p, tmem, m0, n0, q, lane, 1.0f, nullptr, g);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[0]);
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows, cols] (row pitch = cols bytes), box [box_rows, box_cols].
+inline bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                         uint32_t box_cols, CUtensorMapSwizzle sw) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int gemm_num_sms() {
+  int dev = 0, v = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+  return v > 0 ? v : 148;
+}
+
+inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* xg, const uint8_t* wc, const void* ws,
+                               const float* wg, int64_t M, int64_t N, int64_t K, rq_format fmt, void* Y, int64_t ldy,
+                               rq_out out, cudaStream_t st) {
+  if (M < 0 || N < 0 || K <= 0 || ldy < N) return RQ_ERR_INVALID_ARG;
+  if (fmt != RQ_INT4 && fmt != RQ_NVFP4) return RQ_ERR_INVALID_ARG;
+  if (out != RQ_OUT_F32 && out != RQ_OUT_BF16 && out != RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
+  if (fmt == RQ_NVFP4 && out == RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
+  if (M > 0 && N > 0) {
+    if (!xc || !xs || !wc || !ws || !Y) return RQ_ERR_INVALID_ARG;
+    if (fmt == RQ_NVFP4 && (!xg || !wg)) return RQ_ERR_INVALID_ARG;
+  }
+  if (K > 65536 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt == RQ_INT4 && K % kI4BK != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt == RQ_NVFP4 && K % kF4BK != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return RQ_OK;
+  const size_t esz = out == RQ_OUT_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(xc) | reinterpret_cast<uintptr_t>(wc)) & 15) return RQ_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(Y) % esz != 0) return RQ_ERR_ALIGNMENT;
+  if (fmt == RQ_INT4 && ((reinterpret_cast<uintptr_t>(xs) & 3) || (reinterpret_cast<uintptr_t>(ws) & 15)))
+    return RQ_ERR_ALIGNMENT;
+  if (fmt == RQ_NVFP4 && ((reinterpret_cast<uintptr_t>(xs) | reinterpret_cast<uintptr_t>(ws)) & 15))
+    return RQ_ERR_ALIGNMENT;
+
+  GemmParams p;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.xscale = xs;
+  p.wscale = ws;
+  p.xg = xg;
+  p.wg = wg;
+  p.y = Y;
+  p.ldy = ldy;
+  p.out = (int)out;
+  p.vec_ok = ((reinterpret_cast<uintptr_t>(Y) % 16) == 0 && (ldy * (int64_t)esz) % 16 == 0) ? 1 : 0;
+  p.tiles_m = (int)((M + kBM - 1) / kBM);
+  p.tiles_n = (int)((N + kBN - 1) / kBN);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  const int grid = p.num_tiles < gemm_num_sms() ? p.num_tiles : gemm_num_sms();
+
+  CUtensorMap tx, tw;
+  if (fmt == RQ_INT4) {
+    if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+      return RQ_ERR_CUDA;
+    static bool attr_done = false;
+    if (!attr_done) {
+      if (cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem) !=
+          cudaSuccess)
+        return RQ_ERR_CUDA;
+      attr_done = true;
+    }
+    gemm_int4_kernel<<<grid, kGemmThreads, kI4Smem, st>>>(tx, tw, p);
+  } else {
+    if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return RQ_ERR_CUDA;
+    static bool attr_done = false;
+    if (!attr_done) {
+      if (cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kF4Smem) !=
+          cudaSuccess)
+        return RQ_ERR_CUDA;
+      attr_done = true;
+    }
+    gemm_nvfp4_kernel<<<grid, kGemmThreads, kF4Smem, st>>>(tx, tw, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+}  // namespace rq

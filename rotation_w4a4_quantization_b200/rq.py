@@ -1,0 +1,185 @@
+"""Thin Python binding of librq (include/rq.h): argument marshalling only.
+
+Every computation runs in the CUDA kernels of librq.so; this module only
+allocates output tensors with PyTorch, passes raw device pointers, sizes and
+the current CUDA stream, and turns status codes into exceptions.  There is no
+CPU fallback: if librq.so is missing or fails to load, importing this module
+raises.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librq.so")
+
+RQ_INT4, RQ_NVFP4 = 0, 1
+RQ_OUT_F32, RQ_OUT_BF16, RQ_OUT_I32_ACC = 0, 1, 2
+RQ_SCALE_DYNAMIC, RQ_SCALE_STATIC = 0, 1
+STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3: "RQ_ERR_ALIGNMENT",
+          4: "RQ_ERR_UNSUPPORTED_DEVICE", 5: "RQ_ERR_CUDA", 6: "RQ_ERR_TIMEOUT"}
+EXPORTED = ["rq_init", "rq_status_string", "rq_workspace_bytes", "rq_rotate_quantize", "rq_prepare_weights",
+            "rq_w4a4_gemm", "rq_kv_rotate_quantize", "rq_rotate_f32", "rq_get_device_error"]
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("librq.so not built: run `python -m rotation_w4a4_quantization_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i = ctypes.c_int
+lib.rq_init.argtypes = [_i]
+lib.rq_init.restype = _i
+lib.rq_status_string.argtypes = [_i]
+lib.rq_status_string.restype = ctypes.c_char_p
+lib.rq_workspace_bytes.argtypes = [_i]
+lib.rq_workspace_bytes.restype = ctypes.c_size_t
+lib.rq_rotate_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _i, _i, _i, _p, _p, _p, _p, _p]
+lib.rq_rotate_quantize.restype = _i
+lib.rq_prepare_weights.argtypes = [_p, _i64, _i64, _i64, _p, _i, _i, _p, _p, _p, _p, _p]
+lib.rq_prepare_weights.restype = _i
+lib.rq_w4a4_gemm.argtypes = [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i, _p, _i64, _i, _p]
+lib.rq_w4a4_gemm.restype = _i
+lib.rq_kv_rotate_quantize.argtypes = [_p, _i64, _i64, _i64, _i64, ctypes.POINTER(_i64), _p, _p, _p, _p, _p]
+lib.rq_kv_rotate_quantize.restype = _i
+lib.rq_rotate_f32.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i64, _p]
+lib.rq_rotate_f32.restype = _i
+lib.rq_get_device_error.argtypes = [_p]
+lib.rq_get_device_error.restype = _i
+
+
+class RQError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        msg = lib.rq_status_string(status).decode()
+        super().__init__("%s failed: %s (%s)" % (what, STATUS.get(status, status), msg))
+
+
+def _check(status, what):
+    if status != 0:
+        raise RQError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t=None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _fmt(fmt):
+    return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4}[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def init(device=0):
+    _check(lib.rq_init(int(device)), "rq_init")
+
+
+def workspace_bytes(fmt):
+    return int(lib.rq_workspace_bytes(_fmt(fmt)))
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("librq takes CUDA tensors only")
+
+
+def _alloc_quant_outputs(rows, k, fmt, device):
+    codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=device)
+    if fmt == RQ_INT4:
+        scales = torch.empty((rows,), dtype=torch.float32, device=device)
+    else:
+        scales = torch.empty((rows, k // 16), dtype=torch.uint8, device=device)
+    return codes, scales
+
+
+def rotate_quantize(x, signs, block=128, fmt="int4", gmode="dynamic", gscale=None, out=None, workspace=None):
+    """X [M, K] bf16 (row stride ldx) -> (codes, scales, gscale).
+
+    INT4: codes uint8 [M, K/2], scales fp32 [M], gscale None.
+    NVFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/16] (E4M3), gscale fp32 [1].
+    """
+    _require_cuda(x, signs)
+    f = _fmt(fmt)
+    m, k = x.shape
+    codes, scales = out if out is not None else _alloc_quant_outputs(m, k, f, x.device)
+    gm = RQ_SCALE_DYNAMIC if gmode == "dynamic" else RQ_SCALE_STATIC
+    if f == RQ_NVFP4:
+        if gscale is None:
+            gscale = torch.empty((1,), dtype=torch.float32, device=x.device)
+        if workspace is None and gm == RQ_SCALE_DYNAMIC:
+            workspace = torch.empty((16,), dtype=torch.uint8, device=x.device)
+    _check(lib.rq_rotate_quantize(_ptr(x), m, k, x.stride(0), _ptr(signs), int(block), f, gm, _ptr(codes),
+                                  _ptr(scales), _ptr(gscale), _ptr(workspace), _stream(x)), "rq_rotate_quantize")
+    return codes, scales, gscale
+
+
+def prepare_weights(w, signs, block=128, fmt="int4", out=None, workspace=None):
+    """W [N, K] bf16 -> (codes, scales, gscale), the offline weight side."""
+    _require_cuda(w, signs)
+    f = _fmt(fmt)
+    n, k = w.shape
+    codes, scales = out if out is not None else _alloc_quant_outputs(n, k, f, w.device)
+    gscale = torch.empty((1,), dtype=torch.float32, device=w.device) if f == RQ_NVFP4 else None
+    if f == RQ_NVFP4 and workspace is None:
+        workspace = torch.empty((16,), dtype=torch.uint8, device=w.device)
+    _check(lib.rq_prepare_weights(_ptr(w), n, k, w.stride(0), _ptr(signs), int(block), f, _ptr(codes), _ptr(scales),
+                                  _ptr(gscale), _ptr(workspace), _stream(w)), "rq_prepare_weights")
+    return codes, scales, gscale
+
+
+def w4a4_gemm(xq, wq, fmt="int4", out="f32", y=None):
+    """Y = deq(xq) . deq(wq)^T with xq / wq the (codes, scales, gscale) triples."""
+    xc, xs, xg = xq
+    wc, ws, wg = wq
+    _require_cuda(xc, xs, wc, ws)
+    f = _fmt(fmt)
+    o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16, "i32": RQ_OUT_I32_ACC}[out]
+    m, kh = xc.shape
+    n = wc.shape[0]
+    if y is None:
+        dt = {RQ_OUT_F32: torch.float32, RQ_OUT_BF16: torch.bfloat16, RQ_OUT_I32_ACC: torch.int32}[o]
+        y = torch.empty((m, n), dtype=dt, device=xc.device)
+    _check(lib.rq_w4a4_gemm(_ptr(xc), _ptr(xs), _ptr(xg), _ptr(wc), _ptr(ws), _ptr(wg), m, n, 2 * kh, f, _ptr(y),
+                            y.stride(0), o, _stream(xc)), "rq_w4a4_gemm")
+    return y
+
+
+def kv_rotate_quantize(kv, signs, out=None):
+    """K or V [B, H, S, 128] bf16 (head_dim contiguous) -> (codes [B,H,S,64], scale fp16 [B,H,S], zero fp16 [B,H,S])."""
+    _require_cuda(kv, signs)
+    b, h, s, d = kv.shape
+    if kv.stride(3) != 1:
+        raise ValueError("head_dim must be contiguous")
+    if out is None:
+        codes = torch.empty((b, h, s, d // 2), dtype=torch.uint8, device=kv.device)
+        scale = torch.empty((b, h, s), dtype=torch.float16, device=kv.device)
+        zero = torch.empty((b, h, s), dtype=torch.float16, device=kv.device)
+    else:
+        codes, scale, zero = out
+    strides = (ctypes.c_int64 * 3)(kv.stride(0), kv.stride(1), kv.stride(2))
+    _check(lib.rq_kv_rotate_quantize(_ptr(kv), b, h, s, d, strides, _ptr(signs), _ptr(codes), _ptr(scale),
+                                     _ptr(zero), _stream(kv)), "rq_kv_rotate_quantize")
+    return codes, scale, zero
+
+
+def rotate_f32(x, signs, block=128, out=None):
+    """X.Q as fp32 [M, K]."""
+    _require_cuda(x, signs)
+    m, k = x.shape
+    if out is None:
+        out = torch.empty((m, k), dtype=torch.float32, device=x.device)
+    _check(lib.rq_rotate_f32(_ptr(x), m, k, x.stride(0), _ptr(signs), int(block), _ptr(out), out.stride(0),
+                             _stream(x)), "rq_rotate_f32")
+    return out
+
+
+def get_device_error(stream=None):
+    """Synchronize the stream and raise if a kernel recorded a device-side timeout."""
+    s = ctypes.c_void_p(stream) if stream is not None else _stream()
+    _check(lib.rq_get_device_error(s), "rq_get_device_error")

@@ -1,0 +1,127 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every entry
+point that include/rq.h declares, and rejects bad arguments on the host with
+the documented status -- before any CUDA call, so no GPU is needed.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+rq = pytest.importorskip("rotation_w4a4_quantization_b200.rq")
+lib = rq.lib
+
+INVALID, SHAPE, ALIGN = 1, 2, 3
+P = ctypes.c_void_p
+A16 = P(0x10000)      # a 16-byte aligned fake device address (never dereferenced)
+A8 = P(0x10008)
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "rq.h")) as f:
+        text = f.read()
+    return re.findall(r"RQ_API\s+[\w\s\*]+?\b(rq_\w+)\s*\(", text)
+
+
+def test_header_matches_exports():
+    names = declared_functions()
+    assert sorted(names) == sorted(rq.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in range(7):
+        assert lib.rq_status_string(s)
+    assert lib.rq_status_string(99) == b"unknown status"
+
+
+def test_workspace_bytes():
+    assert lib.rq_workspace_bytes(rq.RQ_INT4) == 0
+    assert lib.rq_workspace_bytes(rq.RQ_NVFP4) == 16
+
+
+def rotq(x=A16, m=4, k=512, ldx=512, signs=A16, block=128, fmt=0, gmode=0, codes=A16, scales=A16, g=A16, ws=A16):
+    return lib.rq_rotate_quantize(x, m, k, ldx, signs, block, fmt, gmode, codes, scales, g, ws, None)
+
+
+def test_rotate_quantize_rejections():
+    assert rotq(x=None) == INVALID
+    assert rotq(signs=None) == INVALID
+    assert rotq(codes=None) == INVALID
+    assert rotq(m=-1) == INVALID
+    assert rotq(ldx=100) == INVALID                 # ldx < K
+    assert rotq(k=500, ldx=500) == SHAPE            # K not a multiple of 128
+    assert rotq(k=65536, ldx=65536) == SHAPE        # above the supported K
+    assert rotq(block=64) == SHAPE
+    assert rotq(k=384, ldx=384, block=0) == SHAPE   # full width needs a power of two
+    assert rotq(k=8192, ldx=8192, block=0) == SHAPE
+    assert rotq(x=P(0x10002)) == ALIGN
+    assert rotq(ldx=516) == ALIGN                   # row pitch not a multiple of 16 bytes
+    assert rotq(codes=A8) == ALIGN
+    assert rotq(fmt=7) == INVALID
+    assert rotq(gmode=5) == INVALID
+    assert rotq(fmt=1, block=0) == SHAPE            # NVFP4 needs 128-wide blocks
+    assert rotq(fmt=1, g=None) == INVALID
+    assert rotq(fmt=1, ws=None) == INVALID          # dynamic NVFP4 needs the workspace
+    assert rotq(fmt=1, scales=P(0x10004)) == ALIGN
+
+
+def test_rotate_quantize_empty_is_noop():
+    assert rotq(m=0) == 0
+
+
+def test_prepare_weights_and_rotate_f32_rejections():
+    assert lib.rq_prepare_weights(None, 4, 512, 512, A16, 128, 0, A16, A16, A16, A16, None) == INVALID
+    assert lib.rq_prepare_weights(A16, 4, 500, 500, A16, 128, 0, A16, A16, A16, A16, None) == SHAPE
+    assert lib.rq_rotate_f32(A16, 4, 512, 512, A16, 128, None, 512, None) == INVALID
+    assert lib.rq_rotate_f32(A16, 4, 512, 512, A16, 128, A16, 510, None) == INVALID   # ldo < K
+    assert lib.rq_rotate_f32(A16, 4, 512, 512, A16, 128, A16, 514, None) == ALIGN
+    assert lib.rq_rotate_f32(A16, 0, 512, 512, A16, 128, A16, 512, None) == 0
+
+
+def gemm(xc=A16, xs=A16, xg=A16, wc=A16, ws=A16, wg=A16, m=128, n=256, k=512, fmt=0, y=A16, ldy=256, out=0):
+    return lib.rq_w4a4_gemm(xc, xs, xg, wc, ws, wg, m, n, k, fmt, y, ldy, out, None)
+
+
+def test_gemm_rejections():
+    assert gemm(xc=None) == INVALID
+    assert gemm(y=None) == INVALID
+    assert gemm(m=-1) == INVALID
+    assert gemm(ldy=100) == INVALID
+    assert gemm(fmt=3) == INVALID
+    assert gemm(out=9) == INVALID
+    assert gemm(fmt=1, out=2) == INVALID           # raw accumulators are INT4 only
+    assert gemm(fmt=1, xg=None) == INVALID
+    assert gemm(k=192) == SHAPE                    # INT4 K multiple of 128
+    assert gemm(fmt=1, k=384) == SHAPE             # NVFP4 K multiple of 256
+    assert gemm(k=131072) == SHAPE
+    assert gemm(xc=A8) == ALIGN
+    assert gemm(y=P(0x10002)) == ALIGN             # fp32 Y must be 4-byte aligned
+    assert gemm(m=0) == 0 and gemm(n=0) == 0
+
+
+def kv(x=A16, b=2, h=2, s=8, d=128, strides=(4096, 1024, 128), signs=A16, codes=A16, sc=A16, zr=A16):
+    arr = None if strides is None else (ctypes.c_int64 * 3)(*strides)
+    return lib.rq_kv_rotate_quantize(x, b, h, s, d, arr, signs, codes, sc, zr, None)
+
+
+def test_kv_rejections():
+    assert kv(x=None) == INVALID
+    assert kv(strides=None) == INVALID
+    assert kv(b=-1) == INVALID
+    assert kv(d=64) == SHAPE
+    assert kv(strides=(4096, 1024, 130)) == ALIGN  # vectors must stay 16-byte aligned
+    assert kv(sc=P(0x10001)) == ALIGN
+    assert kv(strides=(4096, -1, 128)) == INVALID
+    assert kv(s=0) == 0
+
+
+def test_init_without_gpu_reports_unsupported_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lib.rq_init(0) == 4
