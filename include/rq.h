@@ -94,8 +94,8 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *  X_dev      bf16 [M, ldx]; rows 16-byte aligned (X_dev and ldx*2 multiples of 16).
  *  M          rows (tokens), >= 0.  M = 0 is a no-op.
  *  K          channels; a multiple of 128, at most 32768.
- *  signs_dev  int8 [K], each +1 or -1 (the random sign diagonal; any other value
- *             is read as +1 if positive and -1 otherwise).
+ *  signs_dev  int8 [K], 16-byte aligned, each +1 or -1 (the random sign diagonal;
+ *             any other value is read as -1 if negative and +1 otherwise).
  *  block      128 for 128-wide blocks, or 0 for a full-width rotation (then K
  *             must be a power of two in [256, 4096]; INT4 only).
  *  fmt        RQ_INT4:
@@ -159,7 +159,7 @@ RQ_API rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev
  *  KV_dev      bf16, element (b,h,t,d) at KV_dev + b*strides_host[0] + h*strides_host[1]
  *              + t*strides_host[2] + d (strides in elements; d contiguous; each
  *              vector 16-byte aligned).
- *  signs_dev   int8 [D].
+ *  signs_dev   int8 [D], 16-byte aligned.
  *  codes_dev   uint8 [B, H, S, D/2] contiguous, 16-byte aligned.
  *  scale_dev, zero_dev  fp16 [B, H, S] contiguous.
  */

@@ -63,72 +63,68 @@ bool ensure_smem(const void* kernel) {
 
 rq_status last_launch_status() { return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
 
+// Geometry of the rotate kernel: warps per group G, rows per stage RPS,
+// groups per CTA GPC and ring depth, for a block-diagonal (full = false) or
+// full-width rotation of K channels.
 struct RotCfg {
-  int R, stages, threads;
+  int G, RPS, GPC, stages, threads;
   size_t smem;
 };
 
-RotCfg block_config(int64_t K) {
+RotCfg rotate_config(int64_t K, bool full, int mode) {
   const int nb = (int)(K / 128);
   RotCfg c;
-  c.R = (256 % nb == 0) ? 256 / nb : (nb <= 384 ? 384 / nb : 1);
-  if (c.R < 1) c.R = 1;
-  c.threads = c.R * nb;
-  const size_t sb = RotSmemLayout::stage_bytes(c.R, (int)K);
-  const size_t fixed = RotSmemLayout::total(c.R, (int)K, 0);
-  int st = (int)((kSmemBudget - fixed) / sb);
-  c.stages = st > 4 ? 4 : st;
-  c.smem = RotSmemLayout::total(c.R, (int)K, c.stages);
+  if (32 % nb == 0) {
+    c.G = 1;
+    c.RPS = 32 / nb;
+  } else {
+    c.G = (nb + 31) / 32;
+    c.RPS = 1;
+  }
+  const int warps = (!full && mode == kModeInt4) ? 12 : 8;  // must match the kernel's launch bounds
+  c.GPC = warps / c.G > 0 ? warps / c.G : 1;
+  for (;;) {
+    const size_t sb = RotSmemLayout::stage_bytes(c.RPS, (int)K);
+    const size_t fixed = RotSmemLayout::total(c.RPS, (int)K, 0, c.GPC, c.G) + (size_t)c.GPC * 4 * 8;
+    const int st = (int)((kSmemBudget - fixed) / (sb * c.GPC));
+    c.stages = st > 4 ? 4 : st;
+    if (c.stages >= 2 || c.GPC == 1) break;
+    --c.GPC;
+  }
+  c.threads = 32 * c.G * c.GPC;
+  c.smem = RotSmemLayout::total(c.RPS, (int)K, c.stages, c.GPC, c.G);
   return c;
 }
 
-RotCfg full_config(int64_t K) {
-  const int NB = (int)(K / 128);
-  RotCfg c;
-  c.R = 256 / NB;
-  c.threads = 256;
-  const size_t sb = RotSmemLayout::stage_bytes(c.R, (int)K);
-  const size_t fixed = RotSmemLayout::total(c.R, (int)K, 0);
-  int st = (int)((kSmemBudget - fixed) / sb);
-  c.stages = st > 3 ? 3 : st;
-  c.smem = RotSmemLayout::total(c.R, (int)K, c.stages);
-  return c;
+template <int MODE, int NBF>
+rq_status launch_rotate(RotParams p, cudaStream_t st) {
+  const RotCfg c = rotate_config(p.K, NBF != 0, MODE);
+  if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
+  p.G = c.G;
+  p.RPS = c.RPS;
+  p.GPC = c.GPC;
+  p.stages = c.stages;
+  p.num_tiles = (p.rows + c.RPS - 1) / c.RPS;
+  const int64_t ctas = (p.num_tiles + c.GPC - 1) / c.GPC;
+  const int64_t grid = ctas < num_sms_of_current_device() ? ctas : num_sms_of_current_device();
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_kernel<MODE, NBF>))) return RQ_ERR_CUDA;
+  rotate_kernel<MODE, NBF><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
+  return last_launch_status();
 }
 
 template <int MODE>
 rq_status launch_block(RotParams p, cudaStream_t st) {
-  const RotCfg c = block_config(p.K);
-  if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
-  p.R = c.R;
-  p.stages = c.stages;
-  p.num_tiles = (p.rows + c.R - 1) / c.R;
-  const int64_t grid = p.num_tiles < num_sms_of_current_device() ? p.num_tiles : num_sms_of_current_device();
-  if (!ensure_smem(reinterpret_cast<const void*>(rotate_block_kernel<MODE>))) return RQ_ERR_CUDA;
-  rotate_block_kernel<MODE><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
-  return last_launch_status();
-}
-
-template <int MODE, int NB>
-rq_status launch_full_nb(RotParams p, cudaStream_t st) {
-  const RotCfg c = full_config(p.K);
-  if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
-  p.R = c.R;
-  p.stages = c.stages;
-  p.num_tiles = (p.rows + c.R - 1) / c.R;
-  const int64_t grid = p.num_tiles < num_sms_of_current_device() ? p.num_tiles : num_sms_of_current_device();
-  if (!ensure_smem(reinterpret_cast<const void*>(rotate_full_kernel<MODE, NB>))) return RQ_ERR_CUDA;
-  rotate_full_kernel<MODE, NB><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
-  return last_launch_status();
+  return launch_rotate<MODE, 0>(p, st);
 }
 
 template <int MODE>
 rq_status launch_full(RotParams p, cudaStream_t st) {
   switch (p.nb) {
-    case 2: return launch_full_nb<MODE, 2>(p, st);
-    case 4: return launch_full_nb<MODE, 4>(p, st);
-    case 8: return launch_full_nb<MODE, 8>(p, st);
-    case 16: return launch_full_nb<MODE, 16>(p, st);
-    case 32: return launch_full_nb<MODE, 32>(p, st);
+    case 2: return launch_rotate<MODE, 2>(p, st);
+    case 4: return launch_rotate<MODE, 4>(p, st);
+    case 8: return launch_rotate<MODE, 8>(p, st);
+    case 16: return launch_rotate<MODE, 16>(p, st);
+    case 32: return launch_rotate<MODE, 32>(p, st);
     default: return RQ_ERR_UNSUPPORTED_SHAPE;
   }
 }
@@ -141,7 +137,7 @@ rq_status check_rotation_args(const void* X, int64_t M, int64_t K, int64_t ldx, 
   if (K % 128 != 0 || K > kMaxKBlock) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (block != 0 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (block == 0 && !(is_pow2(K) && K >= 256 && K <= 4096)) return RQ_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned(X, 16) || (ldx * 2) % 16 != 0) return RQ_ERR_ALIGNMENT;
+  if (!aligned(X, 16) || (ldx * 2) % 16 != 0 || !aligned(signs, 16)) return RQ_ERR_ALIGNMENT;
   return RQ_OK;
 }
 
@@ -157,6 +153,7 @@ RotParams matrix_params(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.sS = ldx * 2;
   p.sH = 0;
   p.sB = 0;
+  p.contiguous = (ldx == K) ? 1 : 0;
   p.signs = signs;
   p.cfull = (float)(1.0 / std::sqrt((double)K));
   return p;
@@ -232,7 +229,7 @@ rq_status rq_init(int device) {
   if (cudaGetDevice(&prev) != cudaSuccess) return RQ_ERR_CUDA;
   if (cudaSetDevice(device) != cudaSuccess) return RQ_ERR_CUDA;
   cudaFuncAttributes attr;
-  const cudaError_t e = cudaFuncGetAttributes(&attr, rotate_block_kernel<kModeInt4>);
+  const cudaError_t e = cudaFuncGetAttributes(&attr, rotate_kernel<kModeInt4, 0>);
   (void)cudaSetDevice(prev);
   if (e != cudaSuccess) return RQ_ERR_UNSUPPORTED_DEVICE;
   return RQ_OK;
@@ -279,7 +276,8 @@ rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H, int64_
   if (!KV_dev || !strides_host || !signs_dev || !codes_dev || !scale_dev || !zero_dev) return RQ_ERR_INVALID_ARG;
   for (int i = 0; i < 3; ++i)
     if (strides_host[i] < 0) return RQ_ERR_INVALID_ARG;
-  if (!aligned(KV_dev, 16) || !aligned(codes_dev, 16) || !aligned(scale_dev, 2) || !aligned(zero_dev, 2))
+  if (!aligned(KV_dev, 16) || !aligned(codes_dev, 16) || !aligned(scale_dev, 2) || !aligned(zero_dev, 2) ||
+      !aligned(signs_dev, 16))
     return RQ_ERR_ALIGNMENT;
   for (int i = 0; i < 3; ++i)
     if ((strides_host[i] * 2) % 16 != 0) return RQ_ERR_ALIGNMENT;
@@ -296,6 +294,8 @@ rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H, int64_
   p.sB = strides_host[0] * 2;
   p.sH = strides_host[1] * 2;
   p.sS = strides_host[2] * 2;
+  p.contiguous = (strides_host[2] == 128 && (H == 1 || strides_host[1] == S * 128) &&
+                  (B == 1 || strides_host[0] == H * S * 128)) ? 1 : 0;
   p.signs = signs_dev;
   p.codes = codes_dev;
   p.kv_scale = static_cast<__half*>(scale_dev);

@@ -30,6 +30,8 @@
 
 #include <cuda.h>
 
+#include <cstring>
+
 #include "rq_common.cuh"
 #include "rq_tc.cuh"
 
@@ -49,6 +51,7 @@ struct GemmParams {
   int64_t ldy;
   int out;              // 0 f32, 1 bf16, 2 i32 accumulators
   int vec_ok;           // 1: Y rows allow 16-byte vector stores
+  int tma_store;        // 1: bf16 Y is written by TMA from a shared-memory staging tile
   int tiles_m, tiles_n, num_tiles;
 };
 
@@ -64,16 +67,19 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, unsigned parity, int
 
 // Epilogue for one 32-row x 256-column slab held by this warp's TMEM lanes.
 // acc_kind 0: int32 accumulators of 256*sum (INT4), 1: fp32 (NVFP4).
+// Arrives on `acc_empty` once the slab has been read out of tensor memory.
 template <int ACC_KIND>
 __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tacc, int m0, int n0, int q, int lane,
-                                               float rowscale, const float* colscale, float gscale) {
+                                               float rowscale, const float* colscale, float gscale,
+                                               uint64_t* acc_empty) {
   const int row = m0 + 32 * q + lane;
   const bool row_ok = row < p.M;
+  const uint32_t tq = tacc + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
   for (int cc = 0; cc < kBN / 32; ++cc) {
     uint32_t r[32];
     __syncwarp();
-    tmem_ld32(tacc + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * cc), r);
+    tmem_ld32(tq + (uint32_t)(32 * cc), r);
     tmem_wait_ld();
     const int c0 = n0 + 32 * cc;
     if (!row_ok || c0 >= p.N) continue;
@@ -93,11 +99,7 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      float a;
-      if (ACC_KIND == 0)
-        a = (float)((int)r[j] >> 8);
-      else
-        a = __uint_as_float(r[j]);
+      const float a = (ACC_KIND == 0) ? (float)((int)r[j] >> 8) : __uint_as_float(r[j]);
       v[j] = a * rowscale;
     }
     if (ACC_KIND == 0) {
@@ -121,7 +123,8 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
       float* dst = reinterpret_cast<float*>(p.y) + (int64_t)row * p.ldy + c0;
       if (full) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       } else {
         for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = v[j];
       }
@@ -130,20 +133,72 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
       if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
-          uint4 w;
           __nv_bfloat162 b0 = __floats2bfloat162_rn(v[j], v[j + 1]);
           __nv_bfloat162 b1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
           __nv_bfloat162 b2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
           __nv_bfloat162 b3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
-          w.x = *reinterpret_cast<uint32_t*>(&b0);
-          w.y = *reinterpret_cast<uint32_t*>(&b1);
-          w.z = *reinterpret_cast<uint32_t*>(&b2);
-          w.w = *reinterpret_cast<uint32_t*>(&b3);
-          *reinterpret_cast<uint4*>(dst + j) = w;
+          *reinterpret_cast<uint4*>(dst + j) =
+              make_uint4(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1),
+                         *reinterpret_cast<uint32_t*>(&b2), *reinterpret_cast<uint32_t*>(&b3));
         }
       } else {
         for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
       }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);
+}
+
+// bf16 epilogue through shared memory: the slab is read out of TMEM in two
+// 128-column halves, scaled, rounded to bf16 and written into two 128B-swizzled
+// 64-column boxes; TMEM is released as soon as the last half has been read;
+// one thread stores each half with TMA (which also clips rows >= M, columns >= N).
+// `stage` is the 32 KB staging buffer, `ytmap` the bf16 Y tensor map with
+// 64 x 128 boxes, `epi_tid` 0..127 the thread's index among the epilogue warps.
+__device__ __forceinline__ void epilogue_bf16_tma(const GemmParams& p, const CUtensorMap* ytmap, uint32_t tacc,
+                                                  int m0, int n0, int q, int lane, int epi_tid, float gscale,
+                                                  uint8_t* stage, uint64_t* acc_empty) {
+  const uint32_t tq = tacc + ((uint32_t)(32 * q) << 16);
+  const int row = 32 * q + lane;  // row within the tile
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
+    if (hh == 1 || epi_tid == 0) {
+      // the staging buffer must have been read by the previous TMA store
+      if (epi_tid == 0) bulk_wait_read0();
+    }
+    named_sync(1, 128);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(tq + (uint32_t)(128 * hh + 32 * cc), r);
+      tmem_wait_ld();
+      uint8_t* box = stage + (cc >> 1) * (kBM * 128);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {  // 4 x 16 bytes = 32 bf16 of this chunk
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 8 * k + 2 * e;
+          __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[j]) * gscale, __uint_as_float(r[j + 1]) * gscale);
+          w[e] = *reinterpret_cast<uint32_t*>(&b);
+        }
+        const int c16 = 4 * (cc & 1) + k;  // 16-byte chunk within the 128-byte box row
+        *reinterpret_cast<uint4*>(box + row * 128 + 16 * (c16 ^ (row & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    if (hh == 1) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);  // accumulator free for the next tile's MMAs
+    }
+    fence_proxy_async_smem();
+    named_sync(1, 128);
+    if (epi_tid == 0) {
+      tma_store_2d(ytmap, stage, n0 + 128 * hh, m0);
+      tma_store_2d(ytmap, stage + kBM * 128, n0 + 128 * hh + 64, m0);
+      bulk_commit();
     }
   }
 }
@@ -152,8 +207,10 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
 // INT4 x INT4 -> int32 (kind::i8)
 // ---------------------------------------------------------------------------
 constexpr int kI4BK = 128;                 // K elements per k-tile (64 packed bytes per row)
-constexpr int kI4Stg = 4;                  // packed staging stages
-constexpr int kI4Ops = 2;                  // widened operand stages
+constexpr int kI4Stg = 3;                  // packed staging stages
+constexpr int kI4Ops = 3;                  // widened operand stages
+constexpr int kI4ConvWarps = 8;            // nibble -> int8 converter warps (warps 2..9)
+constexpr int kI4Threads = 32 * (2 + kI4ConvWarps + 4);
 constexpr int kI4StgA = kBM * 64, kI4StgB = kBN * 64;
 constexpr int kI4OpA = kBM * 128, kI4OpB = kBN * 128;
 constexpr size_t kI4Smem = 1024 + (size_t)kI4Stg * (kI4StgA + kI4StgB) + (size_t)kI4Ops * (kI4OpA + kI4OpB) + 256;
@@ -174,21 +231,20 @@ __device__ __forceinline__ void widen16(const uint4 in, uint4& o0, uint4& o1) {
   o1 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Convert one packed row (64 B, 64B-swizzled staging) into a 128B-swizzled int8 row.
-__device__ __forceinline__ void convert_row(const uint8_t* stg, uint8_t* op, int r) {
-  const int sw_in = (r >> 1) & 3;
+// Widen one 16-byte chunk j (32 codes) of packed row r (64B-swizzled staging)
+// into two 16-byte chunks of the 128B-swizzled int8 row.  Jobs are numbered
+// row-major (4 per row), so the 8 threads of a shared-memory phase touch 8
+// distinct bank groups both when reading and when writing.
+__device__ __forceinline__ void convert_chunk(const uint8_t* stg, uint8_t* op, int r, int j) {
+  const uint4 in = *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (j ^ ((r >> 1) & 3)));
+  uint4 o0, o1;
+  widen16(in, o0, o1);
   const int sw_out = r & 7;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 in = *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (j ^ sw_in));
-    uint4 o0, o1;
-    widen16(in, o0, o1);
-    *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j) ^ sw_out)) = o0;
-    *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j + 1) ^ sw_out)) = o1;
-  }
+  *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j) ^ sw_out)) = o0;
+  *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j + 1) ^ sw_out)) = o1;
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -211,10 +267,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kI4Stg; ++i) {
       mbar_init(&stg_full[i], 1);
-      mbar_init(&stg_empty[i], 4);
+      mbar_init(&stg_empty[i], kI4ConvWarps);
     }
     for (int i = 0; i < kI4Ops; ++i) {
-      mbar_init(&op_full[i], 4);
+      mbar_init(&op_full[i], kI4ConvWarps);
       mbar_init(&op_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -277,8 +333,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_commit(&acc_full[ab]);
       }
     }
-  } else if (warp < 6) {
-    // converters: thread t widens A row t and B rows t, t+128 of each k-tile
+  } else if (warp < 2 + kI4ConvWarps) {
+    // converters: (kBM + kBN) rows x 4 chunks per k-tile, split over the converter threads
     const int t = threadIdx.x - 64;
     int s = 0, o = 0;
     unsigned ph = 0, oph = 0;
@@ -288,9 +344,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
         const uint8_t* sa = stg + (size_t)s * (kI4StgA + kI4StgB);
         uint8_t* oa = op + (size_t)o * (kI4OpA + kI4OpB);
-        convert_row(sa, oa, t);
-        convert_row(sa + kI4StgA, oa + kI4OpA, t);
-        convert_row(sa + kI4StgA, oa + kI4OpA, t + 128);
+        constexpr int kJobs = (kBM + kBN) * 4, kConvThreads = 32 * kI4ConvWarps;
+#pragma unroll
+        for (int jb = t; jb < kJobs; jb += kConvThreads) {
+          const int r = jb >> 2, j = jb & 3;
+          if (r < kBM)
+            convert_chunk(sa, oa, r, j);
+          else
+            convert_chunk(sa + kI4StgA, oa + kI4OpA, r - kBM, j);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -315,10 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int row = m0 + 32 * q + lane;
       const float sx = (row < p.M) ? xs[row] : 0.f;
-      epilogue_store<0>(p, tmem + (uint32_t)(ab * kBN), m0, n0, q, lane, sx, ws, 1.0f);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      epilogue_store<0>(p, tmem + (uint32_t)(ab * kBN), m0, n0, q, lane, sx, ws, 1.0f, &acc_empty[ab]);
     }
   }
 done:
@@ -334,19 +393,24 @@ done:
 // NVFP4 x NVFP4 -> fp32 (kind::mxf4nvf4, block16 E4M3 scales)
 // ---------------------------------------------------------------------------
 constexpr int kF4BK = 256;                 // K elements per k-tile (128 packed bytes per row)
-constexpr int kF4St = 4;
+constexpr int kF4St = 3;
 constexpr int kF4OpA = kBM * 128, kF4OpB = kBN * 128;
-constexpr size_t kF4Smem = 1024 + (size_t)kF4St * (kF4OpA + kF4OpB) + 256;
+constexpr int kF4SfA = kBM * 16, kF4SfB = kBN * 16;          // 16 E4M3 scales per row per k-tile
+constexpr int kF4Stage = kF4OpA + kF4OpB + kF4SfA + kF4SfB;
+constexpr int kEpiStage = kBM * 128 * 2;   // bf16 staging: two 64-column boxes of 128 rows (32 KB)
+constexpr size_t kF4Smem = 1024 + (size_t)kF4St * kF4Stage + kEpiStage + 256;
 constexpr uint32_t kF4SfCol0 = 256;        // TMEM columns [256, 256 + 48*stages) hold the scales
 constexpr uint32_t kF4SfCols = 48;         // per stage: SFA 16 columns, SFB 32 columns
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                      const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmap_sx, const __grid_constant__ CUtensorMap tmap_sw,
+                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* op = base;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(op + (size_t)kF4St * (kF4OpA + kF4OpB));
+  uint8_t* epi_stage = op + (size_t)kF4St * kF4Stage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + kEpiStage);
   uint64_t* op_full = bars;
   uint64_t* op_empty = op_full + kF4St;
   uint64_t* sf_full = op_empty + kF4St;
@@ -370,6 +434,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tmap_x);
     prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_sx);
+    prefetch_tmap(&tmap_sw);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -388,10 +454,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
         for (int kt = 0; kt < KT; ++kt) {
           if (!wait_or_fail(&op_empty[s], ph ^ 1, abort_flag)) goto done;
-          uint8_t* sa = op + (size_t)s * (kF4OpA + kF4OpB);
-          mbar_arrive_expect_tx(&op_full[s], kF4OpA + kF4OpB);
+          uint8_t* sa = op + (size_t)s * kF4Stage;
+          mbar_arrive_expect_tx(&op_full[s], kF4Stage);
           tma_load_2d(sa, &tmap_x, kt * 128, m0, &op_full[s]);
           tma_load_2d(sa + kF4OpA, &tmap_w, kt * 128, n0, &op_full[s]);
+          tma_load_2d(sa + kF4OpA + kF4OpB, &tmap_sx, kt * 16, m0, &op_full[s]);
+          tma_load_2d(sa + kF4OpA + kF4OpB + kF4SfA, &tmap_sw, kt * 16, n0, &op_full[s]);
           if (++s == kF4St) { s = 0; ph ^= 1; }
         }
       }
@@ -409,7 +477,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!wait_or_fail(&op_full[s], ph, abort_flag)) goto done;
           if (!wait_or_fail(&sf_full[s], ph, abort_flag)) goto done;
           tc_fence_after();
-          const uint8_t* a = op + (size_t)s * (kF4OpA + kF4OpB);
+          const uint8_t* a = op + (size_t)s * kF4Stage;
           const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kF4OpA);
           const uint32_t sf = tmem + kF4SfCol0 + (uint32_t)s * kF4SfCols;
 #pragma unroll
@@ -422,29 +490,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp < 6) {
-    // scale loaders: warp covers TMEM lane quadrant q; lane = row within the quadrant
+    // scale movers: the stage's scales arrived by TMA with the operands; this
+    // warp copies the rows of its TMEM lane quadrant q into tensor memory.
     const int q = warp & 3;
-    const uint8_t* sxa = static_cast<const uint8_t*>(p.xscale);
-    const uint8_t* swa = static_cast<const uint8_t*>(p.wscale);
-    const int64_t sld = p.K / 16;
     int s = 0;
     unsigned ph = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
       for (int kt = 0; kt < KT; ++kt) {
+        // op_full of this round implies the MMAs of the previous round on this
+        // stage (and so their reads of its scale columns) have completed
+        if (!wait_or_fail(&op_full[s], ph, abort_flag)) goto done;
+        const uint8_t* sfa = op + (size_t)s * kF4Stage + kF4OpA + kF4OpB;
+        const uint8_t* sfb = sfa + kF4SfA;
         uint4 ua[4], ub[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = m0 + lane + 32 * i;
-          ua[i] = r < p.M ? *reinterpret_cast<const uint4*>(sxa + (int64_t)r * sld + kt * 16) : make_uint4(0, 0, 0, 0);
-        }
+        for (int i = 0; i < 4; ++i) ua[i] = *reinterpret_cast<const uint4*>(sfa + (lane + 32 * i) * 16);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = n0 + lane + 32 * i;
-          ub[i] = r < p.N ? *reinterpret_cast<const uint4*>(swa + (int64_t)r * sld + kt * 16) : make_uint4(0, 0, 0, 0);
-        }
-        if (!wait_or_fail(&op_empty[s], ph ^ 1, abort_flag)) goto done;
-        tc_fence_after();
+        for (int i = 0; i < 8; ++i) ub[i] = *reinterpret_cast<const uint4*>(sfb + (lane + 32 * i) * 16);
         uint32_t da[16], db0[16], db1[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -482,13 +544,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
       if (!wait_or_fail(&acc_full[0], (unsigned)(it & 1), abort_flag)) goto done;
       tc_fence_after();
-      epilogue_store<1>(p, tmem, m0, n0, q, lane, 1.0f, nullptr, g);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[0]);
+      if (p.tma_store)
+        epilogue_bf16_tma(p, &tmap_y, tmem, m0, n0, q, lane, threadIdx.x - 192, g, epi_stage, &acc_empty[0]);
+      else
+        epilogue_store<1>(p, tmem, m0, n0, q, lane, 1.0f, nullptr, g, &acc_empty[0]);
     }
   }
 done:
+  if (threadIdx.x == 192) bulk_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -528,6 +591,19 @@ inline bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_
   return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 Y [rows, cols] with row pitch ld elements, 64 x 128 boxes, 128B swizzle.
+inline bool make_tmap_y_bf16(CUtensorMap* m, void* ptr, uint64_t rows, uint64_t cols, uint64_t ld) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kBM};
+  cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 inline int gemm_num_sms() {
@@ -571,6 +647,7 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
   p.ldy = ldy;
   p.out = (int)out;
   p.vec_ok = ((reinterpret_cast<uintptr_t>(Y) % 16) == 0 && (ldy * (int64_t)esz) % 16 == 0) ? 1 : 0;
+  p.tma_store = 0;
   p.tiles_m = (int)((M + kBM - 1) / kBM);
   p.tiles_n = (int)((N + kBN - 1) / kBN);
   p.num_tiles = p.tiles_m * p.tiles_n;
@@ -588,10 +665,16 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
         return RQ_ERR_CUDA;
       attr_done = true;
     }
-    gemm_int4_kernel<<<grid, kGemmThreads, kI4Smem, st>>>(tx, tw, p);
+    gemm_int4_kernel<<<grid, kI4Threads, kI4Smem, st>>>(tx, tw, p);
   } else {
+    CUtensorMap tsx, tsw, ty;
+    std::memset(&ty, 0, sizeof(ty));
+    p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
+    if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
     if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tsx, xs, (uint64_t)M, (uint64_t)K / 16, kBM, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap_u8(&tsw, ws, (uint64_t)N, (uint64_t)K / 16, kBN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
       return RQ_ERR_CUDA;
     static bool attr_done = false;
     if (!attr_done) {
@@ -600,7 +683,7 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
         return RQ_ERR_CUDA;
       attr_done = true;
     }
-    gemm_nvfp4_kernel<<<grid, kGemmThreads, kF4Smem, st>>>(tx, tw, p);
+    gemm_nvfp4_kernel<<<grid, kGemmThreads, kF4Smem, st>>>(tx, tw, tsx, tsw, ty, p);
   }
   return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }

@@ -13,12 +13,16 @@
 // and packs two codes per byte, element 2i in the low nibble.
 //
 // Design (B200):
-// * A CTA owns a tile of R rows.  One thread owns one 128-wide block of one
-//   row and keeps it in 128 registers, so all seven butterfly stages of the
-//   128-point fast Walsh-Hadamard transform run in registers (no shuffles).
-// * Rows reach shared memory through TMA bulk copies (cp.async.bulk, no tensor
-//   map, no multicast) into a STAGES-deep ring guarded by mbarriers; one
-//   elected thread issues the copies, merging rows that are contiguous in HBM.
+// * One thread owns one 128-wide block of one row and keeps it in 128
+//   registers, so all seven butterfly stages of the 128-point fast
+//   Walsh-Hadamard transform run in registers (no shuffles).
+// * Work is organised in warp groups, not CTAs: a group is the G warps that
+//   cover one row (G = 1 for K <= 4096, where a warp may hold 32/(K/128) rows;
+//   G = K/4096 rounded up otherwise).  Each group owns a ring of shared-memory
+//   stages filled by TMA bulk copies (cp.async.bulk, no tensor map, no
+//   multicast) and guarded by its own mbarriers, so groups never wait on one
+//   another; the only synchronisation is __syncwarp or a named barrier over
+//   the group's warps.  Rows that are contiguous in HBM go in one copy.
 // * Bank conflicts: thread u reads 16-byte chunk (j XOR m) into register slot j,
 //   m = u mod 8, so the 8 threads of every shared-memory phase hit 8 different
 //   bank groups.  Permuting the input by XOR with M = 8m multiplies the
@@ -28,10 +32,10 @@
 // * The sign diagonal is applied to the packed bf16 pairs with one XOR per
 //   pair, using a per-CTA table of sign masks in shared memory.
 // * Full-width rotations (B = K = 128*NB, NB <= 32) use the Kronecker split
-//   H_K = H_NB (x) H_128: after the in-register 128-point transform, the
-//   block's outputs are transposed through shared memory (the consumed input
-//   stage, XOR-swizzled, in two halves) and the NB-point transform across
-//   blocks runs in registers again.
+//   H_K = H_NB (x) H_128: after the in-register 128-point transform, each warp
+//   transposes its rows' block outputs through its own consumed stage buffer
+//   (XOR-swizzled, in two halves) and runs the NB-point transform across blocks
+//   in registers again.
 // * Rounding to integers uses the 1.5*2^23 "magic" add (the FPU's
 //   round-to-nearest-even), whose low mantissa bits are the two's-complement
 //   code; packing gathers low bytes with PRMT.
@@ -51,6 +55,7 @@ struct RotParams {
   // row -> address: t = row % S, bh = row / S, h = bh % H, b = bh / H
   int64_t S, H;
   int64_t sB, sH, sS;  // byte strides
+  int contiguous;      // 1: row r starts at x + r * K * 2
   const int8_t* signs; // [K]
   uint8_t* codes;      // [rows, K/2]
   float* scales_f32;   // INT4: [rows]
@@ -62,56 +67,59 @@ struct RotParams {
   const float* g_in;   // NVFP4 static: the per-tensor scale (device scalar)
   float* g_out;        // NVFP4: the per-tensor scale used (written by CTA 0)
   unsigned* amax_word; // NVFP4 dynamic: max |X~| as fp32 bits (AMAX writes, NVFP4 reads)
-  int R;               // rows per tile
-  int64_t num_tiles;
-  int stages;
   int nvfp4_dynamic;   // 1: g from amax_word, 0: g from g_in
   float cfull;         // 1/sqrt(K) for full-width rotations (rounded once from the exact value)
+  // geometry (host-chosen)
+  int G;               // warps per group
+  int RPS;             // rows per stage
+  int GPC;             // groups per CTA
+  int stages;          // ring depth per group
+  int64_t num_tiles;   // ceil(rows / RPS)
 };
 
 struct RotSmemLayout {
-  // [stages][R*K*2] input ring | sign masks [nb*64] u32 | row amax [2][R] u32 | mbarriers [stages] | flag
-  static __host__ __device__ size_t stage_bytes(int R, int K) { return (size_t)R * K * 2; }
-  static __host__ __device__ size_t total(int R, int K, int stages) {
-    size_t b = stage_bytes(R, K) * stages;
+  // [GPC][stages][RPS*K*2] rings | sign masks [nb*64] u32 | amax slots [GPC][G] u32 | mbarriers [GPC][stages]
+  static __host__ __device__ size_t stage_bytes(int RPS, int K) { return (size_t)RPS * K * 2; }
+  static __host__ __device__ size_t rings(int RPS, int K, int stages, int GPC) {
+    return stage_bytes(RPS, K) * stages * GPC;
+  }
+  static __host__ __device__ size_t total(int RPS, int K, int stages, int GPC, int G) {
+    size_t b = rings(RPS, K, stages, GPC);
     b += (size_t)(K / 128) * 64 * 4;
-    b += 2 * (size_t)R * 4;
+    b += (size_t)GPC * G * 4;
     b = (b + 7) & ~(size_t)7;
-    b += (size_t)stages * 8 + 16;
+    b += (size_t)GPC * stages * 8;
     return b;
   }
 };
 
-__device__ __forceinline__ const uint8_t* row_addr(const RotParams& p, int64_t row) {
-  const int64_t t = row % p.S;
-  const int64_t bh = row / p.S;
-  const int64_t h = bh % p.H;
-  const int64_t b = bh / p.H;
-  return p.x + b * p.sB + h * p.sH + t * p.sS;
-}
-
-// Issue the bulk copies of tile `tile` into `dst` (one elected thread).
+// Issue the bulk copies of tile `tile` (RPS rows) into `dst` (one elected thread).
 __device__ __forceinline__ void issue_tile_load(const RotParams& p, int64_t tile, uint8_t* dst, uint64_t* bar) {
-  const int64_t r0 = tile * p.R;
-  const int nrows = (int)min((int64_t)p.R, p.rows - r0);
+  const int64_t r0 = tile * p.RPS;
+  const int nrows = (int)min((int64_t)p.RPS, p.rows - r0);
   const unsigned row_bytes = (unsigned)p.K * 2u;
   mbar_arrive_expect_tx(bar, row_bytes * (unsigned)nrows);
-  const uint8_t* run_src = row_addr(p, r0);
-  unsigned run_bytes = row_bytes;
-  int run_row = 0;
-  for (int r = 1; r < nrows; ++r) {
-    const uint8_t* a = row_addr(p, r0 + r);
-    if (a == run_src + run_bytes && run_bytes + row_bytes <= (1u << 19)) {
-      run_bytes += row_bytes;
-    } else {
-      bulk_g2s(dst + (size_t)run_row * row_bytes, run_src, run_bytes, bar);
-      run_src = a;
-      run_bytes = row_bytes;
-      run_row = r;
+  if (p.contiguous) {
+    bulk_g2s(dst, p.x + r0 * (int64_t)row_bytes, row_bytes * (unsigned)nrows, bar);
+    return;
+  }
+  // general strides: walk (b, h, t) incrementally from the first row
+  int64_t t = r0 % p.S;
+  int64_t bh = r0 / p.S;
+  int64_t h = bh % p.H;
+  int64_t b = bh / p.H;
+  for (int r = 0; r < nrows; ++r) {
+    bulk_g2s(dst + (size_t)r * row_bytes, p.x + b * p.sB + h * p.sH + t * p.sS, row_bytes, bar);
+    if (++t == p.S) {
+      t = 0;
+      if (++h == p.H) {
+        h = 0;
+        ++b;
+      }
     }
   }
-  bulk_g2s(dst + (size_t)run_row * row_bytes, run_src, run_bytes, bar);
 }
+
 
 // 128-point fast Walsh-Hadamard transform in registers (unnormalized).
 __device__ __forceinline__ void fwht128(float (&v)[128]) {
@@ -184,23 +192,6 @@ __device__ __forceinline__ float absmax128(const float (&v)[128]) {
   return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
 }
 
-// Reduce a non-negative float max over the threads of one row and return it
-// to all of them.  Rows are nb consecutive threads.
-__device__ __forceinline__ float row_max(float a, int nb, int tid, int r, unsigned* slot_base, bool valid) {
-  uint32_t bits = valid ? __float_as_uint(a) : 0u;
-  if ((nb & 31) == 0) {
-    bits = __reduce_max_sync(0xFFFFFFFFu, bits);
-    if ((tid & 31) == 0) atomicMax(slot_base + r, bits);
-  } else if ((32 % nb) == 0) {
-    for (int o = 1; o < nb; o <<= 1) bits = max(bits, __shfl_xor_sync(0xFFFFFFFFu, bits, o));
-    if ((tid % nb) == 0 && valid) slot_base[r] = bits;
-  } else {
-    if (valid) atomicMax(slot_base + r, bits);
-  }
-  __syncthreads();
-  return __uint_as_float(slot_base[r]);
-}
-
 // INT4 per-row quantization of v (true value = v * c * chi) and packing.
 // amax_true: the row's max |x~|.  Writes 64 bytes at dst.
 __device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c, float amax_true, int m,
@@ -208,23 +199,26 @@ __device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c,
   // r = 7/amax; zero rows -> r = 0 -> all codes 0
   const float r = amax_true > 0.f ? __fdiv_rn(7.0f, amax_true) : 0.0f;
   const float cr = c * r;
-  uint32_t words[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {  // chunk j = 8 elements -> one word
-    const float mul = with_sign(cr, chi_signbit(j, m));
-    float q[8];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float2 t = __ffma2_rn(make_float2(v[8 * j + e], v[8 * j + e + 1]), make_float2(mul, mul),
-                                  make_float2(kRoundMagic, kRoundMagic));
-      q[e] = t.x;
-      q[e + 1] = t.y;
-    }
-    words[j] = pack8_magic(q);
-  }
   uint4* out = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) out[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+  for (int j4 = 0; j4 < 4; ++j4) {
+    uint32_t w[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {  // chunk j = 8 elements -> one word
+      const int j = 4 * j4 + jj;
+      const float mul = with_sign(cr, chi_signbit(j, m));
+      float q[8];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float2 t = __ffma2_rn(make_float2(v[8 * j + e], v[8 * j + e + 1]), make_float2(mul, mul),
+                                    make_float2(kRoundMagic, kRoundMagic));
+        q[e] = t.x;
+        q[e + 1] = t.y;
+      }
+      w[jj] = pack8_magic(q);
+    }
+    out[j4] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 // NVFP4 quantization of v (true value = v * c * chi): 8 groups of 16.
@@ -300,27 +294,31 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
   // whether clamping to [0, 15] can be needed for this vector.
   const float tlo = fmaf(lo, inv, off), thi = fmaf(hi, inv, off);
   const bool need_clamp = !(tlo > -0.5f && thi < 15.5f);
-  uint32_t words[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float mul = with_sign(ci, chi_signbit(j, m));
-    float q[8];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      float2 t = __ffma2_rn(make_float2(v[8 * j + e], v[8 * j + e + 1]), make_float2(mul, mul), make_float2(off, off));
-      if (need_clamp) {
-        t.x = fminf(fmaxf(t.x, 0.0f), 15.0f);
-        t.y = fminf(fmaxf(t.y, 0.0f), 15.0f);
-      }
-      t = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
-      q[e] = t.x;
-      q[e + 1] = t.y;
-    }
-    words[j] = pack8_magic(q);
-  }
   uint4* out = reinterpret_cast<uint4*>(dst_codes);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) out[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+  for (int j4 = 0; j4 < 4; ++j4) {
+    uint32_t w[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = 4 * j4 + jj;
+      const float mul = with_sign(ci, chi_signbit(j, m));
+      float q[8];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float2 t = __ffma2_rn(make_float2(v[8 * j + e], v[8 * j + e + 1]), make_float2(mul, mul),
+                              make_float2(off, off));
+        if (need_clamp) {
+          t.x = fminf(fmaxf(t.x, 0.0f), 15.0f);
+          t.y = fminf(fmaxf(t.y, 0.0f), 15.0f);
+        }
+        t = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+        q[e] = t.x;
+        q[e + 1] = t.y;
+      }
+      w[jj] = pack8_magic(q);
+    }
+    out[j4] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
   *dst_scale = s_h;
   *dst_zero = z_h;
 }
@@ -335,310 +333,315 @@ __device__ __forceinline__ void store_f32_block(const float (&v)[128], float c, 
   }
 }
 
-// Kernel prologue shared by both variants: smem carve-up, barrier init, sign
-// table, first loads.  Returns false if this CTA has no work.
-struct RotSmem {
-  uint8_t* ring;
-  uint32_t* smask;
-  unsigned* row_amax;  // [2][R]
-  uint64_t* full;
-  int* flag;
-};
 
-__device__ __forceinline__ RotSmem carve(uint8_t* base, const RotParams& p) {
-  RotSmem s;
-  s.ring = base;
-  size_t off = RotSmemLayout::stage_bytes(p.R, p.K) * p.stages;
-  s.smask = reinterpret_cast<uint32_t*>(base + off);
-  off += (size_t)p.nb * 64 * 4;
-  s.row_amax = reinterpret_cast<unsigned*>(base + off);
-  off += 2 * (size_t)p.R * 4;
-  off = (off + 7) & ~(size_t)7;
-  s.full = reinterpret_cast<uint64_t*>(base + off);
-  off += (size_t)p.stages * 8;
-  s.flag = reinterpret_cast<int*>(base + off);
-  return s;
+// Synchronise the G warps of a group (named barrier 1 + group index).
+__device__ __forceinline__ void group_sync(int G, int grp) {
+  if (G == 1) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(32 * G) : "memory");
+  }
 }
 
-__device__ __forceinline__ void prologue(const RotParams& p, RotSmem& s) {
-  const int tid = threadIdx.x;
-  // sign mask table: pair (2q, 2q+1) of channel block b -> XOR mask on the bf16x2 word
-  for (int i = tid; i < p.nb * 64; i += blockDim.x) {
-    const int b = i >> 6, q = i & 63;
-    const int8_t s0 = p.signs[b * 128 + 2 * q], s1 = p.signs[b * 128 + 2 * q + 1];
-    s.smask[i] = (s0 < 0 ? 0x8000u : 0u) | (s1 < 0 ? 0x80000000u : 0u);
-  }
-  if (tid < 2 * p.R) s.row_amax[tid] = 0u;
-  if (tid == 0) {
-    for (int st = 0; st < p.stages; ++st) mbar_init(&s.full[st], 1);
-    fence_mbar_init();
-    const size_t sb = RotSmemLayout::stage_bytes(p.R, p.K);
-    int64_t tile = blockIdx.x;
-    for (int st = 0; st < p.stages && tile < p.num_tiles; ++st, tile += gridDim.x)
-      issue_tile_load(p, tile, s.ring + st * sb, &s.full[st]);
-  }
-  __syncthreads();
+// Group-wide AND of a predicate (all threads of the group get the result).
+__device__ __forceinline__ bool group_all(bool v, int G, int grp) {
+  if (G == 1) return __all_sync(0xFFFFFFFFu, v);
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(1 + grp), "r"(32 * G)
+      : "memory");
+  return out != 0;
 }
 
-// Wait for stage `st` with parity; thread 0 waits (bounded) and publishes.
-__device__ __forceinline__ bool wait_stage(RotSmem& s, int st, unsigned parity) {
-  if (threadIdx.x == 0) *s.flag = mbar_wait_bounded(&s.full[st], parity) ? 1 : 0;
-  __syncthreads();
-  return *s.flag != 0;
+// Max of a non-negative float over the threads of one row; every thread of
+// the row gets it.  Rows are `seg` consecutive lanes when RPS > 1 (seg = nb, a
+// power of two below 32), a whole warp when G == 1, or the group's G warps.
+__device__ __forceinline__ float row_max(float a, int RPS, int nb, int G, int grp, int wig, unsigned* slots) {
+  uint32_t bits = __float_as_uint(a);
+  if (RPS > 1) {
+    for (int o = 1; o < nb; o <<= 1) bits = max(bits, __shfl_xor_sync(0xFFFFFFFFu, bits, o));
+    return __uint_as_float(bits);
+  }
+  bits = __reduce_max_sync(0xFFFFFFFFu, bits);
+  if (G == 1) return __uint_as_float(bits);
+  if ((threadIdx.x & 31) == 0) slots[grp * G + wig] = bits;
+  group_sync(G, grp);
+  uint32_t m = 0;
+  for (int w = 0; w < G; ++w) m = max(m, ((volatile unsigned*)slots)[grp * G + w]);
+  return __uint_as_float(m);
 }
 
-// After a timeout: wait (bounded) for the copies this CTA issued, then return.
-__device__ __forceinline__ void drain_after_timeout(RotSmem& s, const RotParams& p, int64_t i_fail) {
-  if (threadIdx.x != 0) return;
-  // stages that may still have copies in flight: tiles i_fail .. i_fail+stages-1
-  for (int k = 0; k < p.stages; ++k) {
-    const int64_t i = i_fail + k;
-    const int64_t tile = blockIdx.x + i * gridDim.x;
-    if (tile >= p.num_tiles) break;
-    (void)mbar_wait_bounded(&s.full[i % p.stages], (unsigned)((i / p.stages) & 1));
+// Full-width second phase for one half (h) of every block's outputs: the rows'
+// outputs are transposed through `zbuf` (this warp's consumed stage) and the
+// NB-point transform runs across blocks.  Thread (r, b): on entry v holds
+// chi-signed block outputs of block b of row r; on exit y[bb][c] holds
+// y(bb*128 + 64h + b*COLS + c) for all NB blocks bb.
+template <int NB>
+__device__ __forceinline__ void full_phase2(const float (&v)[128], float (&y)[NB][64 / NB], int h, float* zbuf,
+                                            int r, int b, int lane, int m, float cfull, bool valid) {
+  constexpr int COLS = 64 / NB;
+  float* zrow = zbuf + (size_t)r * NB * 64;
+  {
+    float* zb = zrow + (size_t)b * 64;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float mul = with_sign(cfull, chi_signbit(8 * h + (q >> 1), m));
+      const int k = 64 * h + 4 * q;
+      *reinterpret_cast<float4*>(zb + 4 * (q ^ (lane & 7))) =
+          make_float4(v[k] * mul, v[k + 1] * mul, v[k + 2] * mul, v[k + 3] * mul);
+    }
   }
+  __syncwarp();
+  {
+#pragma unroll
+    for (int bb = 0; bb < NB; ++bb) {
+      const int wl = (NB >= 8) ? (bb & 7) : ((r * NB + bb) & 7);  // XOR key of the lane that wrote block bb
+      const float* zb = zrow + (size_t)bb * 64;
+#pragma unroll
+      for (int pp = 0; pp < COLS / 2; ++pp) {
+        const int P = b * (COLS / 2) + pp;
+        const float2 t = *reinterpret_cast<const float2*>(zb + 4 * ((P >> 1) ^ wl) + 2 * (P & 1));
+        y[bb][2 * pp] = t.x;
+        y[bb][2 * pp + 1] = t.y;
+      }
+    }
+  }
+  __syncwarp();
+  {
+#pragma unroll
+    for (int hh = 1; hh < NB; hh <<= 1) {
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb) {
+        if ((bb & hh) == 0) {
+#pragma unroll
+          for (int cc = 0; cc < COLS; cc += 2) {
+            const float2 a = make_float2(y[bb][cc], y[bb][cc + 1]);
+            const float2 d = make_float2(y[bb + hh][cc], y[bb + hh][cc + 1]);
+            const float2 s = __fadd2_rn(a, d);
+            const float2 e = __ffma2_rn(d, make_float2(-1.0f, -1.0f), a);
+            y[bb][cc] = s.x;
+            y[bb][cc + 1] = s.y;
+            y[bb + hh][cc] = e.x;
+            y[bb + hh][cc + 1] = e.y;
+          }
+        }
+      }
+    }
+  }
+}
+
+// INT4 quantize + store of the full-width layout: COLS values per (block, half).
+template <int NB>
+__device__ __forceinline__ void full_store_int4(const float (&y)[2][NB][64 / NB], float rr, uint8_t* crow, int b) {
+  constexpr int COLS = 64 / NB;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int bb = 0; bb < NB; ++bb) {
+      uint32_t byt[COLS / 2];
+#pragma unroll
+      for (int cc = 0; cc < COLS; cc += 2) {
+        const float2 t = __ffma2_rn(make_float2(y[h][bb][cc], y[h][bb][cc + 1]), make_float2(rr, rr),
+                                    make_float2(kRoundMagic, kRoundMagic));
+        byt[cc / 2] = (__float_as_uint(t.x) & 0xFu) | ((__float_as_uint(t.y) & 0xFu) << 4);
+      }
+      uint8_t* dst = crow + bb * 64 + 32 * h + b * (COLS / 2);
+      if (COLS / 2 == 1) {
+        dst[0] = (uint8_t)byt[0];
+      } else if (COLS / 2 == 2) {
+        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)(byt[0] | (byt[1 % (COLS / 2)] << 8));
+      } else {
+#pragma unroll
+        for (int w4 = 0; w4 < COLS / 8; ++w4)
+          reinterpret_cast<uint32_t*>(dst)[w4] =
+              byt[(4 * w4) % (COLS / 2)] | (byt[(4 * w4 + 1) % (COLS / 2)] << 8) |
+              (byt[(4 * w4 + 2) % (COLS / 2)] << 16) | (byt[(4 * w4 + 3) % (COLS / 2)] << 24);
+      }
+    }
 }
 
 // ---------------------------------------------------------------------------
-// Block-diagonal (B = 128) rotation: every mode.
+// The kernel.  NBF = 0: block-diagonal (B = 128), any mode.  NBF = 2..32:
+// full-width rotation of K = 128*NBF (INT4 and F32 modes).
 // ---------------------------------------------------------------------------
-template <int MODE>
-__global__ void __launch_bounds__(384, 1) rotate_block_kernel(const RotParams p) {
+template <int MODE, int NBF>
+__global__ void __launch_bounds__((MODE == kModeInt4 && NBF == 0) ? 384 : 256, 1) rotate_kernel(const RotParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  RotSmem s = carve(smem_raw, p);
-  prologue(p, s);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G, RPS = p.RPS, nb = p.nb;
+  const int grp = warp / G, wig = warp - grp * G;
+  const size_t sbytes = RotSmemLayout::stage_bytes(RPS, p.K);
+  uint8_t* ring = smem_raw + (size_t)grp * p.stages * sbytes;
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw + RotSmemLayout::rings(RPS, p.K, p.stages, p.GPC));
+  unsigned* slots = reinterpret_cast<unsigned*>(smask + nb * 64);
+  uint64_t* bars_all = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(slots + p.GPC * G) + 7) & ~(uintptr_t)7);
+  uint64_t* full = bars_all + grp * p.stages;
 
-  const int tid = threadIdx.x;
-  const int nb = p.nb;
-  const int r = tid / nb;
-  const int b = tid - r * nb;
-  const int m = tid & 7;
-  const float c = 0.08838834764831845f;  // 1/sqrt(128)
-  const size_t sb = RotSmemLayout::stage_bytes(p.R, p.K);
+  // thread -> (row in stage, block)
+  int r, b;
+  bool active;
+  if (RPS > 1) {
+    r = lane / nb;
+    b = lane - r * nb;
+    active = r < RPS;
+  } else {
+    r = 0;
+    b = wig * 32 + lane;
+    active = b < nb;
+  }
+  const int m = lane & 7;
+  const bool producer = (wig == 0 && lane == 0);
+  const float c = 0.08838834764831845f;  // 1/sqrt(128), rounded once
+  const int64_t TG = (int64_t)gridDim.x * p.GPC;
+  const int64_t gg = (int64_t)blockIdx.x * p.GPC + grp;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.GPC * p.stages; ++i) mbar_init(&bars_all[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (producer) {  // start streaming before anything else
+    int64_t tile = gg;
+    for (int st = 0; st < p.stages && tile < p.num_tiles; ++st, tile += TG)
+      issue_tile_load(p, tile, ring + st * sbytes, &full[st]);
+  }
+  // sign-mask table, 16 signs (8 masks) per thread and pass, while the copies fly
+  for (int i = threadIdx.x; i < nb * 8; i += blockDim.x) {
+    const uint4 sg = __ldg(reinterpret_cast<const uint4*>(p.signs) + i);
+    const uint32_t w[4] = {sg.x, sg.y, sg.z, sg.w};
+    uint32_t mk[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // byte k of w[j] is the sign of channel 16i + 4j + k; negative <=> bit 7 set
+      const uint32_t neg = w[j] & 0x80808080u;
+      mk[2 * j] = ((neg & 0x80u) << 8) | ((neg & 0x8000u) << 16);
+      mk[2 * j + 1] = ((neg & 0x800000u) >> 8) | (neg & 0x80000000u);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(smask + 8 * i);
+    dst[0] = make_uint4(mk[0], mk[1], mk[2], mk[3]);
+    dst[1] = make_uint4(mk[4], mk[5], mk[6], mk[7]);
+  }
+  __syncthreads();
 
   float g = 0.f, inv6g = 0.f;
   if (MODE == kModeNvfp4) {
-    if (p.nvfp4_dynamic) {
-      const float amax = __uint_as_float(*((volatile unsigned*)p.amax_word));
-      g = __fdiv_rn(amax, 2688.0f);
-    } else {
-      g = *p.g_in;
-    }
+    g = p.nvfp4_dynamic ? __fdiv_rn(__uint_as_float(*((volatile unsigned*)p.amax_word)), 2688.0f) : *p.g_in;
     inv6g = g > 0.f ? __frcp_rn(6.0f * g) : 0.0f;
-    if (blockIdx.x == 0 && tid == 0 && p.g_out) *p.g_out = g;
+    if (blockIdx.x == 0 && threadIdx.x == 0 && p.g_out) *p.g_out = g;
   }
   float amax_acc = 0.f;
 
   int64_t i = 0;
-  for (int64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
+  for (int64_t tile = gg; tile < p.num_tiles; tile += TG, ++i) {
     const int st = (int)(i % p.stages);
-    if (!wait_stage(s, st, (unsigned)((i / p.stages) & 1))) {
-      drain_after_timeout(s, p, i + 1);
+    const bool ok = group_all(mbar_wait_bounded(&full[st], (unsigned)((i / p.stages) & 1)), G, grp);
+    if (!ok) {
+      if (producer) {  // let the copies this group issued land before leaving
+        for (int k = 1; k < p.stages; ++k) {
+          const int64_t i2 = i + k;
+          if (gg + i2 * TG >= p.num_tiles) break;
+          (void)mbar_wait_bounded(&full[i2 % p.stages], (unsigned)((i2 / p.stages) & 1));
+        }
+      }
       return;
     }
-    const int64_t r0 = tile * p.R;
-    const int nrows = (int)min((int64_t)p.R, p.rows - r0);
-    const bool valid = r < nrows;
-    unsigned* slot = s.row_amax + (i & 1) * p.R;
-    if (MODE == kModeInt4 && tid < p.R) slot[tid] = 0u;
-
-    float v[128];
-    if (valid) {
-      load_block(s.ring + st * sb + (size_t)r * p.K * 2 + (size_t)b * 256, s.smask + b * 64, m, v);
-    }
-    __syncthreads();  // stage consumed; row slots reset
-    if (tid == 0) {
-      const int64_t nt = tile + (int64_t)p.stages * gridDim.x;
-      if (nt < p.num_tiles) {
-        fence_proxy_async_smem();
-        issue_tile_load(p, nt, s.ring + st * sb, &s.full[st]);
-      }
-    }
-    if (valid) fwht128(v);
+    const int64_t r0 = tile * RPS;
+    const int nrows = (int)min((int64_t)RPS, p.rows - r0);
+    const bool valid = active && r < nrows;
+    uint8_t* stage = ring + st * sbytes;
     const int64_t row = r0 + r;
 
-    if (MODE == kModeInt4) {
-      const float a = valid ? absmax128(v) * c : 0.f;
-      const float amax_row = row_max(a, nb, tid, r, slot, valid);
-      if (valid) {
-        quant_int4_store(v, c, amax_row, m, p.codes + row * (p.K / 2) + (size_t)b * 64);
-        if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
-      }
-    } else if (MODE == kModeNvfp4) {
-      if (valid)
-        quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                          p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
-    } else if (MODE == kModeF32) {
-      if (valid) store_f32_block(v, c, m, p.out_f32 + row * p.ldo + (size_t)b * 128);
-    } else if (MODE == kModeAmax) {
-      if (valid) amax_acc = fmaxf(amax_acc, absmax128(v) * c);
-    } else if (MODE == kModeKv4) {
-      if (valid) quant_kv4_store(v, c, m, p.codes + row * 64, p.kv_scale + row, p.kv_zero + row);
-    }
-  }
-  if (MODE == kModeAmax) {
-    const unsigned bits = __reduce_max_sync(__activemask(), __float_as_uint(amax_acc));
-    if ((tid & 31) == 0) atomicMax(p.amax_word, bits);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Full-width rotation, K = 128 * NB (NB = 2..32): INT4 and F32.
-// ---------------------------------------------------------------------------
-template <int MODE, int NB>
-__global__ void __launch_bounds__(256, 1) rotate_full_kernel(const RotParams p) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  RotSmem s = carve(smem_raw, p);
-  prologue(p, s);
-
-  constexpr int COLS = 64 / NB;   // i-columns per thread per half
-  const int tid = threadIdx.x;
-  const int r = tid / NB;
-  const int b = tid - r * NB;     // phase 1: block; phase 2: column group t'
-  const int m = tid & 7;
-  const float cfull = p.cfull;
-  const size_t sb = RotSmemLayout::stage_bytes(p.R, p.K);
-
-  int64_t i = 0;
-  for (int64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
-    const int st = (int)(i % p.stages);
-    if (!wait_stage(s, st, (unsigned)((i / p.stages) & 1))) {
-      drain_after_timeout(s, p, i + 1);
-      return;
-    }
-    const int64_t r0 = tile * p.R;
-    const int nrows = (int)min((int64_t)p.R, p.rows - r0);
-    const bool valid = r < nrows;
-    unsigned* slot = s.row_amax + (i & 1) * p.R;
-    if (MODE == kModeInt4 && tid < p.R) slot[tid] = 0u;
-    uint8_t* stage = s.ring + st * sb;
-
     float v[128];
-    if (valid) load_block(stage + (size_t)r * p.K * 2 + (size_t)b * 256, s.smask + b * 64, m, v);
-    __syncthreads();  // stage consumed: reuse it as the transpose buffer
-    if (valid) fwht128(v);
+    // every thread loads and transforms (no predication of the 128-register block);
+    // threads without a row read an in-bounds block and store nothing
+    const int bl = active ? b : 0;
+    load_block(stage + (size_t)(active ? r : 0) * p.K * 2 + (size_t)bl * 256, smask + bl * 64, m, v);
 
-    // y[bb][col] for this thread's 2*COLS columns (half h: columns 64h + b*COLS + c)
-    float y[2][NB][COLS];
-    float* zrow = reinterpret_cast<float*>(stage) + (size_t)r * NB * 64;  // [NB][64] per row
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (valid) {
-        // write half h of this block's outputs: 16 chunks of 4 floats, XOR-swizzled by the writer index
-        float* zb = zrow + (size_t)b * 64;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float mul = with_sign(cfull, chi_signbit(8 * h + (q >> 1), m));
-          const int k = 64 * h + 4 * q;
-          *reinterpret_cast<float4*>(zb + 4 * (q ^ (tid & 7))) =
-              make_float4(v[k] * mul, v[k + 1] * mul, v[k + 2] * mul, v[k + 3] * mul);
+    if (NBF == 0) {
+      group_sync(G, grp);  // stage consumed: refill it while this tile is computed
+      if (producer) {
+        const int64_t nt = tile + (int64_t)p.stages * TG;
+        if (nt < p.num_tiles) {
+          fence_proxy_async_smem();
+          issue_tile_load(p, nt, stage, &full[st]);
         }
       }
-      __syncthreads();
-      if (valid) {
-#pragma unroll
-        for (int bb = 0; bb < NB; ++bb) {
-          const int wtid = r * NB + bb;  // writer thread of block bb
-          const float* zb = zrow + (size_t)bb * 64;
-#pragma unroll
-          for (int pp = 0; pp < COLS / 2; ++pp) {
-            const int P = b * (COLS / 2) + pp;  // float2 index within the half row
-            const int q = P >> 1;
-            const float2 t = *reinterpret_cast<const float2*>(zb + 4 * (q ^ (wtid & 7)) + 2 * (P & 1));
-            y[h][bb][2 * pp] = t.x;
-            y[h][bb][2 * pp + 1] = t.y;
-          }
+      fwht128(v);
+      if (MODE == kModeInt4) {
+        const float a = valid ? absmax128(v) * c : 0.f;
+        const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
+        if (valid) {
+          quant_int4_store(v, c, amax_row, m, p.codes + row * (p.K / 2) + (size_t)b * 64);
+          if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
+        }
+      } else if (MODE == kModeNvfp4) {
+        if (valid)
+          quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                            p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+      } else if (MODE == kModeF32) {
+        if (valid) store_f32_block(v, c, m, p.out_f32 + row * p.ldo + (size_t)b * 128);
+      } else if (MODE == kModeAmax) {
+        if (valid) amax_acc = fmaxf(amax_acc, absmax128(v) * c);
+      } else if (MODE == kModeKv4) {
+        if (valid) quant_kv4_store(v, c, m, p.codes + row * 64, p.kv_scale + row, p.kv_zero + row);
+      }
+    } else {
+      constexpr int NB = NBF ? NBF : 1;
+      constexpr int COLS = 64 / NB;
+      float y[2][NB][COLS];
+      fwht128(v);
+      __syncwarp();  // every lane has read the stage: reuse it as the transpose buffer
+      float* zbuf = reinterpret_cast<float*>(stage);
+      full_phase2<NB>(v, y[0], 0, zbuf, r, b, lane, m, p.cfull, valid);
+      full_phase2<NB>(v, y[1], 1, zbuf, r, b, lane, m, p.cfull, valid);
+      if (producer) {
+        const int64_t nt = tile + (int64_t)p.stages * TG;
+        if (nt < p.num_tiles) {
+          fence_proxy_async_smem();
+          issue_tile_load(p, nt, stage, &full[st]);
         }
       }
-      __syncthreads();
-      if (valid) {
-        // NB-point transform across blocks, per column
-#pragma unroll
-        for (int hh = 1; hh < NB; hh <<= 1) {
-#pragma unroll
-          for (int bb = 0; bb < NB; ++bb) {
-            if ((bb & hh) == 0) {
-#pragma unroll
-              for (int cc = 0; cc < COLS; cc += 2) {
-                const float2 a = make_float2(y[h][bb][cc], y[h][bb][cc + 1]);
-                const float2 d = make_float2(y[h][bb + hh][cc], y[h][bb + hh][cc + 1]);
-                const float2 sum = __fadd2_rn(a, d);
-                const float2 dif = __ffma2_rn(d, make_float2(-1.0f, -1.0f), a);
-                y[h][bb][cc] = sum.x;
-                y[h][bb][cc + 1] = sum.y;
-                y[h][bb + hh][cc] = dif.x;
-                y[h][bb + hh][cc + 1] = dif.y;
-              }
-            }
-          }
-        }
-      }
-    }
-    if (tid == 0) {
-      const int64_t nt = tile + (int64_t)p.stages * gridDim.x;
-      if (nt < p.num_tiles) {
-        fence_proxy_async_smem();
-        issue_tile_load(p, nt, stage, &s.full[st]);
-      }
-    }
-    const int64_t row = r0 + r;
-    if (MODE == kModeInt4) {
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int bb = 0; bb < NB; ++bb)
-#pragma unroll
-          for (int cc = 0; cc < COLS; cc += 2) {
-            a0 = fmaxf(a0, fabsf(y[h][bb][cc]));
-            a1 = fmaxf(a1, fabsf(y[h][bb][cc + 1]));
-          }
-      const float amax_row = row_max(valid ? fmaxf(a0, a1) : 0.f, NB, tid, r, slot, valid);
-      if (valid) {
-        const float rr = amax_row > 0.f ? __fdiv_rn(7.0f, amax_row) : 0.0f;
-        uint8_t* crow = p.codes + row * (p.K / 2);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int bb = 0; bb < NB; ++bb) {
-            // COLS values -> COLS/2 bytes at byte offset bb*64 + 32h + b*COLS/2
-            uint32_t byt[COLS / 2];
-#pragma unroll
-            for (int cc = 0; cc < COLS; cc += 2) {
-              const float2 t = __ffma2_rn(make_float2(y[h][bb][cc], y[h][bb][cc + 1]), make_float2(rr, rr),
-                                          make_float2(kRoundMagic, kRoundMagic));
-              byt[cc / 2] = (__float_as_uint(t.x) & 0xFu) | ((__float_as_uint(t.y) & 0xFu) << 4);
-            }
-            uint8_t* dst = crow + bb * 64 + 32 * h + b * (COLS / 2);
-            if (COLS / 2 == 1) {
-              dst[0] = (uint8_t)byt[0];
-            } else if (COLS / 2 == 2) {
-              *reinterpret_cast<uint16_t*>(dst) = (uint16_t)(byt[0] | (byt[1 % (COLS / 2)] << 8));
-            } else {
-#pragma unroll
-              for (int w4 = 0; w4 < COLS / 8; ++w4) {
-                const uint32_t word = byt[(4 * w4) % (COLS / 2)] | (byt[(4 * w4 + 1) % (COLS / 2)] << 8) |
-                                      (byt[(4 * w4 + 2) % (COLS / 2)] << 16) | (byt[(4 * w4 + 3) % (COLS / 2)] << 24);
-                reinterpret_cast<uint32_t*>(dst)[w4] = word;
-              }
-            }
-          }
-        if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
-      }
-    } else if (MODE == kModeF32) {
-      if (valid) {
-        float* orow = p.out_f32 + row * p.ldo;
+      if (MODE == kModeInt4) {
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int bb = 0; bb < NB; ++bb)
 #pragma unroll
-            for (int cc = 0; cc < COLS; cc += 2)
-              *reinterpret_cast<float2*>(orow + bb * 128 + 64 * h + b * COLS + cc) =
-                  make_float2(y[h][bb][cc], y[h][bb][cc + 1]);
+            for (int cc = 0; cc < COLS; cc += 2) {
+              a0 = fmaxf(a0, fabsf(y[h][bb][cc]));
+              a1 = fmaxf(a1, fabsf(y[h][bb][cc + 1]));
+            }
+        const float amax_row = row_max(valid ? fmaxf(a0, a1) : 0.f, RPS, nb, 1, grp, 0, slots);
+        if (valid) {
+          const float rr = amax_row > 0.f ? __fdiv_rn(7.0f, amax_row) : 0.0f;
+          full_store_int4<NB>(y, rr, p.codes + row * (p.K / 2), b);
+          if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
+        }
+      } else if (MODE == kModeF32) {
+        if (valid) {
+          float* orow = p.out_f32 + row * p.ldo;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb)
+#pragma unroll
+              for (int cc = 0; cc < COLS; cc += 2)
+                *reinterpret_cast<float2*>(orow + bb * 128 + 64 * h + b * COLS + cc) =
+                    make_float2(y[h][bb][cc], y[h][bb][cc + 1]);
+        }
       }
     }
-    __syncthreads();  // row slots / stage reuse ordering before the next tile
+  }
+  if (MODE == kModeAmax) {
+    const unsigned bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax_acc));
+    if (lane == 0) atomicMax(p.amax_word, bits);
   }
 }
 

@@ -159,6 +159,21 @@ def nvfp4_tie_bounds(e, sc, g, tie_e, tie_s):
     return xhat, d
 
 
+def check_bf16_y(y_gpu_bf16, y_ref, abs_terms, k):
+    """bf16 Y: within one bf16 step of the oracle's Y rounded to bf16, plus the
+    fp32 accumulation bound gamma_K * sum_k |x_k w_k| (abs_terms) of the GPU's
+    own sum (which matters where terms cancel and Y is near zero)."""
+    got = np.asarray(y_gpu_bf16, dtype=np.float64)
+    rb = bf16_round(y_ref)
+    gamma = k * 2.0 ** -24 / (1 - k * 2.0 ** -24)
+    tol = np.abs(rb) * 2.0 ** -7 + gamma * abs_terms * 2.0 + 1e-30
+    bad = np.abs(got - rb) > tol
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        raise AssertionError("%d bf16 elements off, e.g. %s" % (bad.sum(), [
+            (tuple(i), float(got[tuple(i)]), float(y_ref[tuple(i)]), float(tol[tuple(i)])) for i in idx]))
+
+
 def bf16_round(v):
     return torch.from_numpy(np.asarray(v, dtype=np.float64)).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
 

@@ -62,6 +62,7 @@ def test_rotate_quantize_rejections():
     assert rotq(x=P(0x10002)) == ALIGN
     assert rotq(ldx=516) == ALIGN                   # row pitch not a multiple of 16 bytes
     assert rotq(codes=A8) == ALIGN
+    assert rotq(signs=A8) == ALIGN                 # the sign vector is read 16 bytes at a time
     assert rotq(fmt=7) == INVALID
     assert rotq(gmode=5) == INVALID
     assert rotq(fmt=1, block=0) == SHAPE            # NVFP4 needs 128-wide blocks
@@ -116,6 +117,7 @@ def test_kv_rejections():
     assert kv(d=64) == SHAPE
     assert kv(strides=(4096, 1024, 130)) == ALIGN  # vectors must stay 16-byte aligned
     assert kv(sc=P(0x10001)) == ALIGN
+    assert kv(signs=A8) == ALIGN
     assert kv(strides=(4096, -1, 128)) == INVALID
     assert kv(s=0) == 0
 

@@ -136,6 +136,20 @@ def test_nvfp4_gemm_y(rq, m, n, k):
     assert err < 1e-5
 
 
+@pytest.mark.parametrize("m,n,k", [(1100, 4200, 512), (5, 40, 256), (300, 300, 1024), (2048, 4096, 4096)])
+def test_nvfp4_gemm_bf16(rq, m, n, k):
+    """bf16 Y: each element within one bf16 step of the rounded oracle value
+    (rows of 16-byte multiples go through the TMA-store epilogue, others not)."""
+    gx, gw = np.float32(0.0071), np.float32(0.00013)
+    ex, sx = _rand_nvfp4_operands(m, k, 5 * m + k, gx)
+    ew, sw = _rand_nvfp4_operands(n, k, n + 7 * k, gw)
+    y = rq.w4a4_gemm(_dev_nvfp4(ex, sx, gx), _dev_nvfp4(ew, sw, gw), "nvfp4", "bf16")
+    torch.cuda.synchronize()
+    ref = gemm.nvfp4_y(ex, sx, gx, ew, sw, gw)
+    absterms = np.abs(quant.nvfp4_dequant(ex, sx, gx)) @ np.abs(quant.nvfp4_dequant(ew, sw, gw)).T
+    parity.check_bf16_y(y.float().cpu().numpy(), ref, absterms, k)
+
+
 # ---------------------------------------------------------------- end to end: X, W -> Y
 @pytest.mark.parametrize("fmt,block", [("int4", 128), ("int4", 0), ("nvfp4", 128)])
 def test_end_to_end(rq, fmt, block):
