@@ -81,7 +81,7 @@ RotCfg rotate_config(int64_t K, bool full, int mode) {
     c.G = (nb + 31) / 32;
     c.RPS = 1;
   }
-  const int warps = (!full && mode == kModeInt4) ? 12 : 8;  // must match the kernel's launch bounds
+  const int warps = full ? RQ_FULL_WIDTH_THREADS / 32 : 12;  // must match the kernel's launch bounds
   c.GPC = warps / c.G > 0 ? warps / c.G : 1;
   for (;;) {
     const size_t sb = RotSmemLayout::stage_bytes(c.RPS, (int)K);

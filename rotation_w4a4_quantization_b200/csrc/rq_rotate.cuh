@@ -45,6 +45,11 @@
 
 namespace rq {
 
+// Threads per CTA of the full-width variant (8 warps; 218 registers, no spills).
+#ifndef RQ_FULL_WIDTH_THREADS
+#define RQ_FULL_WIDTH_THREADS 256
+#endif
+
 enum RotMode : int { kModeInt4 = 0, kModeNvfp4 = 1, kModeF32 = 2, kModeAmax = 3, kModeKv4 = 4 };
 
 struct RotParams {
@@ -470,7 +475,7 @@ __device__ __forceinline__ void full_store_int4(const float (&y)[2][NB][64 / NB]
 // full-width rotation of K = 128*NBF (INT4 and F32 modes).
 // ---------------------------------------------------------------------------
 template <int MODE, int NBF>
-__global__ void __launch_bounds__((MODE == kModeInt4 && NBF == 0) ? 384 : 256, 1) rotate_kernel(const RotParams p) {
+__global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_kernel(const RotParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G, RPS = p.RPS, nb = p.nb;
