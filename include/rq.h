@@ -176,6 +176,31 @@ RQ_API rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H,
 RQ_API rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev, int block,
                         float* out_dev, int64_t ldo, rq_stream_t stream);
 
+/*
+ * rq_rotate_quantize_nvfp4_noalloc: rq_rotate_quantize with fmt = RQ_NVFP4,
+ * block = 128 and RQ_SCALE_DYNAMIC, for callers that cannot allocate device
+ * memory -- engines that hand every byte of the GPU to a fixed arena sized at
+ * start-up, plugin interfaces that offer no workspace, and latency-sensitive
+ * hosts that avoid cudaMalloc (which synchronizes the device) after start-up.
+ * It allocates nothing and needs no workspace argument: the 16 bytes of scratch
+ * the dynamic scale needs live in a 256-byte static device array inside the
+ * library (held by every GPU that loads the library until the process exits).
+ * Not part of the method on the pages; it only changes where the scratch lives.
+ *  - Same arguments, layouts and results as rq_rotate_quantize (NVFP4, dynamic
+ *    scale; gscale_dev is written).  The scratch need does not depend on M or
+ *    K; a scratch need above the array's 256 bytes would be rejected with
+ *    RQ_ERR_UNSUPPORTED_SHAPE before anything runs.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call clears the scratch it uses before use, but all calls share the
+ *    one array: calls that may overlap on the GPU (different streams, or
+ *    different host threads) race on it and must be serialized by the caller.
+ */
+RQ_API rq_status rq_rotate_quantize_nvfp4_noalloc(const void* X_dev, int64_t M, int64_t K, int64_t ldx,
+                                                  const int8_t* signs_dev, uint8_t* codes_dev, void* scales_dev,
+                                                  float* gscale_dev, rq_stream_t stream);
+
 /* Synchronizes `stream`, returns RQ_ERR_TIMEOUT if any kernel of this library
  * recorded a device-side timeout since the last call (and clears the record),
  * RQ_ERR_CUDA if the stream reports an error, else RQ_OK. */

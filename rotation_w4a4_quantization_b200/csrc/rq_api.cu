@@ -202,9 +202,52 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
   return launch_block<kModeNvfp4>(p, st);
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for rq_rotate_quantize_nvfp4_noalloc.  The dynamic NVFP4 scale needs
+// one word of device memory that starts at zero (the max of |X~| is gathered
+// there by atomics); this entry point takes it from this static array instead
+// of a caller-allocated workspace.  Every GPU that loads the library holds
+// these 256 bytes until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[256];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+rq_status noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RQ_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return RQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+rq_status rq_rotate_quantize_nvfp4_noalloc(const void* X_dev, int64_t M, int64_t K, int64_t ldx,
+                                           const int8_t* signs_dev, uint8_t* codes_dev, void* scales_dev,
+                                           float* gscale_dev, rq_stream_t stream) {
+  // The scratch this path needs does not grow with M or K; the check keeps the
+  // static array's stated size honest if that ever changes.
+  if (rq_workspace_bytes(RQ_NVFP4) > sizeof(g_noalloc_scratch)) return RQ_ERR_UNSUPPORTED_SHAPE;
+  rq_status s = check_rotation_args(X_dev, M, K, ldx, signs_dev, 128);
+  if (s != RQ_OK) return s;
+  if (M == 0) return RQ_OK;
+  void* scratch = nullptr;
+  s = noalloc_scratch_address(&scratch);
+  if (s != RQ_OK) return s;
+  // the max word is cleared by the call itself (cudaMemsetAsync on the stream)
+  return rotate_quantize_impl(X_dev, M, K, ldx, signs_dev, 128, RQ_NVFP4, RQ_SCALE_DYNAMIC, codes_dev, scales_dev,
+                              gscale_dev, scratch, static_cast<cudaStream_t>(stream));
+}
 
 const char* rq_status_string(rq_status status) {
   switch (status) {

@@ -21,7 +21,8 @@ RQ_SCALE_DYNAMIC, RQ_SCALE_STATIC = 0, 1
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3: "RQ_ERR_ALIGNMENT",
           4: "RQ_ERR_UNSUPPORTED_DEVICE", 5: "RQ_ERR_CUDA", 6: "RQ_ERR_TIMEOUT"}
 EXPORTED = ["rq_init", "rq_status_string", "rq_workspace_bytes", "rq_rotate_quantize", "rq_prepare_weights",
-            "rq_w4a4_gemm", "rq_kv_rotate_quantize", "rq_rotate_f32", "rq_get_device_error"]
+            "rq_w4a4_gemm", "rq_kv_rotate_quantize", "rq_rotate_f32", "rq_get_device_error",
+            "rq_rotate_quantize_nvfp4_noalloc"]
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("librq.so not built: run `python -m rotation_w4a4_quantization_b200.build`")
@@ -46,6 +47,8 @@ lib.rq_kv_rotate_quantize.argtypes = [_p, _i64, _i64, _i64, _i64, ctypes.POINTER
 lib.rq_kv_rotate_quantize.restype = _i
 lib.rq_rotate_f32.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i64, _p]
 lib.rq_rotate_f32.restype = _i
+lib.rq_rotate_quantize_nvfp4_noalloc.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p]
+lib.rq_rotate_quantize_nvfp4_noalloc.restype = _i
 lib.rq_get_device_error.argtypes = [_p]
 lib.rq_get_device_error.restype = _i
 
@@ -177,6 +180,20 @@ def rotate_f32(x, signs, block=128, out=None):
     _check(lib.rq_rotate_f32(_ptr(x), m, k, x.stride(0), _ptr(signs), int(block), _ptr(out), out.stride(0),
                              _stream(x)), "rq_rotate_f32")
     return out
+
+
+def rotate_quantize_nvfp4_noalloc(x, signs, out=None, gscale=None):
+    """NVFP4 (128-wide blocks, dynamic per-tensor scale) without any device
+    workspace: for callers that cannot allocate device memory.  Returns
+    (codes, scales, gscale) like rotate_quantize; outputs may be passed in."""
+    _require_cuda(x, signs)
+    m, k = x.shape
+    codes, scales = out if out is not None else _alloc_quant_outputs(m, k, RQ_NVFP4, x.device)
+    if gscale is None:
+        gscale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    _check(lib.rq_rotate_quantize_nvfp4_noalloc(_ptr(x), m, k, x.stride(0), _ptr(signs), _ptr(codes), _ptr(scales),
+                                                _ptr(gscale), _stream(x)), "rq_rotate_quantize_nvfp4_noalloc")
+    return codes, scales, gscale
 
 
 def get_device_error(stream=None):
