@@ -71,7 +71,7 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, unsigned parity, int
 template <int ACC_KIND>
 __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tacc, int m0, int n0, int q, int lane,
                                                float rowscale, const float* colscale, float gscale,
-                                               uint64_t* acc_empty) {
+                                               uint64_t* acc_empty, uint32_t acc_empty_cluster = 0) {
   const int row = m0 + 32 * q + lane;
   const bool row_ok = row < p.M;
   const uint32_t tq = tacc + ((uint32_t)(32 * q) << 16);
@@ -148,7 +148,12 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
   }
   tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive(acc_empty);
+  if (lane == 0) {
+    if (acc_empty_cluster)
+      mbar_arrive_cluster(acc_empty_cluster);
+    else
+      mbar_arrive(acc_empty);
+  }
 }
 
 // bf16 epilogue through shared memory: the slab is read out of TMEM in two
@@ -386,6 +391,179 @@ done:
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// INT4 on two SMs (cta_group::2): a cluster of two CTAs computes a 256 x 256
+// tile with one M = 256 MMA per k-step issued by the even CTA.  Each CTA
+// stages and widens its own 128 rows of X and its own 128 of the tile's 256
+// rows of W (so per SM a third less operand data than the one-SM kernel), and
+// holds its 128 x 256 int32 accumulator slab in its own tensor memory.
+// Cross-CTA traffic is only mbarrier arrivals: the converters of both CTAs
+// arrive on the even CTA's operand-ready barrier, the MMA commits multicast to
+// both CTAs, and both epilogues arrive on the even CTA's accumulator-free
+// barrier.
+// ---------------------------------------------------------------------------
+constexpr int kI2Stg = 4, kI2Ops = 4;
+constexpr int kI2StgA = 128 * 64, kI2StgB = 128 * 64;
+constexpr int kI2OpA = 128 * 128, kI2OpB = 128 * 128;
+constexpr size_t kI2Smem = 1024 + (size_t)kI2Stg * (kI2StgA + kI2StgB) + (size_t)kI2Ops * (kI2OpA + kI2OpB) + 256;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI4Threads, 1)
+    gemm_int4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                         const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* op = base;                                            // [kI2Ops][A 16K | B 16K]
+  uint8_t* stg = op + (size_t)kI2Ops * (kI2OpA + kI2OpB);        // [kI2Stg][A 8K | B 8K]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (size_t)kI2Stg * (kI2StgA + kI2StgB));
+  uint64_t* stg_full = bars;
+  uint64_t* stg_empty = stg_full + kI2Stg;
+  uint64_t* op_full = stg_empty + kI2Stg;     // used in the even CTA only
+  uint64_t* op_empty = op_full + kI2Ops;
+  uint64_t* acc_full = op_empty + kI2Ops;
+  uint64_t* acc_empty = acc_full + 2;         // used in the even CTA only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int KT = p.K / kI4BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kI2Stg; ++i) {
+      mbar_init(&stg_full[i], 1);
+      mbar_init(&stg_empty[i], kI4ConvWarps);
+    }
+    for (int i = 0; i < kI2Ops; ++i) {
+      mbar_init(&op_full[i], 2 * kI4ConvWarps);
+      mbar_init(&op_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc_2cta(tmem_slot, 512);
+    tmem_relinquish_2cta();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      unsigned ph = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+        const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
+        const int nb = (tile / p.tiles_m) * 256 + 128 * (int)rank;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&stg_empty[s], ph ^ 1, abort_flag)) goto done;
+          uint8_t* sa = stg + (size_t)s * (kI2StgA + kI2StgB);
+          mbar_arrive_expect_tx(&stg_full[s], kI2StgA + kI2StgB);
+          tma_load_2d(sa, &tmap_x, kt * 64, m0, &stg_full[s]);
+          tma_load_2d(sa + kI2StgA, &tmap_w, kt * 64, nb, &stg_full[s]);
+          if (++s == kI2Stg) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_i8(256, kBN);
+      int o = 0;
+      unsigned oph = 0;
+      int it = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+        const int ab = it & 1;
+        const unsigned aph = (unsigned)((it >> 1) & 1);
+        if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&acc_empty[ab], aph ^ 1)) {
+          *((volatile int*)abort_flag) = 1;
+          goto done;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(ab * kBN);
+        for (int kt = 0; kt < KT; ++kt) {
+          if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&op_full[o], oph)) {
+            *((volatile int*)abort_flag) = 1;
+            goto done;
+          }
+          tc_fence_after();
+          const uint8_t* a = op + (size_t)o * (kI2OpA + kI2OpB);
+          const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kI2OpA);
+#pragma unroll
+          for (int j = 0; j < kI4BK / 32; ++j) mma_i8_2cta(d, ad + 2 * j, bd + 2 * j, idesc, (kt | j) != 0);
+          tc_commit_2cta_mc(&op_empty[o], 0x3);
+          if (++o == kI2Ops) { o = 0; oph ^= 1; }
+        }
+        tc_commit_2cta_mc(&acc_full[ab], 0x3);
+      }
+    }
+  } else if (warp < 2 + kI4ConvWarps) {
+    const int t = threadIdx.x - 64;
+    int s = 0, o = 0;
+    unsigned ph = 0, oph = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!wait_or_fail(&stg_full[s], ph, abort_flag)) goto done;
+        if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
+        const uint8_t* sa = stg + (size_t)s * (kI2StgA + kI2StgB);
+        uint8_t* oa = op + (size_t)o * (kI2OpA + kI2OpB);
+        constexpr int kJobs = 256 * 4, kConvThreads = 32 * kI4ConvWarps;
+#pragma unroll
+        for (int jb = t; jb < kJobs; jb += kConvThreads) {
+          const int r = jb >> 2, j = jb & 3;
+          if (r < 128)
+            convert_chunk(sa, oa, r, j);
+          else
+            convert_chunk(sa + kI2StgA, oa + kI2OpA, r - 128, j);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(mapa_u32(&op_full[o], 0));
+          mbar_arrive(&stg_empty[s]);
+        }
+        if (++s == kI2Stg) { s = 0; ph ^= 1; }
+        if (++o == kI2Ops) { o = 0; oph ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const float* xs = static_cast<const float*>(p.xscale);
+    const float* ws = static_cast<const float*>(p.wscale);
+    int it = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+      const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
+      const int n0 = (tile / p.tiles_m) * kBN;
+      const int ab = it & 1;
+      const unsigned aph = (unsigned)((it >> 1) & 1);
+      if (!wait_or_fail(&acc_full[ab], aph, abort_flag)) goto done;
+      tc_fence_after();
+      const int row = m0 + 32 * q + lane;
+      const float sx = (row < p.M) ? xs[row] : 0.f;
+      epilogue_store<0>(p, tmem + (uint32_t)(ab * kBN), m0, n0, q, lane, sx, ws, 1.0f, &acc_empty[ab],
+                        mapa_u32(&acc_empty[ab], 0));
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // no CTA leaves while the pair's MMAs may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_2cta(tmem, 512);
   }
 }
 
@@ -658,6 +836,27 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
     if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 64, CU_TENSOR_MAP_SWIZZLE_64B))
       return RQ_ERR_CUDA;
+    if (M > kBM) {
+      // two SMs per 256 x 256 tile
+      CUtensorMap tx2, tw2;
+      if (!make_tmap_u8(&tx2, xc, (uint64_t)M, (uint64_t)K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+          !make_tmap_u8(&tw2, wc, (uint64_t)N, (uint64_t)K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+        return RQ_ERR_CUDA;
+      p.tiles_m = (int)((M + 255) / 256);
+      p.tiles_n = (int)((N + kBN - 1) / kBN);
+      p.num_tiles = p.tiles_m * p.tiles_n;
+      const int sms = gemm_num_sms() & ~1;
+      const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
+      static bool attr2_done = false;
+      if (!attr2_done) {
+        if (cudaFuncSetAttribute(gemm_int4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI2Smem) !=
+            cudaSuccess)
+          return RQ_ERR_CUDA;
+        attr2_done = true;
+      }
+      gemm_int4_2sm_kernel<<<grid2, kI4Threads, kI2Smem, st>>>(tx2, tw2, p);
+      return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+    }
     static bool attr_done = false;
     if (!attr_done) {
       if (cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem) !=
