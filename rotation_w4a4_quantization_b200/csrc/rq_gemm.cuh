@@ -164,7 +164,8 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
 // 64 x 128 boxes, `epi_tid` 0..127 the thread's index among the epilogue warps.
 __device__ __forceinline__ void epilogue_bf16_tma(const GemmParams& p, const CUtensorMap* ytmap, uint32_t tacc,
                                                   int m0, int n0, int q, int lane, int epi_tid, float gscale,
-                                                  uint8_t* stage, uint64_t* acc_empty) {
+                                                  uint8_t* stage, uint64_t* acc_empty,
+                                                  uint32_t acc_empty_cluster = 0) {
   const uint32_t tq = tacc + ((uint32_t)(32 * q) << 16);
   const int row = 32 * q + lane;  // row within the tile
 #pragma unroll 1
@@ -196,7 +197,12 @@ __device__ __forceinline__ void epilogue_bf16_tma(const GemmParams& p, const CUt
     if (hh == 1) {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);  // accumulator free for the next tile's MMAs
+      if (lane == 0) {  // accumulator free for the next tile's MMAs
+        if (acc_empty_cluster)
+          mbar_arrive_cluster(acc_empty_cluster);
+        else
+          mbar_arrive(acc_empty);
+      }
     }
     fence_proxy_async_smem();
     named_sync(1, 128);
@@ -739,6 +745,199 @@ done:
 }
 
 // ---------------------------------------------------------------------------
+// NVFP4 on two SMs (cta_group::2, 256 x 256 tiles).  Each CTA loads its own 128
+// rows of X and its own 128 of the tile's 256 rows of W; those copies count on
+// the even CTA's barrier, whose MMA consumes both halves.  Each CTA's scales
+// come by a local copy; its scale warps move them into its own tensor memory,
+// one 32-bit column per 32 rows and 64-wide K slice, replicated in the four
+// lane quadrants: SFA of its own 128 X rows, and SFB of ALL 256 W rows of the
+// tile (each SM's tensor core multiplies its rows by every column of the tile,
+// so it reads the scales of both W halves from its own tensor memory).  Then
+// they arrive on the even CTA's scales-ready barrier.
+// ---------------------------------------------------------------------------
+constexpr int kN2St = 5;
+constexpr int kN2OpA = 128 * 128, kN2OpB = 128 * 128, kN2SfA = 128 * 16, kN2SfB = 256 * 16;
+constexpr int kN2Stage = kN2OpA + kN2OpB + kN2SfA + kN2SfB;       // 38 KB
+constexpr size_t kN2Smem = 1024 + (size_t)kN2St * kN2Stage + kEpiStage + 256;
+constexpr uint32_t kN2SfCols = 48;                                // per stage: SFA 16 + SFB 32 columns
+constexpr int kN2SfWarps = 8;                                     // scale movers (warps 2..9)
+constexpr int kN2Threads = 32 * (2 + kN2SfWarps + 4);
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
+    gemm_nvfp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                          const __grid_constant__ CUtensorMap tmap_sx, const __grid_constant__ CUtensorMap tmap_sw,
+                          const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* op = base;
+  uint8_t* epi_stage = op + (size_t)kN2St * kN2Stage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + kEpiStage);
+  uint64_t* op_full = bars;                 // even CTA: both CTAs' X/W copies
+  uint64_t* op_empty = op_full + kN2St;     // both: multicast MMA commit
+  uint64_t* sf_full = op_empty + kN2St;     // local: this CTA's scale copies
+  uint64_t* sf_ready = sf_full + kN2St;     // even CTA: both CTAs' scales in TMEM
+  uint64_t* acc_full = sf_ready + kN2St;
+  uint64_t* acc_empty = acc_full + 1;       // even CTA: both epilogues
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int KT = p.K / kF4BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kN2St; ++i) {
+      mbar_init(&op_full[i], 1);
+      mbar_init(&op_empty[i], 1);
+      mbar_init(&sf_full[i], 1);
+      mbar_init(&sf_ready[i], 8);  // 4 quadrants x 2 CTAs (one mover warp per quadrant per k-tile)
+    }
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_empty[0], 8);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_sx);
+    prefetch_tmap(&tmap_sw);
+  }
+  if (warp == 1) {
+    tmem_alloc_2cta(tmem_slot, 512);
+    tmem_relinquish_2cta();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      unsigned ph = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+        const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
+        const int nb = (tile / p.tiles_m) * 256 + 128 * (int)rank;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&op_empty[s], ph ^ 1, abort_flag)) goto done;
+          uint8_t* sa = op + (size_t)s * kN2Stage;
+          if (leader) mbar_arrive_expect_tx(&op_full[s], 2 * (kN2OpA + kN2OpB));
+          const uint32_t fb = mapa_u32(&op_full[s], 0);
+          tma_load_2d_2cta(sa, &tmap_x, kt * 128, m0, fb);
+          tma_load_2d_2cta(sa + kN2OpA, &tmap_w, kt * 128, nb, fb);
+          mbar_arrive_expect_tx(&sf_full[s], kN2SfA + kN2SfB);
+          tma_load_2d(sa + kN2OpA + kN2OpB, &tmap_sx, kt * 16, m0, &sf_full[s]);
+          tma_load_2d(sa + kN2OpA + kN2OpB + kN2SfA, &tmap_sw, kt * 16, nb - 128 * (int)rank, &sf_full[s]);
+          if (++s == kN2St) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_nvf4(256, kBN);
+      int s = 0;
+      unsigned ph = 0;
+      int it = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+        if (!wait_or_fail(&acc_empty[0], (unsigned)(it & 1) ^ 1, abort_flag)) goto done;
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&op_full[s], ph, abort_flag)) goto done;
+          if (!wait_or_fail(&sf_ready[s], ph, abort_flag)) goto done;
+          tc_fence_after();
+          const uint8_t* a = op + (size_t)s * kN2Stage;
+          const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kN2OpA);
+          const uint32_t sf = tmem + kF4SfCol0 + (uint32_t)s * kN2SfCols;
+#pragma unroll
+          for (int j = 0; j < kF4BK / 64; ++j)
+            mma_nvf4_2cta(tmem, ad + 2 * j, bd + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (kt | j) != 0);
+          tc_commit_2cta_mc(&op_empty[s], 0x3);
+          if (++s == kN2St) { s = 0; ph ^= 1; }
+        }
+        tc_commit_2cta_mc(&acc_full[0], 0x3);
+      }
+    }
+  } else if (warp < 2 + kN2SfWarps) {
+    // scale movers: two warps per lane quadrant take alternate k-tiles
+    const int q = warp & 3;
+    const int par = (warp - 2) >> 2;
+    int s = 0;
+    unsigned ph = 0;
+    int n = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+      for (int kt = 0; kt < KT; ++kt, ++n) {
+        if ((n & 1) != par) {
+          if (++s == kN2St) { s = 0; ph ^= 1; }
+          continue;
+        }
+        // the scale copy of this round follows the producer's wait on op_empty, so
+        // the MMAs of the previous round (which read these columns) are done
+        if (!wait_or_fail(&sf_full[s], ph, abort_flag)) goto done;
+        const uint8_t* sfa = op + (size_t)s * kN2Stage + kN2OpA + kN2OpB;
+        const uint8_t* sfb = sfa + kN2SfA;
+        uint4 ua[4], ub[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ua[i] = *reinterpret_cast<const uint4*>(sfa + (lane + 32 * i) * 16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ub[i] = *reinterpret_cast<const uint4*>(sfb + (lane + 32 * i) * 16);
+        tc_fence_after();
+        uint32_t da[16], db0[16], db1[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) da[4 * j + i] = reinterpret_cast<const uint32_t*>(&ua[i])[j];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = 8 * j + i;
+            if (c < 16)
+              db0[c] = reinterpret_cast<const uint32_t*>(&ub[i])[j];
+            else
+              db1[c - 16] = reinterpret_cast<const uint32_t*>(&ub[i])[j];
+          }
+        }
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + kF4SfCol0 + (uint32_t)s * kN2SfCols;
+        tmem_st16(tq, da);
+        tmem_st16(tq + 16, db0);
+        tmem_st16(tq + 32, db1);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_u32(&sf_ready[s], 0));
+        if (++s == kN2St) { s = 0; ph ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const float g = (*p.xg) * (*p.wg);
+    int it = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+      const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
+      const int n0 = (tile / p.tiles_m) * kBN;
+      if (!wait_or_fail(&acc_full[0], (unsigned)(it & 1), abort_flag)) goto done;
+      tc_fence_after();
+      const uint32_t ae = mapa_u32(&acc_empty[0], 0);
+      if (p.tma_store)
+        epilogue_bf16_tma(p, &tmap_y, tmem, m0, n0, q, lane, threadIdx.x - 32 * (2 + kN2SfWarps), g, epi_stage,
+                          &acc_empty[0], ae);
+      else
+        epilogue_store<1>(p, tmem, m0, n0, q, lane, 1.0f, nullptr, g, &acc_empty[0], ae);
+    }
+  }
+done:
+  if (threadIdx.x == 32 * (2 + kN2SfWarps)) bulk_wait0();
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_2cta(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -870,6 +1069,28 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
     std::memset(&ty, 0, sizeof(ty));
     p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
     if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
+    if (M > kBM) {
+      // two SMs per 256 x 256 tile
+      if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !make_tmap_u8(&tsx, xs, (uint64_t)M, (uint64_t)K / 16, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+          !make_tmap_u8(&tsw, ws, (uint64_t)N, (uint64_t)K / 16, 256, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return RQ_ERR_CUDA;
+      p.tiles_m = (int)((M + 255) / 256);
+      p.tiles_n = (int)((N + kBN - 1) / kBN);
+      p.num_tiles = p.tiles_m * p.tiles_n;
+      const int sms = gemm_num_sms() & ~1;
+      const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
+      static bool attr2_done = false;
+      if (!attr2_done) {
+        if (cudaFuncSetAttribute(gemm_nvfp4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kN2Smem) != cudaSuccess)
+          return RQ_ERR_CUDA;
+        attr2_done = true;
+      }
+      gemm_nvfp4_2sm_kernel<<<grid2, kN2Threads, kN2Smem, st>>>(tx, tw, tsx, tsw, ty, p);
+      return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+    }
     if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_u8(&tsx, xs, (uint64_t)M, (uint64_t)K / 16, kBM, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
