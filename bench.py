@@ -20,7 +20,6 @@ collective) and the time is the max over ranks.
 import argparse
 import json
 import os
-import subprocess
 import sys
 import time
 
@@ -41,7 +40,7 @@ DEFAULT_WORKLOAD = "q_proj_int4"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -58,6 +57,41 @@ def load_peaks():
         return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
                     bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# ncu captures summarised in profiles/, with a fingerprint of the kernel sources
+# they were taken on; a number is reported only while those sources are
+# unchanged.  kv4 was captured on a quarter of one tensor and is scaled by the
+# vectors processed; q_proj_nvfp4 is the mean of its two launches (max pass,
+# quantize pass).
+ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
+GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
+TRAFFIC = {
+    ("hadamard_quant", "q_proj_int4"): (16846848, "6171dfa5d6c3486c"),
+    ("hadamard_quant", "down_proj_int4"): (100730880 + 4858368, "6171dfa5d6c3486c"),
+    ("hadamard_quant", "kv4"): ((134337280 + 12498688) * 4, "6171dfa5d6c3486c"),
+    ("hadamard_quant", "q_proj_nvfp4"): ((16825600 + 16836608) // 2, "6171dfa5d6c3486c"),
+    ("gemm", "q_proj_int4"): (12637696 + 8704, "046b718da8bfd820"),
+    ("gemm", "down_proj_int4"): (50567424 + 8494592, "046b718da8bfd820"),
+}
+
+
+def source_fingerprint(files):
+    import hashlib
+    m = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "rotation_w4a4_quantization_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def traffic(kind, workload):
+    entry = TRAFFIC.get((kind, workload))
+    if entry is None:
+        return None
+    files = ROTATE_SOURCES if kind == "hadamard_quant" else GEMM_SOURCES
+    return entry[0] if source_fingerprint(files) == entry[1] else None
 
 
 # --------------------------------------------------------------------------- workload
@@ -132,52 +166,65 @@ class Workload:
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML
+    from a background thread every ~2 ms while the timed region runs (read-only;
+    nothing is changed on the GPU)."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.path = os.path.join("/tmp", "rq_clocks_%d_%d.csv" % (os.getpid(), index))
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = False
+        self._thread = None
 
     def start(self):
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:  # NVML numbers GPUs physically; find ours by PCI bus id
+                pr = torch.cuda.get_device_properties(self.index)
+                bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
+            self._thread = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop:
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS:
+                    if r & getattr(nv, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [t.strip() for t in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    mhz.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
-                    continue
-                for nm, val in zip(names, parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        if not mhz:
+        self._stop = True
+        self._thread.join(timeout=2)
+        if not self.samples:
             return None
-        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
 
 
 # --------------------------------------------------------------------------- CPU oracle leg
@@ -332,8 +379,8 @@ def main():
     }
     q_launch_ms = q_mean_ms / wl.quant_launches()
     roof_q = {"bound": "hbm", "achieved": round(wl.quant_bytes / wl.quant_launches() / (q_launch_ms * 1e-3) / 1e9, 1),
-              "peak": peaks["hbm"], "unit": "GB/s", "traffic": None,
-              "kernel": "rotate_full_kernel" if (not wl.kv and wl.block == 0) else "rotate_block_kernel",
+              "peak": peaks["hbm"], "unit": "GB/s", "traffic": traffic("hadamard_quant", args.workload),
+              "kernel": "rotate_kernel<full width>" if (not wl.kv and wl.block == 0) else "rotate_kernel<128-blocks>",
               "peak_source": peaks["src"]}
     roof_q["frac"] = round(roof_q["achieved"] / roof_q["peak"], 4)
     if wl.gemm_launches():
@@ -342,9 +389,10 @@ def main():
             ratio = 4.0
         tops = wl.gemm_ops * world / (g_mean_ms * 1e-3) / 1e12
         peak_t = peaks["bf16"] * ratio
+        two_sm = wl.cfg["M"] > 128
         roof_g = {"bound": "tensor", "achieved": round(wl.gemm_ops / (g_mean_ms * 1e-3) / 1e12, 1), "peak": peak_t,
-                  "unit": "TFLOP/s", "traffic": None,
-                  "kernel": "gemm_int4_kernel" if wl.fmt == "int4" else "gemm_nvfp4_kernel",
+                  "unit": "TFLOP/s", "traffic": traffic("gemm", args.workload),
+                  "kernel": ("gemm_int4" if wl.fmt == "int4" else "gemm_nvfp4") + ("_2sm_kernel" if two_sm else "_kernel"),
                   "peak_source": "%s bf16 x %g (nominal %s/bf16 ratio)" % (peaks["src"], ratio,
                                                                            "int8" if ratio == 2 else "fp4")}
         roof_g["frac"] = round(roof_g["achieved"] / peak_t, 4)
