@@ -138,10 +138,26 @@ class Workload:
             self.h2d_bytes = self.x.numel() * 2
         self.d2h_bytes = 0
 
+    def nvfp4_one_pass(self):
+        # librq quantizes dynamic NVFP4 in one launch when each SM's share of
+        # the rows (plus the sign table) fits its 220 KiB of shared memory;
+        # otherwise a max launch precedes the quantize launch
+        m, k = self.cfg["M"], self.cfg["K"]
+        sms = torch.cuda.get_device_properties(self.x.device).multi_processor_count
+        rpc = -(-m // sms)
+        return rpc * k * 2 + (k // 128) * 256 + 32 <= 220 * 1024
+
     def quant_launches(self):
         if self.kv:
             return 2
-        return 2 if self.fmt == "nvfp4" else 1
+        if self.fmt == "nvfp4":
+            return 1 if self.nvfp4_one_pass() else 2
+        return 1
+
+    def quant_kernel(self):
+        if self.fmt == "nvfp4" and self.nvfp4_one_pass():
+            return "rotate_nvfp4_resident_kernel"
+        return "rotate_kernel<full width>" if (not self.kv and self.block == 0) else "rotate_kernel<128-blocks>"
 
     def gemm_launches(self):
         return 0 if self.kv else 1
@@ -380,7 +396,7 @@ def main():
     q_launch_ms = q_mean_ms / wl.quant_launches()
     roof_q = {"bound": "hbm", "achieved": round(wl.quant_bytes / wl.quant_launches() / (q_launch_ms * 1e-3) / 1e9, 1),
               "peak": peaks["hbm"], "unit": "GB/s", "traffic": traffic("hadamard_quant", args.workload),
-              "kernel": "rotate_kernel<full width>" if (not wl.kv and wl.block == 0) else "rotate_kernel<128-blocks>",
+              "kernel": wl.quant_kernel(),
               "peak_source": peaks["src"]}
     roof_q["frac"] = round(roof_q["achieved"] / roof_q["peak"], 4)
     if wl.gemm_launches():

@@ -129,6 +129,43 @@ rq_status launch_full(RotParams p, cudaStream_t st) {
   }
 }
 
+// Dynamic NVFP4 in one pass (rotate_nvfp4_resident_kernel): every CTA keeps its
+// rows in shared memory; needs all CTAs resident (cooperative launch).  Returns
+// RQ_ERR_UNSUPPORTED_SHAPE (nothing launched) when the rows do not fit.
+rq_status launch_nvfp4_resident(RotParams p, cudaStream_t st) {
+  int dev = 0, coop = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop)
+    return RQ_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms_of_current_device();
+  const int64_t rpc = (p.rows + sms - 1) / sms;
+  const size_t smem = (size_t)rpc * p.K * 2 + (size_t)p.nb * 64 * 4 + 32;
+  if (smem > kSmemBudget) return RQ_ERR_UNSUPPORTED_SHAPE;
+  const int grid = (int)((p.rows + rpc - 1) / rpc);
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel))) return RQ_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_nvfp4_resident_kernel, 384, smem) !=
+          cudaSuccess ||
+      per_sm < 1 || grid > per_sm * sms)
+    return RQ_ERR_UNSUPPORTED_SHAPE;
+  p.nvfp4_dynamic = 1;
+  int rows_per_cta = (int)rpc;
+  void* args[] = {&p, &rows_per_cta};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(384);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel), args) != cudaSuccess)
+    return RQ_ERR_CUDA;
+  return RQ_OK;
+}
+
 // Common checks of the X / K / signs / block arguments.
 // Pointers are only required (and checked) when there is work: M = 0 is a no-op.
 rq_status check_rotation_args(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* signs, int block) {
@@ -190,7 +227,11 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
   p.scales_e4m3 = static_cast<uint8_t*>(scales);
   if (gmode == RQ_SCALE_DYNAMIC) {
     p.amax_word = static_cast<unsigned*>(workspace);
-    if (cudaMemsetAsync(workspace, 0, sizeof(unsigned), st) != cudaSuccess) return RQ_ERR_CUDA;
+    p.g_out = gscale;
+    if (cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned), st) != cudaSuccess) return RQ_ERR_CUDA;
+    // one pass over HBM when the whole tensor fits in the SMs' shared memory
+    s = launch_nvfp4_resident(p, st);
+    if (s != RQ_ERR_UNSUPPORTED_SHAPE) return s;
     s = launch_block<kModeAmax>(p, st);
     if (s != RQ_OK) return s;
     p.nvfp4_dynamic = 1;

@@ -650,4 +650,116 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
   }
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 with the dynamic per-tensor scale in ONE pass over HBM, for tensors that
+// fit in the SMs' combined shared memory: a cooperative launch (all CTAs
+// resident) where each CTA copies its rows into shared memory once, computes
+// the max |X~| of its rows, meets the other CTAs at a grid-wide barrier
+// (atomic counter, bounded spin), and then rotates its rows again from shared
+// memory and quantizes them with g = max/(6*448).
+// p.amax_word[0] gathers the max, p.amax_word[1] counts arrivals; both are
+// zeroed by the host before the launch.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const RotParams p, int rows_per_cta) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const int nb = p.nb;
+  const int64_t r0 = (int64_t)blockIdx.x * rows_per_cta;
+  const int nrows = (int)max((int64_t)0, min((int64_t)rows_per_cta, p.rows - r0));
+  const size_t row_bytes = (size_t)p.K * 2;
+  uint8_t* rows = smem_raw;
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw + (size_t)rows_per_cta * row_bytes);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smask + nb * 64);
+  unsigned* cta_max = reinterpret_cast<unsigned*>(bar + 1);
+  int* flag = reinterpret_cast<int*>(cta_max + 1);
+  const int tid = threadIdx.x;
+  const int m = tid & 7;
+  const float c = 0.08838834764831845f;  // 1/sqrt(128), rounded once
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    *cta_max = 0u;
+  }
+  __syncthreads();
+  if (tid == 0 && nrows > 0) {
+    mbar_arrive_expect_tx(bar, (unsigned)(nrows * row_bytes));
+    if (p.contiguous) {  // the CTA's rows are one span of at most the shared-memory budget
+      bulk_g2s(rows, p.x + r0 * (int64_t)row_bytes, (unsigned)(nrows * row_bytes), bar);
+    } else {
+      for (int rr = 0; rr < nrows; ++rr)
+        bulk_g2s(rows + (size_t)rr * row_bytes, p.x + (r0 + rr) * p.sS, (unsigned)row_bytes, bar);
+    }
+  }
+  for (int i = tid; i < nb * 8; i += blockDim.x) {
+    const uint4 sg = __ldg(reinterpret_cast<const uint4*>(p.signs) + i);
+    const uint32_t w[4] = {sg.x, sg.y, sg.z, sg.w};
+    uint32_t mk[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t neg = w[j] & 0x80808080u;
+      mk[2 * j] = ((neg & 0x80u) << 8) | ((neg & 0x8000u) << 16);
+      mk[2 * j + 1] = ((neg & 0x800000u) >> 8) | (neg & 0x80000000u);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(smask + 8 * i);
+    dst[0] = make_uint4(mk[0], mk[1], mk[2], mk[3]);
+    dst[1] = make_uint4(mk[4], mk[5], mk[6], mk[7]);
+  }
+  if (tid == 0) *flag = (nrows == 0 || mbar_wait_bounded(bar, 0)) ? 1 : 0;
+  __syncthreads();
+  const bool loaded = *flag != 0;
+
+  // pass 1: max |X~| over this CTA's rows
+  const int units = nrows * nb;
+  float amax = 0.f;
+  if (loaded) {
+    for (int u = tid; u < units; u += blockDim.x) {
+      const int r = u / nb, b = u - r * nb;
+      float v[128];
+      load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+      fwht128(v);
+      amax = fmaxf(amax, absmax128(v) * c);
+    }
+  }
+  const unsigned wbits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
+  if ((tid & 31) == 0) atomicMax(cta_max, wbits);
+  __syncthreads();
+
+  // grid-wide barrier: publish this CTA's max, count arrivals, wait for all
+  volatile unsigned* gmax = p.amax_word;
+  volatile unsigned* count = p.amax_word + 1;
+  if (tid == 0) {
+    atomicMax(p.amax_word, *cta_max);
+    __threadfence();
+    atomicAdd(p.amax_word + 1, 1u);
+    bool ok = true;
+    const long long t0 = clock64();
+    while (*count < gridDim.x) {
+      __nanosleep(64);
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+        ok = false;
+        break;
+      }
+    }
+    __threadfence();
+    *flag = (ok && loaded) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!*flag) return;
+
+  // pass 2: quantize with the tensor's scale
+  const float g = __fdiv_rn(__uint_as_float(*gmax), 2688.0f);
+  const float inv6g = g > 0.f ? __frcp_rn(6.0f * g) : 0.0f;
+  if (blockIdx.x == 0 && tid == 0 && p.g_out) *p.g_out = g;
+  for (int u = tid; u < units; u += blockDim.x) {
+    const int r = u / nb, b = u - r * nb;
+    const int64_t row = r0 + r;
+    float v[128];
+    load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+    fwht128(v);
+    quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                      p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+  }
+}
+
 }  // namespace rq

@@ -136,6 +136,32 @@ def test_nvfp4_rotate_quantize_dynamic(rq, m, k):
     parity.check_nvfp4_quant(parity.to_np(codes), parity.to_np(sc), parity.to_np(g)[0], xr)
 
 
+def test_nvfp4_dynamic_strided_rows(rq):
+    # rows ldx = K + 256 apart: the one-pass kernel copies them row by row
+    m, k = 300, 4096
+    big = _gauss(m, k + 256, 91, outliers=[(7, 25.0)])
+    x = big.cuda()[:, :k]
+    s = _signs(k, 92)
+    codes, sc, g = rq.rotate_quantize(x, s.cuda(), 128, "nvfp4", "dynamic")
+    xr = hadamard.rotate(parity.bf16_to_f64(big[:, :k]), s.numpy(), 128)
+    parity.check_nvfp4_quant(parity.to_np(codes), parity.to_np(sc), parity.to_np(g)[0], xr)
+
+
+def test_nvfp4_dynamic_larger_than_shared_memory(rq):
+    # 4100 x 4096 bf16 (33.6 MB) exceeds what the SMs' shared memory holds at
+    # once, so the max pass and the quantize pass stream X from HBM twice;
+    # the scale is checked against the whole tensor, the codes on sampled rows
+    m, k = 4100, 4096
+    x = _gauss(m, k, 93, outliers=[(100, 40.0)])
+    s = _signs(k, 94)
+    codes, sc, g = rq.rotate_quantize(x.cuda(), s.cuda(), 128, "nvfp4", "dynamic")
+    xr = hadamard.rotate(parity.bf16_to_f64(x), s.numpy(), 128)
+    g_o = quant.nvfp4_global_scale(xr)
+    assert abs(float(parity.to_np(g)[0]) - float(g_o)) <= parity.SCALE_RTOL * float(g_o)
+    rows = np.unique(np.concatenate([np.arange(0, m, 67), [m - 1]]))
+    parity.check_nvfp4_quant(parity.to_np(codes)[rows], parity.to_np(sc)[rows], None, xr[rows], g_ref=g_o)
+
+
 def test_nvfp4_static_scale(rq):
     m, k = 300, 1024
     x = _gauss(m, k, 55)
