@@ -126,6 +126,45 @@ __device__ __forceinline__ void issue_tile_load(const RotParams& p, int64_t tile
 }
 
 
+// 16 int8 signs (+1 / -1) -> 8 XOR masks, one per bf16 pair (bit 15 / bit 31).
+__device__ __forceinline__ void sign_masks16(const uint4 sg, uint32_t* dst) {
+  const uint32_t w[4] = {sg.x, sg.y, sg.z, sg.w};
+  uint32_t mk[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // byte k of w[j] is the sign of channel 4j + k; negative <=> bit 7 set
+    const uint32_t neg = w[j] & 0x80808080u;
+    mk[2 * j] = ((neg & 0x80u) << 8) | ((neg & 0x8000u) << 16);
+    mk[2 * j + 1] = ((neg & 0x800000u) >> 8) | (neg & 0x80000000u);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(mk[0], mk[1], mk[2], mk[3]);
+  d[1] = make_uint4(mk[4], mk[5], mk[6], mk[7]);
+}
+
+// Build the CTA's sign-mask table (nb*64 words) from the K signs.  The first
+// (up to 2 per thread) sign loads are issued before `issue` runs -- the
+// caller's first tile copies -- so they do not queue behind those copies; the
+// conversion follows.
+template <typename IssueFn>
+__device__ __forceinline__ void build_sign_table(const int8_t* signs, int nb, uint32_t* smask, IssueFn issue) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(signs);
+  const int n = nb * 8;
+  uint4 sg[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = threadIdx.x + k * blockDim.x;
+    if (i < n) sg[k] = __ldg(s4 + i);
+  }
+  issue();
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = threadIdx.x + k * blockDim.x;
+    if (i < n) sign_masks16(sg[k], smask + 8 * i);
+  }
+  for (int i = threadIdx.x + 2 * blockDim.x; i < n; i += blockDim.x) sign_masks16(__ldg(s4 + i), smask + 8 * i);
+}
+
 // 128-point fast Walsh-Hadamard transform in registers (unnormalized).
 __device__ __forceinline__ void fwht128(float (&v)[128]) {
 #pragma unroll
@@ -511,27 +550,13 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
     fence_mbar_init();
   }
   __syncthreads();
-  if (producer) {  // start streaming before anything else
-    int64_t tile = gg;
-    for (int st = 0; st < p.stages && tile < p.num_tiles; ++st, tile += TG)
-      issue_tile_load(p, tile, ring + st * sbytes, &full[st]);
-  }
-  // sign-mask table, 16 signs (8 masks) per thread and pass, while the copies fly
-  for (int i = threadIdx.x; i < nb * 8; i += blockDim.x) {
-    const uint4 sg = __ldg(reinterpret_cast<const uint4*>(p.signs) + i);
-    const uint32_t w[4] = {sg.x, sg.y, sg.z, sg.w};
-    uint32_t mk[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      // byte k of w[j] is the sign of channel 16i + 4j + k; negative <=> bit 7 set
-      const uint32_t neg = w[j] & 0x80808080u;
-      mk[2 * j] = ((neg & 0x80u) << 8) | ((neg & 0x8000u) << 16);
-      mk[2 * j + 1] = ((neg & 0x800000u) >> 8) | (neg & 0x80000000u);
+  build_sign_table(p.signs, nb, smask, [&]() {
+    if (producer) {  // the first tile copies of this group
+      int64_t tile = gg;
+      for (int st = 0; st < p.stages && tile < p.num_tiles; ++st, tile += TG)
+        issue_tile_load(p, tile, ring + st * sbytes, &full[st]);
     }
-    uint4* dst = reinterpret_cast<uint4*>(smask + 8 * i);
-    dst[0] = make_uint4(mk[0], mk[1], mk[2], mk[3]);
-    dst[1] = make_uint4(mk[4], mk[5], mk[6], mk[7]);
-  }
+  });
   __syncthreads();
 
   float g = 0.f, inv6g = 0.f;
@@ -681,29 +706,17 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
     *cta_max = 0u;
   }
   __syncthreads();
-  if (tid == 0 && nrows > 0) {
-    mbar_arrive_expect_tx(bar, (unsigned)(nrows * row_bytes));
-    if (p.contiguous) {  // the CTA's rows are one span of at most the shared-memory budget
-      bulk_g2s(rows, p.x + r0 * (int64_t)row_bytes, (unsigned)(nrows * row_bytes), bar);
-    } else {
-      for (int rr = 0; rr < nrows; ++rr)
-        bulk_g2s(rows + (size_t)rr * row_bytes, p.x + (r0 + rr) * p.sS, (unsigned)row_bytes, bar);
+  build_sign_table(p.signs, nb, smask, [&]() {
+    if (tid == 0 && nrows > 0) {
+      mbar_arrive_expect_tx(bar, (unsigned)(nrows * row_bytes));
+      if (p.contiguous) {  // the CTA's rows are one span of at most the shared-memory budget
+        bulk_g2s(rows, p.x + r0 * (int64_t)row_bytes, (unsigned)(nrows * row_bytes), bar);
+      } else {
+        for (int rr = 0; rr < nrows; ++rr)
+          bulk_g2s(rows + (size_t)rr * row_bytes, p.x + (r0 + rr) * p.sS, (unsigned)row_bytes, bar);
+      }
     }
-  }
-  for (int i = tid; i < nb * 8; i += blockDim.x) {
-    const uint4 sg = __ldg(reinterpret_cast<const uint4*>(p.signs) + i);
-    const uint32_t w[4] = {sg.x, sg.y, sg.z, sg.w};
-    uint32_t mk[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t neg = w[j] & 0x80808080u;
-      mk[2 * j] = ((neg & 0x80u) << 8) | ((neg & 0x8000u) << 16);
-      mk[2 * j + 1] = ((neg & 0x800000u) >> 8) | (neg & 0x80000000u);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(smask + 8 * i);
-    dst[0] = make_uint4(mk[0], mk[1], mk[2], mk[3]);
-    dst[1] = make_uint4(mk[4], mk[5], mk[6], mk[7]);
-  }
+  });
   if (tid == 0) *flag = (nrows == 0 || mbar_wait_bounded(bar, 0)) ? 1 : 0;
   __syncthreads();
   const bool loaded = *flag != 0;
