@@ -408,7 +408,8 @@ def main():
         two_sm = wl.cfg["M"] > 128
         roof_g = {"bound": "tensor", "achieved": round(wl.gemm_ops / (g_mean_ms * 1e-3) / 1e12, 1), "peak": peak_t,
                   "unit": "TFLOP/s", "traffic": traffic("gemm", args.workload),
-                  "kernel": ("gemm_int4" if wl.fmt == "int4" else "gemm_nvfp4") + ("_2sm_kernel" if two_sm else "_kernel"),
+                  "kernel": ("gemm_int4" if wl.fmt == "int4" else "gemm_nvfp4") +
+                            (("_2sm_ts_kernel" if wl.fmt == "int4" else "_2sm_kernel") if two_sm else "_kernel"),
                   "peak_source": "%s bf16 x %g (nominal %s/bf16 ratio)" % (peaks["src"], ratio,
                                                                            "int8" if ratio == 2 else "fp4")}
         roof_g["frac"] = round(roof_g["achieved"] / peak_t, 4)

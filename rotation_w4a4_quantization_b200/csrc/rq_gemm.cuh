@@ -8,11 +8,11 @@
 //
 // INT4 path (kind::i8).  Blackwell has no 4-bit x 4-bit integer MMA (the
 // SpinQuant and QuaRot pages make the same point about earlier hardware), so
-// the packed nibbles are widened to int8 in shared memory.  Each nibble q is
-// placed in the HIGH half of its byte (the byte is 16*q, exact in int8), which
-// needs only a mask and a byte permute per four codes; the MMA then
-// accumulates 256 * sum(qx*qw) exactly in int32 (|acc| <= 2^14 K < 2^31 for
-// K <= 65536) and the epilogue shifts right by 8.
+// the packed nibbles are widened to int8: W in shared memory, X (M > 128) in
+// tensor memory.  Each nibble q is placed in the HIGH half of its byte (the
+// byte is 16*q, exact in int8), which needs only a mask and a byte permute
+// per four codes; the MMA then accumulates 256 * sum(qx*qw) exactly in int32
+// (|acc| <= 2^14 K < 2^31 for K <= 65536) and the epilogue shifts right by 8.
 //
 // NVFP4 path (kind::mxf4nvf4, block16).  E2M1 codes go by TMA straight into
 // 128B-swizzled shared memory; the E4M3 block scales are written into tensor
@@ -20,12 +20,16 @@
 // 64-wide K slice, row r's four scales sit in lane (r mod 32) of every lane
 // quadrant, column r/32.
 //
-// Both kernels are persistent (one CTA per SM) and warp-specialized:
-//   warp 0      TMA producer (one elected lane)
-//   warp 1      TMEM allocator + MMA issuer (one elected lane)
-//   warps 2-5   INT4: nibble -> int8 converters;  NVFP4: scale loaders
-//   warps 6-9   epilogue: TMEM -> registers -> scale -> global
-// CTA tile 128 x 256 (M x N), accumulators in TMEM (int32 or fp32).
+// All kernels are persistent and warp-specialized: warp 0 is the TMA
+// producer, warp 1 allocates TMEM and issues the MMAs, converter / scale-mover
+// warps feed the operands, and epilogue warps drain the accumulators
+// (TMEM -> registers -> scale -> global, through shared memory and TMA for
+// bf16).  For M <= 128 one SM computes a 128 x 256 tile; above that two SMs
+// (cta_group::2) share one M = 256 MMA per K step of a 256 x 256 tile: each
+// CTA holds its own 128 rows of X and 128 of the tile's rows of W, the
+// operand-ready arrivals of both CTAs go to the even CTA, the MMA commits
+// multicast to both, and both epilogues arrive on the even CTA's
+// accumulator-free barrier.
 #pragma once
 
 #include <cuda.h>
@@ -401,179 +405,6 @@ done:
 }
 
 // ---------------------------------------------------------------------------
-// INT4 on two SMs (cta_group::2): a cluster of two CTAs computes a 256 x 256
-// tile with one M = 256 MMA per k-step issued by the even CTA.  Each CTA
-// stages and widens its own 128 rows of X and its own 128 of the tile's 256
-// rows of W (so per SM a third less operand data than the one-SM kernel), and
-// holds its 128 x 256 int32 accumulator slab in its own tensor memory.
-// Cross-CTA traffic is only mbarrier arrivals: the converters of both CTAs
-// arrive on the even CTA's operand-ready barrier, the MMA commits multicast to
-// both CTAs, and both epilogues arrive on the even CTA's accumulator-free
-// barrier.
-// ---------------------------------------------------------------------------
-constexpr int kI2Stg = 4, kI2Ops = 4;
-constexpr int kI2StgA = 128 * 64, kI2StgB = 128 * 64;
-constexpr int kI2OpA = 128 * 128, kI2OpB = 128 * 128;
-constexpr size_t kI2Smem = 1024 + (size_t)kI2Stg * (kI2StgA + kI2StgB) + (size_t)kI2Ops * (kI2OpA + kI2OpB) + 256;
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI4Threads, 1)
-    gemm_int4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                         const GemmParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* op = base;                                            // [kI2Ops][A 16K | B 16K]
-  uint8_t* stg = op + (size_t)kI2Ops * (kI2OpA + kI2OpB);        // [kI2Stg][A 8K | B 8K]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (size_t)kI2Stg * (kI2StgA + kI2StgB));
-  uint64_t* stg_full = bars;
-  uint64_t* stg_empty = stg_full + kI2Stg;
-  uint64_t* op_full = stg_empty + kI2Stg;     // used in the even CTA only
-  uint64_t* op_empty = op_full + kI2Ops;
-  uint64_t* acc_full = op_empty + kI2Ops;
-  uint64_t* acc_empty = acc_full + 2;         // used in the even CTA only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int KT = p.K / kI4BK;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kI2Stg; ++i) {
-      mbar_init(&stg_full[i], 1);
-      mbar_init(&stg_empty[i], kI4ConvWarps);
-    }
-    for (int i = 0; i < kI2Ops; ++i) {
-      mbar_init(&op_full[i], 2 * kI4ConvWarps);
-      mbar_init(&op_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 8);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-    prefetch_tmap(&tmap_x);
-    prefetch_tmap(&tmap_w);
-  }
-  if (warp == 1) {
-    tmem_alloc_2cta(tmem_slot, 512);
-    tmem_relinquish_2cta();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();  // both CTAs' barriers exist before any remote arrival
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int s = 0;
-      unsigned ph = 0;
-      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
-        const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
-        const int nb = (tile / p.tiles_m) * 256 + 128 * (int)rank;
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!wait_or_fail(&stg_empty[s], ph ^ 1, abort_flag)) goto done;
-          uint8_t* sa = stg + (size_t)s * (kI2StgA + kI2StgB);
-          mbar_arrive_expect_tx(&stg_full[s], kI2StgA + kI2StgB);
-          tma_load_2d(sa, &tmap_x, kt * 64, m0, &stg_full[s]);
-          tma_load_2d(sa + kI2StgA, &tmap_w, kt * 64, nb, &stg_full[s]);
-          if (++s == kI2Stg) { s = 0; ph ^= 1; }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_i8(256, kBN);
-      int o = 0;
-      unsigned oph = 0;
-      int it = 0;
-      for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
-        const int ab = it & 1;
-        const unsigned aph = (unsigned)((it >> 1) & 1);
-        if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&acc_empty[ab], aph ^ 1)) {
-          *((volatile int*)abort_flag) = 1;
-          goto done;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(ab * kBN);
-        for (int kt = 0; kt < KT; ++kt) {
-          if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&op_full[o], oph)) {
-            *((volatile int*)abort_flag) = 1;
-            goto done;
-          }
-          tc_fence_after();
-          const uint8_t* a = op + (size_t)o * (kI2OpA + kI2OpB);
-          const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kI2OpA);
-#pragma unroll
-          for (int j = 0; j < kI4BK / 32; ++j) mma_i8_2cta(d, ad + 2 * j, bd + 2 * j, idesc, (kt | j) != 0);
-          tc_commit_2cta_mc(&op_empty[o], 0x3);
-          if (++o == kI2Ops) { o = 0; oph ^= 1; }
-        }
-        tc_commit_2cta_mc(&acc_full[ab], 0x3);
-      }
-    }
-  } else if (warp < 2 + kI4ConvWarps) {
-    const int t = threadIdx.x - 64;
-    int s = 0, o = 0;
-    unsigned ph = 0, oph = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
-      for (int kt = 0; kt < KT; ++kt) {
-        if (!wait_or_fail(&stg_full[s], ph, abort_flag)) goto done;
-        if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
-        const uint8_t* sa = stg + (size_t)s * (kI2StgA + kI2StgB);
-        uint8_t* oa = op + (size_t)o * (kI2OpA + kI2OpB);
-        constexpr int kJobs = 256 * 4, kConvThreads = 32 * kI4ConvWarps;
-#pragma unroll
-        for (int jb = t; jb < kJobs; jb += kConvThreads) {
-          const int r = jb >> 2, j = jb & 3;
-          if (r < 128)
-            convert_chunk(sa, oa, r, j);
-          else
-            convert_chunk(sa + kI2StgA, oa + kI2OpA, r - 128, j);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_cluster(mapa_u32(&op_full[o], 0));
-          mbar_arrive(&stg_empty[s]);
-        }
-        if (++s == kI2Stg) { s = 0; ph ^= 1; }
-        if (++o == kI2Ops) { o = 0; oph ^= 1; }
-      }
-    }
-  } else {
-    const int q = warp & 3;
-    const float* xs = static_cast<const float*>(p.xscale);
-    const float* ws = static_cast<const float*>(p.wscale);
-    int it = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
-      const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
-      const int n0 = (tile / p.tiles_m) * kBN;
-      const int ab = it & 1;
-      const unsigned aph = (unsigned)((it >> 1) & 1);
-      if (!wait_or_fail(&acc_full[ab], aph, abort_flag)) goto done;
-      tc_fence_after();
-      const int row = m0 + 32 * q + lane;
-      const float sx = (row < p.M) ? xs[row] : 0.f;
-      epilogue_store<0>(p, tmem + (uint32_t)(ab * kBN), m0, n0, q, lane, sx, ws, 1.0f, &acc_empty[ab],
-                        mapa_u32(&acc_empty[ab], 0));
-    }
-  }
-done:
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync();  // no CTA leaves while the pair's MMAs may still touch its memory
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_2cta(tmem, 512);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // NVFP4 x NVFP4 -> fp32 (kind::mxf4nvf4, block16 E4M3 scales)
 // ---------------------------------------------------------------------------
 constexpr int kF4BK = 256;                 // K elements per k-tile (128 packed bytes per row)
@@ -938,6 +769,295 @@ done:
 }
 
 // ---------------------------------------------------------------------------
+// INT4 x INT4 on two SMs with A in tensor memory (kind::i8, cta_group::2).
+//
+// Widening nibbles to int8 through shared memory costs a store and a tensor
+// core read of every widened byte; with both operands there, the stores, the
+// staging writes and the MMA reads together exceed the shared-memory
+// bandwidth that an M = 256 MMA leaves.  Here only B goes through shared
+// memory: four warps, one per TMEM lane quadrant, widen the A rows in
+// registers and write them into TMEM with tcgen05.st (32 columns per k-tile),
+// and the MMA reads A from there.  TMEM: accumulator columns [0, 256), A
+// stages from column 256 (32 columns each).  With the accumulator single
+// buffered, the epilogue releases it as soon as its last columns are read
+// and stores bf16 through shared memory with TMA.
+//
+// Warps: 0 TMA producer, 1 MMA issuer (even CTA), 2..9 B converters,
+// 10..13 A converters, 14..17 epilogue.
+// ---------------------------------------------------------------------------
+constexpr int kI3Stg = 4, kI3Ops = 4;
+constexpr int kI3BWarps = 8;
+constexpr int kI3AWarp0 = 2 + kI3BWarps;      // 10
+constexpr int kI3EpiWarp0 = kI3AWarp0 + 4;    // 14
+constexpr int kI3EpiWarps = 8;                // two per TMEM lane quadrant, 128 columns each
+constexpr int kI3Threads = 32 * (kI3EpiWarp0 + kI3EpiWarps);
+constexpr int kI3StgA = 128 * 64, kI3StgB = 128 * 64, kI3OpB = 128 * 128;
+constexpr uint32_t kI3ACol0 = 256;
+constexpr size_t kI3Smem =
+    1024 + (size_t)kI3Ops * kI3OpB + (size_t)kI3Stg * (kI3StgA + kI3StgB) + 2 * kEpiStage + 256;
+
+// INT4 bf16 epilogue through shared memory for one 128-column half `ch` of the
+// CTA's 128 x 256 accumulator, by the four warps (one per lane quadrant) that
+// own that half: y = (acc >> 8) * sx[row] * sw[col], the arithmetic of
+// epilogue_store.  acc >> 8 (|.| < 2^22 for K <= 65536) becomes a float
+// exactly through the 1.5 * 2^23 magic number.  `stage` is this half's 32 KB
+// of staging (two 128B-swizzled 64-column boxes); one thread stores it with
+// TMA (which clips rows >= M and columns >= N).  Named barrier 1 + ch.
+__device__ __forceinline__ void epilogue_int4_bf16_tma(const GemmParams& p, const CUtensorMap* ytmap, uint32_t tacc,
+                                                       int m0, int n0, int q, int ch, int lane, float sx,
+                                                       const float* ws, uint8_t* stage,
+                                                       uint32_t acc_empty_cluster) {
+  const uint32_t tq = tacc + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * ch);
+  const int row = 32 * q + lane;  // row within the CTA's 128
+  const bool issuer = (q == 0 && lane == 0);
+  if (issuer) bulk_wait_read0();  // the previous tile's TMA store has read the staging buffer
+  named_sync(1 + ch, 128);
+#pragma unroll 1
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t r[32];
+    tmem_ld32(tq + (uint32_t)(32 * cc), r);
+    tmem_wait_ld();
+    if (cc == 3) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_cluster);  // this warp's accumulator lanes are read
+    }
+    const int c0 = n0 + 128 * ch + 32 * cc;
+    float sw[32];
+    if (c0 + 32 <= p.N) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 t = *reinterpret_cast<const float4*>(ws + c0 + j);
+        sw[j] = t.x;
+        sw[j + 1] = t.y;
+        sw[j + 2] = t.z;
+        sw[j + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sw[j] = (c0 + j < p.N) ? ws[c0 + j] : 0.f;
+    }
+    uint8_t* box = stage + (cc >> 1) * (kBM * 128);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 8 * k + 2 * e;
+        const float i0 = __int_as_float(((int)r[j] >> 8) + 0x4B400000) - kRoundMagic;
+        const float i1 = __int_as_float(((int)r[j + 1] >> 8) + 0x4B400000) - kRoundMagic;
+        __nv_bfloat162 b = __floats2bfloat162_rn(i0 * sx * sw[j], i1 * sx * sw[j + 1]);
+        w[e] = *reinterpret_cast<uint32_t*>(&b);
+      }
+      const int c16 = 4 * (cc & 1) + k;
+      *reinterpret_cast<uint4*>(box + row * 128 + 16 * (c16 ^ (row & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  fence_proxy_async_smem();
+  named_sync(1 + ch, 128);
+  if (issuer) {
+    tma_store_2d(ytmap, stage, n0 + 128 * ch, m0);
+    tma_store_2d(ytmap, stage + kBM * 128, n0 + 128 * ch + 64, m0);
+    bulk_commit();
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
+    gemm_int4_2sm_ts_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                            const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* opb = base;                                         // [kI3Ops][B 16K], 128B-swizzled int8
+  uint8_t* stg = opb + (size_t)kI3Ops * kI3OpB;                // [kI3Stg][A 8K | B 8K], 64B-swizzled nibbles
+  uint8_t* epi = stg + (size_t)kI3Stg * (kI3StgA + kI3StgB);   // bf16 output staging, one 32 KB half per column half
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi + 2 * kEpiStage);
+  uint64_t* stg_full = bars;
+  uint64_t* stg_empty = stg_full + kI3Stg;
+  uint64_t* op_full = stg_empty + kI3Stg;     // used in the even CTA only
+  uint64_t* op_empty = op_full + kI3Ops;
+  uint64_t* acc_full = op_empty + kI3Ops;
+  uint64_t* acc_empty = acc_full + 1;         // used in the even CTA only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int KT = p.K / kI4BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kI3Stg; ++i) {
+      mbar_init(&stg_full[i], 1);
+      mbar_init(&stg_empty[i], kI3BWarps + 4);
+    }
+    for (int i = 0; i < kI3Ops; ++i) {
+      mbar_init(&op_full[i], 2 * (kI3BWarps + 4));
+      mbar_init(&op_empty[i], 1);
+    }
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_empty[0], 2 * kI3EpiWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+    if (p.tma_store) prefetch_tmap(&tmap_y);
+  }
+  if (warp == 1) {
+    tmem_alloc_2cta(tmem_slot, 512);
+    tmem_relinquish_2cta();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      unsigned ph = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+        const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
+        const int nb = (tile / p.tiles_m) * 256 + 128 * (int)rank;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_or_fail(&stg_empty[s], ph ^ 1, abort_flag)) goto done;
+          uint8_t* sa = stg + (size_t)s * (kI3StgA + kI3StgB);
+          mbar_arrive_expect_tx(&stg_full[s], kI3StgA + kI3StgB);
+          tma_load_2d(sa, &tmap_x, kt * 64, m0, &stg_full[s]);
+          tma_load_2d(sa + kI3StgA, &tmap_w, kt * 64, nb, &stg_full[s]);
+          if (++s == kI3Stg) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_i8(256, 256);
+      int o = 0;
+      unsigned oph = 0;
+      int it = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+        if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&acc_empty[0], (unsigned)((it & 1) ^ 1))) {
+          *((volatile int*)abort_flag) = 1;
+          goto done;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&op_full[o], oph)) {
+            *((volatile int*)abort_flag) = 1;
+            goto done;
+          }
+          tc_fence_after();
+          const uint64_t bd = smem_desc_sw128(opb + (size_t)o * kI3OpB);
+          const uint32_t ta = tmem + kI3ACol0 + 32u * (uint32_t)o;
+#pragma unroll
+          for (int j = 0; j < kI4BK / 32; ++j) mma_i8_2cta_ts(tmem, ta + 8u * (uint32_t)j, bd + 2 * j, idesc, (kt | j) != 0);
+          tc_commit_2cta_mc(&op_empty[o], 0x3);
+          if (++o == kI3Ops) { o = 0; oph ^= 1; }
+        }
+        tc_commit_2cta_mc(&acc_full[0], 0x3);
+      }
+    }
+  } else if (warp < kI3AWarp0) {
+    // B: packed rows -> 128B-swizzled int8 in shared memory
+    const int t = threadIdx.x - 64;
+    int s = 0, o = 0;
+    unsigned ph = 0, oph = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!wait_or_fail(&stg_full[s], ph, abort_flag)) goto done;
+        if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
+        const uint8_t* sb = stg + (size_t)s * (kI3StgA + kI3StgB) + kI3StgA;
+        uint8_t* ob = opb + (size_t)o * kI3OpB;
+#pragma unroll
+        for (int jb = t; jb < 128 * 4; jb += 32 * kI3BWarps) convert_chunk(sb, ob, jb >> 2, jb & 3);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(mapa_u32(&op_full[o], 0));
+          mbar_arrive(&stg_empty[s]);
+        }
+        if (++s == kI3Stg) { s = 0; ph ^= 1; }
+        if (++o == kI3Ops) { o = 0; oph ^= 1; }
+      }
+    }
+  } else if (warp < kI3EpiWarp0) {
+    // A: one row per thread, widened in registers, written to this warp's TMEM lanes
+    const int quad = warp & 3;
+    const int row = 32 * quad + lane;
+    const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16) + kI3ACol0;
+    int s = 0, o = 0;
+    unsigned ph = 0, oph = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!wait_or_fail(&stg_full[s], ph, abort_flag)) goto done;
+        if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
+        tc_fence_after();
+        const uint8_t* sa = stg + (size_t)s * (kI3StgA + kI3StgB) + row * 64;
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 in = *reinterpret_cast<const uint4*>(sa + 16 * (j ^ ((row >> 1) & 3)));
+          uint4 o0, o1;
+          widen16(in, o0, o1);
+          w[8 * j + 0] = o0.x;
+          w[8 * j + 1] = o0.y;
+          w[8 * j + 2] = o0.z;
+          w[8 * j + 3] = o0.w;
+          w[8 * j + 4] = o1.x;
+          w[8 * j + 5] = o1.y;
+          w[8 * j + 6] = o1.z;
+          w[8 * j + 7] = o1.w;
+        }
+        tmem_st32(trow + 32u * (uint32_t)o, w);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(mapa_u32(&op_full[o], 0));
+          mbar_arrive(&stg_empty[s]);
+        }
+        if (++s == kI3Stg) { s = 0; ph ^= 1; }
+        if (++o == kI3Ops) { o = 0; oph ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int ch = (warp - kI3EpiWarp0) >> 2;  // column half of the accumulator
+    const float* xs = static_cast<const float*>(p.xscale);
+    const float* ws = static_cast<const float*>(p.wscale);
+    int it = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+      const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
+      const int n0 = (tile / p.tiles_m) * 256;
+      if (!wait_or_fail(&acc_full[0], (unsigned)(it & 1), abort_flag)) goto done;
+      tc_fence_after();
+      const int row = m0 + 32 * q + lane;
+      const float sx = (row < p.M) ? xs[row] : 0.f;
+      if (p.tma_store) {
+        epilogue_int4_bf16_tma(p, &tmap_y, tmem, m0, n0, q, ch, lane, sx, ws, epi + (size_t)ch * kEpiStage,
+                               mapa_u32(&acc_empty[0], 0));
+      } else if (ch == 0) {
+        epilogue_store<0>(p, tmem, m0, n0, q, lane, sx, ws, 1.0f, &acc_empty[0], mapa_u32(&acc_empty[0], 0));
+      } else {
+        __syncwarp();  // the other half's warps do the whole slab on this path
+        if (lane == 0) mbar_arrive_cluster(mapa_u32(&acc_empty[0], 0));
+      }
+    }
+    if (q == 0 && lane == 0) bulk_wait0();  // stores out of shared memory complete before the CTA exits
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // no CTA leaves while the pair's MMAs may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_2cta(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1046,14 +1166,18 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
       p.num_tiles = p.tiles_m * p.tiles_n;
       const int sms = gemm_num_sms() & ~1;
       const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
-      static bool attr2_done = false;
-      if (!attr2_done) {
-        if (cudaFuncSetAttribute(gemm_int4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI2Smem) !=
-            cudaSuccess)
+      CUtensorMap ty;
+      std::memset(&ty, 0, sizeof(ty));
+      p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
+      if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
+      static bool attr3_done = false;
+      if (!attr3_done) {
+        if (cudaFuncSetAttribute(gemm_int4_2sm_ts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kI3Smem) != cudaSuccess)
           return RQ_ERR_CUDA;
-        attr2_done = true;
+        attr3_done = true;
       }
-      gemm_int4_2sm_kernel<<<grid2, kI4Threads, kI2Smem, st>>>(tx2, tw2, p);
+      gemm_int4_2sm_ts_kernel<<<grid2, kI3Threads, kI3Smem, st>>>(tx2, tw2, ty, p);
       return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
     }
     static bool attr_done = false;
