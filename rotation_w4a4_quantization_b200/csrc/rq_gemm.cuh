@@ -785,7 +785,7 @@ done:
 // Warps: 0 TMA producer, 1 MMA issuer (even CTA), 2..9 B converters,
 // 10..13 A converters, 14..17 epilogue.
 // ---------------------------------------------------------------------------
-constexpr int kI3Stg = 4, kI3Ops = 4;
+constexpr int kI3Stg = 6, kI3Ops = 4;
 constexpr int kI3BWarps = 8;
 constexpr int kI3AWarp0 = 2 + kI3BWarps;      // 10
 constexpr int kI3EpiWarp0 = kI3AWarp0 + 4;    // 14
