@@ -112,6 +112,24 @@ def e4m3_round_unsigned(v):
     return codes.astype(np.int64), tie_dist
 
 
+def e8m0_decode(code):
+    """Value of an 8-bit E8M0 scale code: 2^(code - 127); code 255 is NaN.
+
+    E8M0 is the OCP Microscaling shared-scale format: an 8-bit unsigned
+    biased exponent, no sign, no mantissa ("powers of two", as the pages
+    describe MXFP4's scales).
+    """
+    code = int(code)
+    if code == 255:
+        return float("nan")
+    return 2.0 ** (code - 127)
+
+
+def e8m0_values(codes):
+    table = np.array([e8m0_decode(c) for c in range(256)])
+    return table[np.asarray(codes, dtype=np.int64)]
+
+
 def e2m1_values(codes):
     table = np.array([e2m1_decode(c) for c in range(16)])
     return table[np.asarray(codes, dtype=np.int64)]

@@ -45,3 +45,10 @@ def nvfp4_y(ex, sx, gx, ew, sw, gw):
     xh = quant.nvfp4_dequant(ex, sx, gx)
     wh = quant.nvfp4_dequant(ew, sw, gw)
     return xh @ wh.T
+
+
+def mxfp4_y(ex, sx, ew, sw):
+    """Y = deq(X) . deq(W)^T in fp64 from MXFP4 codes and E8M0 scales."""
+    xh = quant.mxfp4_dequant(ex, sx)
+    wh = quant.mxfp4_dequant(ew, sw)
+    return xh @ wh.T

@@ -11,6 +11,9 @@ Sources on the pages:
 * NVFP4 -- E2M1 values with an FP8 (E4M3) scale for every block of 16 values:
   same section.  The fp32 per-tensor scale is the second level of NVFP4's
   two-level scaling.
+* MXFP4 -- E2M1 values whose scales are powers of two shared by 32 values:
+  same article, section "The full model in NVFP4, on vLLM" (the FP4 study it
+  cites) and section "When to rotate".
 * KV cache at 4 bits, asymmetric: "SpinQuant (learned rotations + W4A4KV4)",
   field "Activation scheme" (per-group INT4 asymmetric for the KV cache), and
   "QuaRot (rotation-based outlier removal, W4A4KV4)", field "Activation scheme"
@@ -24,6 +27,12 @@ Readings where the pages are silent (each also listed in the design notes):
   (dynamic) or given by the caller (static).  Per block b of 16 along K:
   S_b = E4M3_rn_satfinite(amax_b / (6 g)); e = E2M1_rn_satfinite(x / (S_b g));
   S_b = 0 -> e = 0.
+* MXFP4: per block b of 32 along K, the E8M0 scale 2^e with
+  e = floor(log2(amax_b)) - 2 (2 = the exponent of E2M1's largest value 6),
+  clamped to E8M0's range [-127, 127]; e = E2M1_rn_satfinite(x / 2^e).  The
+  pages give no scale rule; this is the shared-exponent rule of the OCP
+  Microscaling formats.  amax_b = 0 -> scale code 0 (2^-127), e = 0.  There
+  is no per-tensor scale.
 * KV4 per (batch, head, token) vector of head_dim after the Hadamard:
   z = min, s = (max - min)/15, z_h = fp16(z), s_h = fp16(s);
   q = clamp(rint((x - z_h)/s_h), 0, 15); s_h = 0 -> q = 0.
@@ -49,6 +58,9 @@ TIE_EPS = 2.0 ** -15
 
 INT4_QMAX = 7
 NVFP4_BLOCK = 16
+MXFP4_BLOCK = 32
+E2M1_EMAX = 2          # 6 = 1.5 * 2^2
+E8M0_EMIN, E8M0_EMAX = -127, 127
 E2M1_MAX = 6.0
 E4M3_MAX = 448.0
 
@@ -120,6 +132,44 @@ def nvfp4_dequant(e_codes, s_codes, g):
     s = formats.e4m3_values(s_codes)
     return (e.reshape(rows, k // NVFP4_BLOCK, NVFP4_BLOCK) * s[:, :, None]
             * np.float64(np.float32(g))).reshape(rows, k)
+
+
+def mxfp4_rows(xr):
+    """MXFP4 quantization of fp64 [rows, K].
+
+    Returns (e codes int64 [rows, K] (sign in bit 3), scale codes int64
+    [rows, K/32] (E8M0 bits), tie_e bool [rows, K], tie_s bool [rows, K/32]).
+    tie_s flags blocks whose amax lies within the tie band of a power of two,
+    where floor(log2(amax)) flips between neighbours under fp32 rounding.
+    """
+    xr = np.asarray(xr, dtype=np.float64)
+    rows, k = xr.shape
+    if k % MXFP4_BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    blocks = xr.reshape(rows, k // MXFP4_BLOCK, MXFP4_BLOCK)
+    amax_b = np.abs(blocks).max(axis=2)
+    pos = amax_b > 0
+    with np.errstate(divide="ignore"):
+        # frexp gives amax = f * 2^p with f in [0.5, 1): floor(log2(amax)) = p - 1 exactly
+        _, p2 = np.frexp(np.where(pos, amax_b, 1.0))
+    e = np.where(pos, p2.astype(np.int64) - 1 - E2M1_EMAX, E8M0_EMIN)
+    e = np.clip(e, E8M0_EMIN, E8M0_EMAX)
+    s_codes = (e + 127).astype(np.int64)
+    # within the band of a power of two: fp32 rounding of amax may change floor(log2)
+    pw = np.ldexp(1.0, np.where(pos, p2.astype(np.int64) - 1, 0))
+    near = (np.abs(amax_b - pw) <= TIE_EPS * amax_b) | (np.abs(amax_b - 2 * pw) <= TIE_EPS * amax_b)
+    tie_s = near & pos
+    v = blocks / np.ldexp(1.0, e)[:, :, None]                 # exact: a power-of-two division
+    e_codes, e_tie_dist = formats.e2m1_round(v)
+    tie_e = (e_tie_dist <= TIE_EPS * np.maximum(1.0, np.abs(v))) & pos[:, :, None]
+    return (e_codes.reshape(rows, k), s_codes, tie_e.reshape(rows, k), tie_s)
+
+
+def mxfp4_dequant(e_codes, s_codes):
+    e = formats.e2m1_values(e_codes)
+    rows, k = e.shape
+    s = formats.e8m0_values(s_codes)
+    return (e.reshape(rows, k // MXFP4_BLOCK, MXFP4_BLOCK) * s[:, :, None]).reshape(rows, k)
 
 
 def _fp16_tie(v):

@@ -8,7 +8,10 @@ stand-ins (CPU only).
 * section "What it buys in 4 bits, and what it doesn't": rotation cuts INT4
   product error by a large factor (46% -> 11%, 75% -> 22%); NVFP4 starts six
   to seven times lower than INT4 and the rotation does not lower it (6.6% ->
-  7.2%, 11.9% -> 12.4%).
+  7.2%, 11.9% -> 12.4%);
+* section "The full model in NVFP4, on vLLM" (the FP4 study it cites) and
+  section "When to rotate": rotations help MXFP4, whose scales are powers of
+  two shared by 32 values.
 
 The exact figures came from real Qwen3-8B layers and are not reproducible here
 (parity unpinned); the tests check the direction and a margin.
@@ -84,3 +87,17 @@ def test_nvfp4_lower_and_not_helped(which, request):
     f0, f1 = _fp4_err(y, x, w), _fp4_err(y, xr, wr)
     assert f0 < i0 / 3
     assert f1 >= 0.95 * f0
+
+
+def _mx_err(y, a, b):
+    ea, sa, _, _ = quant.mxfp4_rows(a)
+    eb, sb, _, _ = quant.mxfp4_rows(b)
+    return metrics.rel_product_error(y, gemm.mxfp4_y(ea, sa, eb, sb))
+
+
+@pytest.mark.parametrize("which", ["qproj", "downproj"])
+def test_rotation_helps_mxfp4(which, request):
+    x, w, _, xr, wr = request.getfixturevalue(which)
+    y = x @ w.T
+    m0, m1 = _mx_err(y, x, w), _mx_err(y, xr, wr)
+    assert m1 < 0.95 * m0

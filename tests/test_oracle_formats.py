@@ -74,3 +74,14 @@ def test_fp16_rounds_fp64_directly():
     """fp64 -> fp16 in one rounding: just above a midpoint goes up (no double rounding)."""
     assert formats.to_fp16(np.array([1 + 2 ** -11 + 2 ** -40]))[0] == 1 + 2 ** -10
     assert formats.to_fp16(np.array([1 + 2 ** -11]))[0] == 1.0
+
+
+def test_e8m0_decode_closed_form():
+    # E8M0 (OCP Microscaling shared scale): value 2^(code - 127), code 255 = NaN
+    import math
+    for c in range(255):
+        assert formats.e8m0_decode(c) == math.ldexp(1.0, c - 127)
+    assert math.isnan(formats.e8m0_decode(255))
+    assert formats.e8m0_decode(127) == 1.0
+    v = formats.e8m0_values(np.arange(255))
+    assert np.all(v[1:] == 2.0 * v[:-1])

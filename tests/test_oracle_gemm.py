@@ -61,3 +61,23 @@ def test_dequant_roundtrip_nvfp4_codes():
     # re-quantizing a dequantized tensor is idempotent on its codes wherever the block scale is kept
     same_scale = (s2 == s)[:, :, None].repeat(16, axis=2).reshape(4, 64)
     assert np.array_equal(formats.e2m1_values(e2)[same_scale], formats.e2m1_values(e)[same_scale])
+
+
+def test_mxfp4_y_matches_blockwise_sum():
+    """Y = sum_b 2^(sx[m,b]-127) 2^(sw[n,b]-127) sum_{k in b} e_x e_w, by explicit loops."""
+    import math
+    rng = np.random.default_rng(3)
+    m, n, k = 3, 2, 64
+    ex = rng.integers(0, 16, size=(m, k))
+    ew = rng.integers(0, 16, size=(n, k))
+    sx = rng.integers(100, 150, size=(m, k // 32))
+    sw = rng.integers(100, 150, size=(n, k // 32))
+    y = gemm.mxfp4_y(ex, sx, ew, sw)
+    for i in range(m):
+        for j in range(n):
+            tot = 0.0
+            for b in range(k // 32):
+                inner = sum(formats.e2m1_decode(ex[i, t]) * formats.e2m1_decode(ew[j, t])
+                            for t in range(32 * b, 32 * b + 32))
+                tot += math.ldexp(inner, int(sx[i, b]) - 127 + int(sw[j, b]) - 127)
+            assert y[i, j] == tot

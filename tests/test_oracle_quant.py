@@ -143,3 +143,81 @@ def test_unpack_roundtrip_unsigned(k):
     rng = np.random.default_rng(k)
     c = rng.integers(0, 16, size=(3, k))
     assert np.array_equal(quant.unpack_nibbles(quant.pack_nibbles(c), signed=False), c)
+
+
+# ---------------------------------------------------------------- MXFP4
+def _mx_block(vals):
+    x = np.zeros((1, 32))
+    x[0, :len(vals)] = vals
+    return x
+
+
+def test_mxfp4_hand_block():
+    # amax = 6: floor(log2 6) - 2 = 0, scale 1; codes are E2M1 of the values
+    # themselves, nearest with ties to the even code, saturating at 6.
+    vals = [6.0, -3.0, 1.5, 0.75, 0.25, 0.3, -0.26, 5.0, 2.5, -1.25, 3.5]
+    want = [7, 8 | 5, 3, 2, 0, 1, 8 | 1, 6, 4, 8 | 2, 6]
+    #       6  -3     1.5 1(tie 0.5|1 -> even 1.0) 0(tie 0|0.5 -> even 0) 0.5 -0.5
+    #       4(tie 4|6 -> even 4) 2(tie 2|3 -> even 2) -1(tie 1|1.5 -> even 1) 4(tie 3|4 -> even 4)
+    e, s, tie_e, tie_s = quant.mxfp4_rows(_mx_block(vals))
+    assert s[0, 0] == 127
+    assert list(e[0, :len(vals)]) == want
+    assert np.all(e[0, len(vals):] == 0)
+    assert tie_e[0, 3] and tie_e[0, 4] and tie_e[0, 7] and not tie_e[0, 0]
+
+
+def test_mxfp4_saturates_and_scales():
+    # amax = 7.9 * 2^5: exponent floor(log2 7.9) + 5 - 2 = 5; 7.9 -> 6 (saturation)
+    x = _mx_block([7.9 * 32, 1.0 * 32, -0.5 * 32])
+    e, s, _, _ = quant.mxfp4_rows(x)
+    assert s[0, 0] == 127 + 5
+    assert list(e[0, :3]) == [7, 2, 8 | 1]
+    # amax = 1: exponent -2, scale 1/4, so 1 -> 4 and 0.3 -> 1.2 -> 1
+    e, s, _, _ = quant.mxfp4_rows(_mx_block([1.0, 0.3]))
+    assert s[0, 0] == 125 and list(e[0, :2]) == [6, 2]
+
+
+def test_mxfp4_scale_rule_by_search():
+    # the shared exponent is the unique integer e with 2^(e+2) <= amax < 2^(e+3)
+    rng = np.random.default_rng(11)
+    for _ in range(400):
+        mag = np.ldexp(rng.uniform(1.0, 2.0), int(rng.integers(-60, 60)))
+        x = _mx_block(rng.uniform(-1, 1, 32) * mag)
+        amax = np.abs(x).max()
+        e_search = next(c for c in range(-200, 200) if 2.0 ** (c + 2) <= amax < 2.0 ** (c + 3))
+        _, s, _, _ = quant.mxfp4_rows(x)
+        assert s[0, 0] - 127 == min(max(e_search, -127), 127)
+
+
+def test_mxfp4_power_of_two_equivariance():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((4, 64)) * 3
+    e0, s0, _, _ = quant.mxfp4_rows(x)
+    for j in (-9, -1, 1, 13):
+        e1, s1, _, _ = quant.mxfp4_rows(x * 2.0 ** j)
+        assert np.array_equal(e0, e1) and np.array_equal(s1, s0 + j)
+
+
+def test_mxfp4_roundtrip_bound_and_zero_block():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((8, 128)) * rng.uniform(0.01, 100, size=(8, 1))
+    x[3, 32:64] = 0.0
+    e, s, _, _ = quant.mxfp4_rows(x)
+    xh = quant.mxfp4_dequant(e, s)
+    sc = np.repeat(formats.e8m0_values(s), 32, axis=1)
+    v = np.abs(x) / sc
+    grid = formats.E2M1_POS_VALUES
+    # half the local grid spacing below 6; saturated values sit at 6 * scale
+    idx = np.clip(np.searchsorted(grid, np.minimum(v, 6.0)), 1, len(grid) - 1)
+    half_gap = 0.5 * (grid[idx] - grid[idx - 1])
+    ok = np.where(v <= 6.0, np.abs(x - xh) <= half_gap * sc + 1e-300, np.abs(xh) == 6.0 * sc)
+    assert ok.all()
+    assert s[3, 1] == 0 and np.all(e[3, 32:64] == 0)
+
+
+def test_mxfp4_power_of_two_amax_is_a_scale_tie():
+    x = _mx_block([4.0, 1.0])
+    _, s, _, tie_s = quant.mxfp4_rows(x)
+    assert s[0, 0] == 127 and tie_s[0, 0]
+    _, _, _, tie_s = quant.mxfp4_rows(_mx_block([5.0, 1.0]))
+    assert not tie_s[0, 0]
