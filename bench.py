@@ -132,7 +132,7 @@ class Workload:
             self.ws = torch.empty((16,), dtype=torch.uint8, device=device)
             self.y = torch.empty((m, n), dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32,
                                  device=device)
-            scale_bytes = m * 4 if self.fmt == "int4" else m * (k // 16)
+            scale_bytes = {"int4": m * 4, "nvfp4": m * (k // 16), "mxfp4": m * (k // 32)}[self.fmt]
             self.quant_bytes = m * k * 2 + m * k // 2 + scale_bytes
             self.gemm_ops = 2 * m * n * k
             self.h2d_bytes = self.x.numel() * 2
@@ -267,25 +267,32 @@ def oracle_sample(name, rows):
     wr = ohad.rotate(w, s, block)
     if c["fmt"] == "int4":
         qw, sw, _ = oquant.int4_sym_rows(wr)
-    else:
+    elif c["fmt"] == "nvfp4":
         gw = oquant.nvfp4_global_scale(wr)
         ew, sfw, _, _ = oquant.nvfp4_rows(wr, gw)
+    else:
+        ew, sfw, _, _ = oquant.mxfp4_rows(wr)
     t0 = time.perf_counter()
     xr = ohad.rotate(x, s, block)
     if c["fmt"] == "int4":
         qx, sx, _ = oquant.int4_sym_rows(xr)
         oquant.pack_nibbles(qx)
-    else:
+    elif c["fmt"] == "nvfp4":
         gx = oquant.nvfp4_global_scale(xr)
         ex, sfx, _, _ = oquant.nvfp4_rows(xr, gx)
+        oquant.pack_nibbles(ex)
+    else:
+        ex, sfx, _, _ = oquant.mxfp4_rows(xr)
         oquant.pack_nibbles(ex)
     t1 = time.perf_counter()
     if c["fmt"] == "int4":
         ogemm.int4_y(ogemm.int4_acc(qx, qw), sx, sw)
-    else:
+    elif c["fmt"] == "nvfp4":
         ogemm.nvfp4_y(ex, sfx, gx, ew, sfw, gw)
+    else:
+        ogemm.mxfp4_y(ex, sfx, ew, sfw)
     t2 = time.perf_counter()
-    scale_bytes = rows * 4 if c["fmt"] == "int4" else rows * (k // 16)
+    scale_bytes = {"int4": rows * 4, "nvfp4": rows * (k // 16), "mxfp4": rows * (k // 32)}[c["fmt"]]
     nbytes = rows * k * 2 + rows * k // 2 + scale_bytes
     return (nbytes / (t1 - t0) / 1e9, 2.0 * rows * n * k / (t2 - t1) / 1e12, t2 - t0,
             "%d of %d rows of X with the full W" % (rows, c["M"]))
@@ -301,7 +308,8 @@ def blas_threads():
 
 
 def sample_rows(name):
-    return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096}[name]
+    return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096,
+            "q_proj_mxfp4": 256}[name]
 
 
 # --------------------------------------------------------------------------- main
@@ -388,7 +396,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4" if args.workload != "q_proj_nvfp4" else "nvfp4",
+        "dtype": wl.cfg.get("fmt", "int4"),
         "data": "synthetic (seeded, shaped like the article's Qwen3-8B layer inputs)",
         "config": workload_config(args, wl),
         "gpu_launches": K * (wl.quant_launches() + wl.gemm_launches()),
@@ -401,15 +409,15 @@ def main():
     roof_q["frac"] = round(roof_q["achieved"] / roof_q["peak"], 4)
     if wl.gemm_launches():
         ratio = 2.0  # INT8 and FP4 dense tensor peaks are 2x / 4x the bf16 one (nominal ratios)
-        if wl.fmt == "nvfp4":
+        if wl.fmt in ("nvfp4", "mxfp4"):
             ratio = 4.0
         tops = wl.gemm_ops * world / (g_mean_ms * 1e-3) / 1e12
         peak_t = peaks["bf16"] * ratio
         two_sm = wl.cfg["M"] > 128
         roof_g = {"bound": "tensor", "achieved": round(wl.gemm_ops / (g_mean_ms * 1e-3) / 1e12, 1), "peak": peak_t,
                   "unit": "TFLOP/s", "traffic": traffic("gemm", args.workload),
-                  "kernel": ("gemm_int4" if wl.fmt == "int4" else "gemm_nvfp4") +
-                            (("_2sm_ts_kernel" if wl.fmt == "int4" else "_2sm_kernel") if two_sm else "_kernel"),
+                  "kernel": ("gemm_int4_2sm_ts_kernel" if two_sm else "gemm_int4_kernel") if wl.fmt == "int4" else
+                            ("gemm_fp4_2sm_kernel" if two_sm else "gemm_fp4_kernel") + "<%s>" % wl.fmt,
                   "peak_source": "%s bf16 x %g (nominal %s/bf16 ratio)" % (peaks["src"], ratio,
                                                                            "int8" if ratio == 2 else "fp4")}
         roof_g["frac"] = round(roof_g["achieved"] / peak_t, 4)

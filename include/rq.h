@@ -60,7 +60,11 @@ typedef enum {
   RQ_ERR_TIMEOUT = 6            /* a kernel gave up on a bounded wait (see rq_get_device_error) */
 } rq_status;
 
-typedef enum { RQ_INT4 = 0, RQ_NVFP4 = 1 } rq_format;
+typedef enum {
+  RQ_INT4 = 0,  /* symmetric INT4, one fp32 scale per row */
+  RQ_NVFP4 = 1, /* E2M1, one E4M3 scale per 16 values, fp32 per-tensor scale */
+  RQ_MXFP4 = 2  /* E2M1, one E8M0 (power-of-two) scale per 32 values */
+} rq_format;
 
 typedef enum {
   RQ_OUT_F32 = 0,     /* Y as fp32 */
@@ -82,14 +86,16 @@ RQ_API rq_status rq_init(int device);
 RQ_API const char* rq_status_string(rq_status status);
 
 /* Bytes of device workspace rq_rotate_quantize / rq_prepare_weights need:
- * 16 for NVFP4 (the dynamic-scale max word), 0 for INT4.  The workspace must
+ * 16 for NVFP4 (the dynamic-scale max word), 0 for INT4 and MXFP4.  The workspace must
  * be 16-byte aligned; its contents need not be initialised. */
 RQ_API size_t rq_workspace_bytes(rq_format fmt);
 
 /*
  * rq_rotate_quantize: X~ = X.Q, then quantize and pack (the online activation
  * side; "What it buys in 4 bits, and what it doesn't": INT4 with one scale per
- * token, or NVFP4 with an FP8 scale for every block of 16 values).
+ * token, or NVFP4 with an FP8 scale for every block of 16 values; "The full
+ * model in NVFP4, on vLLM" and "When to rotate": MXFP4, whose scales are
+ * powers of two shared by 32 values).
  *
  *  X_dev      bf16 [M, ldx]; rows 16-byte aligned (X_dev and ldx*2 multiples of 16).
  *  M          rows (tokens), >= 0.  M = 0 is a no-op.
@@ -109,6 +115,14 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *                 RQ_SCALE_STATIC : read.
  *               S_b = E4M3_rn_satfinite(amax_b / (6 g));
  *               e = E2M1_rn_satfinite(x~ / (S_b g)); S_b = 0 gives e = 0.
+ *             RQ_MXFP4 (block must be 128):
+ *               codes_dev  uint8 [M, K/2] E2M1 codes,
+ *               scales_dev uint8 [M, K/32] E8M0 block scales (4-byte aligned):
+ *               per block b of 32, 2^e_b with e_b = floor(log2(amax_b)) - 2
+ *               clamped to [-127, 127] (the OCP Microscaling shared-exponent
+ *               rule; the pages name only powers of two); e = E2M1_rn_satfinite(x~ / 2^e_b).
+ *               amax_b = 0 gives scale code 0 and e = 0.  gscale_dev and
+ *               workspace_dev are unused (may be NULL).
  *  workspace_dev  rq_workspace_bytes(fmt) bytes (may be NULL when that is 0).
  *  codes_dev and scales_dev 16-byte aligned (8 for NVFP4 scales).
  * Values that sit within a few fp32 ulps of a rounding boundary may round
@@ -139,8 +153,12 @@ RQ_API rq_status rq_prepare_weights(const void* W_dev, int64_t N, int64_t K, int
  *  RQ_NVFP4: xscales_dev uint8 [M, K/16], wscales_dev uint8 [N, K/16] (E4M3, 16-byte aligned),
  *            xgscale_dev / wgscale_dev float scalars;
  *            Y = gx gw sum_b Sx[m,b] Sw[n,b] sum_{k in b} ex ew.
+ *  RQ_MXFP4: xscales_dev uint8 [M, K/32], wscales_dev uint8 [N, K/32] (E8M0, 16-byte aligned);
+ *            Y = sum_b 2^(sx[m,b]-127) 2^(sw[n,b]-127) sum_{k in b} ex ew; the global
+ *            scale pointers are unused (may be NULL).  RQ_OUT_I32_ACC is INT4 only.
  *  xcodes_dev uint8 [M, K/2], wcodes_dev uint8 [N, K/2], both 16-byte aligned.
- *  K a multiple of 128 (INT4) or 256 (NVFP4), at most 65536; M, N >= 0.
+ *  K a multiple of 128 (INT4), 256 (NVFP4) or 512 (MXFP4: scale rows of K/32
+ *  bytes are copied in 16-byte units), at most 65536; M, N >= 0.
  *  Y_dev [M, ldy] of fp32, bf16 or int32 per `out`; ldy >= N; Y_dev aligned to
  *  its element size (16-byte aligned rows are stored with vector stores).
  */

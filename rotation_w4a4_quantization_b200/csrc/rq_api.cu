@@ -201,9 +201,9 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
                                void* workspace, cudaStream_t st) {
   rq_status s = check_rotation_args(X, M, K, ldx, signs, block);
   if (s != RQ_OK) return s;
-  if (fmt != RQ_INT4 && fmt != RQ_NVFP4) return RQ_ERR_INVALID_ARG;
+  if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4) return RQ_ERR_INVALID_ARG;
   if (gmode != RQ_SCALE_DYNAMIC && gmode != RQ_SCALE_STATIC) return RQ_ERR_INVALID_ARG;
-  if (fmt == RQ_NVFP4 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt != RQ_INT4 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return RQ_OK;
   if (!codes || !scales) return RQ_ERR_INVALID_ARG;
   if (!aligned(codes, 16)) return RQ_ERR_ALIGNMENT;
@@ -213,7 +213,7 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
     if (!aligned(scales, 8) || !aligned(gscale, 4)) return RQ_ERR_ALIGNMENT;
     if (workspace && !aligned(workspace, 16)) return RQ_ERR_ALIGNMENT;
   } else {
-    if (!aligned(scales, 4)) return RQ_ERR_ALIGNMENT;
+    if (!aligned(scales, 4)) return RQ_ERR_ALIGNMENT;  // INT4 fp32 scales, MXFP4 4 bytes per 128-block
   }
   if (M == 0) return RQ_OK;
 
@@ -223,6 +223,10 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
     p.scales_f32 = static_cast<float*>(scales);
     if (block == 0) return launch_full<kModeInt4>(p, st);
     return launch_block<kModeInt4>(p, st);
+  }
+  if (fmt == RQ_MXFP4) {
+    p.scales_e4m3 = static_cast<uint8_t*>(scales);
+    return launch_block<kModeMxfp4>(p, st);
   }
   p.scales_e4m3 = static_cast<uint8_t*>(scales);
   if (gmode == RQ_SCALE_DYNAMIC) {

@@ -35,6 +35,9 @@
 #include <cuda.h>
 
 #include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 #include "rq_common.cuh"
 #include "rq_tc.cuh"
@@ -407,6 +410,19 @@ done:
 // ---------------------------------------------------------------------------
 // NVFP4 x NVFP4 -> fp32 (kind::mxf4nvf4, block16 E4M3 scales)
 // ---------------------------------------------------------------------------
+// The 32-bit tensor-memory word of one row's scales for MMA j (K = 64) of
+// k-tile kt, from the row's 16 staged scale bytes.  NVFP4: the four E4M3
+// scales 4j..4j+3 of the k-tile.  MXFP4: the two E8M0 scales of the MMA,
+// bytes 8*(kt & 1) + 2j and + 1 (the 16 bytes span two k-tiles), in the low
+// half of the word.
+template <bool MX>
+__device__ __forceinline__ uint32_t sf_word(const uint4& row16, int j, int kt) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&row16);
+  if (!MX) return w[j];
+  const uint32_t h = w[2 * (kt & 1) + (j >> 1)];
+  return (j & 1) ? (h >> 16) : (h & 0xFFFFu);
+}
+
 constexpr int kF4BK = 256;                 // K elements per k-tile (128 packed bytes per row)
 constexpr int kF4St = 3;
 constexpr int kF4OpA = kBM * 128, kF4OpB = kBN * 128;
@@ -417,8 +433,9 @@ constexpr size_t kF4Smem = 1024 + (size_t)kF4St * kF4Stage + kEpiStage + 256;
 constexpr uint32_t kF4SfCol0 = 256;        // TMEM columns [256, 256 + 48*stages) hold the scales
 constexpr uint32_t kF4SfCols = 48;         // per stage: SFA 16 columns, SFB 32 columns
 
+template <bool MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+    gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_sx, const __grid_constant__ CUtensorMap tmap_sw,
                       const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -473,15 +490,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&op_full[s], kF4Stage);
           tma_load_2d(sa, &tmap_x, kt * 128, m0, &op_full[s]);
           tma_load_2d(sa + kF4OpA, &tmap_w, kt * 128, n0, &op_full[s]);
-          tma_load_2d(sa + kF4OpA + kF4OpB, &tmap_sx, kt * 16, m0, &op_full[s]);
-          tma_load_2d(sa + kF4OpA + kF4OpB + kF4SfA, &tmap_sw, kt * 16, n0, &op_full[s]);
+          const int sx0 = MX ? (kt >> 1) * 16 : kt * 16;  // 16-byte aligned scale column
+          tma_load_2d(sa + kF4OpA + kF4OpB, &tmap_sx, sx0, m0, &op_full[s]);
+          tma_load_2d(sa + kF4OpA + kF4OpB + kF4SfA, &tmap_sw, sx0, n0, &op_full[s]);
           if (++s == kF4St) { s = 0; ph ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_nvf4(kBM, kBN);
+      const uint32_t idesc = idesc_fp4(kBM, kBN, MX);
       int s = 0;
       unsigned ph = 0;
       int it = 0;
@@ -497,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sf = tmem + kF4SfCol0 + (uint32_t)s * kF4SfCols;
 #pragma unroll
           for (int j = 0; j < kF4BK / 64; ++j)
-            mma_nvf4(tmem, ad + 2 * j, bd + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (kt | j) != 0);
+            mma_fp4<MX>(tmem, ad + 2 * j, bd + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (kt | j) != 0);
           tc_commit(&op_empty[s]);
           if (++s == kF4St) { s = 0; ph ^= 1; }
         }
@@ -526,18 +544,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&ua[i]);
-            da[4 * j + i] = w[j];
-          }
+          for (int i = 0; i < 4; ++i) da[4 * j + i] = sf_word<MX>(ua[i], j, kt);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&ub[i]);
             const int c = 8 * j + i;
             if (c < 16)
-              db0[c] = w[j];
+              db0[c] = sf_word<MX>(ub[i], j, kt);
             else
-              db1[c - 16] = w[j];
+              db1[c - 16] = sf_word<MX>(ub[i], j, kt);
           }
         }
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + kF4SfCol0 + (uint32_t)s * kF4SfCols;
@@ -553,7 +567,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     const int q = warp & 3;
-    const float g = (*p.xg) * (*p.wg);
+    const float g = MX ? 1.0f : (*p.xg) * (*p.wg);
     int it = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
       const int m0 = (tile % p.tiles_m) * kBM, n0 = (tile / p.tiles_m) * kBN;
@@ -594,8 +608,9 @@ constexpr uint32_t kN2SfCols = 48;                                // per stage: 
 constexpr int kN2SfWarps = 8;                                     // scale movers (warps 2..9)
 constexpr int kN2Threads = 32 * (2 + kN2SfWarps + 4);
 
+template <bool MX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
-    gemm_nvfp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+    gemm_fp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                           const __grid_constant__ CUtensorMap tmap_sx, const __grid_constant__ CUtensorMap tmap_sw,
                           const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -659,15 +674,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
           tma_load_2d_2cta(sa, &tmap_x, kt * 128, m0, fb);
           tma_load_2d_2cta(sa + kN2OpA, &tmap_w, kt * 128, nb, fb);
           mbar_arrive_expect_tx(&sf_full[s], kN2SfA + kN2SfB);
-          tma_load_2d(sa + kN2OpA + kN2OpB, &tmap_sx, kt * 16, m0, &sf_full[s]);
-          tma_load_2d(sa + kN2OpA + kN2OpB + kN2SfA, &tmap_sw, kt * 16, nb - 128 * (int)rank, &sf_full[s]);
+          const int sx0 = MX ? (kt >> 1) * 16 : kt * 16;  // 16-byte aligned scale column
+          tma_load_2d(sa + kN2OpA + kN2OpB, &tmap_sx, sx0, m0, &sf_full[s]);
+          tma_load_2d(sa + kN2OpA + kN2OpB + kN2SfA, &tmap_sw, sx0, nb - 128 * (int)rank, &sf_full[s]);
           if (++s == kN2St) { s = 0; ph ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_nvf4(256, kBN);
+      const uint32_t idesc = idesc_fp4(256, kBN, MX);
       int s = 0;
       unsigned ph = 0;
       int it = 0;
@@ -683,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
           const uint32_t sf = tmem + kF4SfCol0 + (uint32_t)s * kN2SfCols;
 #pragma unroll
           for (int j = 0; j < kF4BK / 64; ++j)
-            mma_nvf4_2cta(tmem, ad + 2 * j, bd + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (kt | j) != 0);
+            mma_fp4_2cta<MX>(tmem, ad + 2 * j, bd + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (kt | j) != 0);
           tc_commit_2cta_mc(&op_empty[s], 0x3);
           if (++s == kN2St) { s = 0; ph ^= 1; }
         }
@@ -718,14 +734,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) da[4 * j + i] = reinterpret_cast<const uint32_t*>(&ua[i])[j];
+          for (int i = 0; i < 4; ++i) da[4 * j + i] = sf_word<MX>(ua[i], j, kt);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int c = 8 * j + i;
             if (c < 16)
-              db0[c] = reinterpret_cast<const uint32_t*>(&ub[i])[j];
+              db0[c] = sf_word<MX>(ub[i], j, kt);
             else
-              db1[c - 16] = reinterpret_cast<const uint32_t*>(&ub[i])[j];
+              db1[c - 16] = sf_word<MX>(ub[i], j, kt);
           }
         }
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + kF4SfCol0 + (uint32_t)s * kN2SfCols;
@@ -741,7 +757,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
     }
   } else {
     const int q = warp & 3;
-    const float g = (*p.xg) * (*p.wg);
+    const float g = MX ? 1.0f : (*p.xg) * (*p.wg);
     int it = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
       const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
@@ -1109,13 +1125,70 @@ inline int gemm_num_sms() {
   return v > 0 ? v : 148;
 }
 
+// Raise a GEMM kernel's dynamic shared-memory limit once per (kernel, device).
+inline bool gemm_ensure_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, uint64_t>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : done)
+    if (e.first == kernel && bit && (e.second & bit)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  for (auto& e : done)
+    if (e.first == kernel) {
+      e.second |= bit;
+      return true;
+    }
+  done.emplace_back(kernel, bit);
+  return true;
+}
+
+// NVFP4 (MX = false: E4M3 scales [rows, K/16]) or MXFP4 (MX = true: E8M0
+// scales [rows, K/32]) launch: 2-SM kernel above 128 rows, else 1-SM.
+template <bool MX>
+rq_status launch_fp4(GemmParams p, const uint8_t* xc, const void* xs, const uint8_t* wc, const void* ws, void* Y,
+                     int64_t M, int64_t N, int64_t K, int64_t ldy, rq_out out, cudaStream_t st) {
+  const uint64_t sf_cols = (uint64_t)K / (MX ? 32 : 16);
+  CUtensorMap tx, tw, tsx, tsw, ty;
+  std::memset(&ty, 0, sizeof(ty));
+  p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
+  if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
+  if (M > kBM) {
+    // two SMs per 256 x 256 tile
+    if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tsx, xs, (uint64_t)M, sf_cols, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap_u8(&tsw, ws, (uint64_t)N, sf_cols, 256, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return RQ_ERR_CUDA;
+    p.tiles_m = (int)((M + 255) / 256);
+    p.tiles_n = (int)((N + kBN - 1) / kBN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    const int sms = gemm_num_sms() & ~1;
+    const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
+    if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_fp4_2sm_kernel<MX>), (int)kN2Smem)) return RQ_ERR_CUDA;
+    gemm_fp4_2sm_kernel<MX><<<grid2, kN2Threads, kN2Smem, st>>>(tx, tw, tsx, tsw, ty, p);
+    return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+  }
+  if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_u8(&tsx, xs, (uint64_t)M, sf_cols, kBM, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_u8(&tsw, ws, (uint64_t)N, sf_cols, kBN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return RQ_ERR_CUDA;
+  const int grid = p.num_tiles < gemm_num_sms() ? p.num_tiles : gemm_num_sms();
+  if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_fp4_kernel<MX>), (int)kF4Smem)) return RQ_ERR_CUDA;
+  gemm_fp4_kernel<MX><<<grid, kGemmThreads, kF4Smem, st>>>(tx, tw, tsx, tsw, ty, p);
+  return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
 inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* xg, const uint8_t* wc, const void* ws,
                                const float* wg, int64_t M, int64_t N, int64_t K, rq_format fmt, void* Y, int64_t ldy,
                                rq_out out, cudaStream_t st) {
   if (M < 0 || N < 0 || K <= 0 || ldy < N) return RQ_ERR_INVALID_ARG;
-  if (fmt != RQ_INT4 && fmt != RQ_NVFP4) return RQ_ERR_INVALID_ARG;
+  if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4) return RQ_ERR_INVALID_ARG;
   if (out != RQ_OUT_F32 && out != RQ_OUT_BF16 && out != RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
-  if (fmt == RQ_NVFP4 && out == RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
+  if (fmt != RQ_INT4 && out == RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
   if (M > 0 && N > 0) {
     if (!xc || !xs || !wc || !ws || !Y) return RQ_ERR_INVALID_ARG;
     if (fmt == RQ_NVFP4 && (!xg || !wg)) return RQ_ERR_INVALID_ARG;
@@ -1123,13 +1196,14 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
   if (K > 65536 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (fmt == RQ_INT4 && K % kI4BK != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (fmt == RQ_NVFP4 && K % kF4BK != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt == RQ_MXFP4 && K % 512 != 0) return RQ_ERR_UNSUPPORTED_SHAPE;  // scale rows of K/32 bytes, 16-byte multiples
   if (M == 0 || N == 0) return RQ_OK;
   const size_t esz = out == RQ_OUT_BF16 ? 2 : 4;
   if ((reinterpret_cast<uintptr_t>(xc) | reinterpret_cast<uintptr_t>(wc)) & 15) return RQ_ERR_ALIGNMENT;
   if (reinterpret_cast<uintptr_t>(Y) % esz != 0) return RQ_ERR_ALIGNMENT;
   if (fmt == RQ_INT4 && ((reinterpret_cast<uintptr_t>(xs) & 3) || (reinterpret_cast<uintptr_t>(ws) & 15)))
     return RQ_ERR_ALIGNMENT;
-  if (fmt == RQ_NVFP4 && ((reinterpret_cast<uintptr_t>(xs) | reinterpret_cast<uintptr_t>(ws)) & 15))
+  if (fmt != RQ_INT4 && ((reinterpret_cast<uintptr_t>(xs) | reinterpret_cast<uintptr_t>(ws)) & 15))
     return RQ_ERR_ALIGNMENT;
 
   GemmParams p;
@@ -1170,64 +1244,16 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
       std::memset(&ty, 0, sizeof(ty));
       p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
       if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
-      static bool attr3_done = false;
-      if (!attr3_done) {
-        if (cudaFuncSetAttribute(gemm_int4_2sm_ts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kI3Smem) != cudaSuccess)
-          return RQ_ERR_CUDA;
-        attr3_done = true;
-      }
+      if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int4_2sm_ts_kernel), (int)kI3Smem))
+        return RQ_ERR_CUDA;
       gemm_int4_2sm_ts_kernel<<<grid2, kI3Threads, kI3Smem, st>>>(tx2, tw2, ty, p);
       return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
     }
-    static bool attr_done = false;
-    if (!attr_done) {
-      if (cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI4Smem) !=
-          cudaSuccess)
-        return RQ_ERR_CUDA;
-      attr_done = true;
-    }
+    if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int4_kernel), (int)kI4Smem)) return RQ_ERR_CUDA;
     gemm_int4_kernel<<<grid, kI4Threads, kI4Smem, st>>>(tx, tw, p);
   } else {
-    CUtensorMap tsx, tsw, ty;
-    std::memset(&ty, 0, sizeof(ty));
-    p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
-    if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
-    if (M > kBM) {
-      // two SMs per 256 x 256 tile
-      if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !make_tmap_u8(&tsx, xs, (uint64_t)M, (uint64_t)K / 16, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-          !make_tmap_u8(&tsw, ws, (uint64_t)N, (uint64_t)K / 16, 256, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return RQ_ERR_CUDA;
-      p.tiles_m = (int)((M + 255) / 256);
-      p.tiles_n = (int)((N + kBN - 1) / kBN);
-      p.num_tiles = p.tiles_m * p.tiles_n;
-      const int sms = gemm_num_sms() & ~1;
-      const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
-      static bool attr2_done = false;
-      if (!attr2_done) {
-        if (cudaFuncSetAttribute(gemm_nvfp4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kN2Smem) != cudaSuccess)
-          return RQ_ERR_CUDA;
-        attr2_done = true;
-      }
-      gemm_nvfp4_2sm_kernel<<<grid2, kN2Threads, kN2Smem, st>>>(tx, tw, tsx, tsw, ty, p);
-      return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
-    }
-    if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, kBN, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_u8(&tsx, xs, (uint64_t)M, (uint64_t)K / 16, kBM, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_tmap_u8(&tsw, ws, (uint64_t)N, (uint64_t)K / 16, kBN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return RQ_ERR_CUDA;
-    static bool attr_done = false;
-    if (!attr_done) {
-      if (cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kF4Smem) !=
-          cudaSuccess)
-        return RQ_ERR_CUDA;
-      attr_done = true;
-    }
-    gemm_nvfp4_kernel<<<grid, kGemmThreads, kF4Smem, st>>>(tx, tw, tsx, tsw, ty, p);
+    return fmt == RQ_MXFP4 ? launch_fp4<true>(p, xc, xs, wc, ws, Y, M, N, K, ldy, out, st)
+                           : launch_fp4<false>(p, xc, xs, wc, ws, Y, M, N, K, ldy, out, st);
   }
   return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }

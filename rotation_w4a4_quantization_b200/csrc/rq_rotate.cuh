@@ -7,6 +7,7 @@
 // then one of
 //   INT4  : per-row symmetric, s = amax/7, q = rint(x/s)          (tokens / output channels)
 //   NVFP4 : E2M1 codes, one E4M3 scale per 16 values, fp32 tensor scale g
+//   MXFP4 : E2M1 codes, one E8M0 (power-of-two) scale per 32 values
 //   KV4   : per-vector asymmetric, z = min, s = (max-min)/15 (fp16 scale and zero)
 //   F32   : the rotated values themselves (parity checks)
 //   AMAX  : only the global max |X~| (first pass of dynamic NVFP4)
@@ -50,7 +51,7 @@ namespace rq {
 #define RQ_FULL_WIDTH_THREADS 256
 #endif
 
-enum RotMode : int { kModeInt4 = 0, kModeNvfp4 = 1, kModeF32 = 2, kModeAmax = 3, kModeKv4 = 4 };
+enum RotMode : int { kModeInt4 = 0, kModeNvfp4 = 1, kModeF32 = 2, kModeAmax = 3, kModeKv4 = 4, kModeMxfp4 = 5 };
 
 struct RotParams {
   const uint8_t* x;    // bf16 input (bytes)
@@ -64,7 +65,7 @@ struct RotParams {
   const int8_t* signs; // [K]
   uint8_t* codes;      // [rows, K/2]
   float* scales_f32;   // INT4: [rows]
-  uint8_t* scales_e4m3;// NVFP4: [rows, K/16]
+  uint8_t* scales_e4m3;// NVFP4: [rows, K/16]; MXFP4: E8M0 [rows, K/32]
   __half* kv_scale;    // KV4: [rows]
   __half* kv_zero;     // KV4: [rows]
   float* out_f32;      // F32: [rows, ldo]
@@ -302,6 +303,46 @@ __device__ __forceinline__ void quant_nvfp4_store(const float (&v)[128], float c
 #pragma unroll
   for (int j = 0; j < 4; ++j) out[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
   *reinterpret_cast<uint2*>(dst_scales) = make_uint2(sc_lo, sc_hi);
+}
+
+// MXFP4 quantization of v (true value = v * c * chi): 4 groups of 32 with an
+// E8M0 scale 2^e each, e = floor(log2(amax)) - 2 clamped to [-127, 127].
+// floor(log2(amax)) is the exponent field of the fp32 amax (a zero or
+// subnormal amax gives -127 - 2 and clamps to -127).  x / 2^e is exact, so the
+// only rounding left is the E2M1 conversion.  Writes 64 bytes of codes and 4
+// bytes of scales.
+__device__ __forceinline__ void quant_mxfp4_store(const float (&v)[128], float c, int m, uint8_t* dst_codes,
+                                                  uint8_t* dst_scales) {
+  uint32_t words[16];
+  uint32_t sc = 0;
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      a0 = fmaxf(a0, fabsf(v[32 * gi + e]));
+      a1 = fmaxf(a1, fabsf(v[32 * gi + e + 1]));
+    }
+    const float amax_b = fmaxf(a0, a1) * c;  // true block max
+    int ex = (int)((__float_as_uint(amax_b) >> 23) & 0xFFu) - 127 - 2;
+    ex = min(max(ex, -127), 127);
+    sc |= (uint32_t)(ex + 127) << (8 * gi);
+    // 2^-ex: a normal fp32 for ex <= 126; 2^-127 is the subnormal 0x00400000
+    const float inv = ex == 127 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - ex) << 23);
+    const float ci = c * inv;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int j = 4 * gi + q4;
+      const float mul = with_sign(ci, chi_signbit(j, m));
+      const float* s = &v[8 * j];
+      words[j] = pack8_e2m1(s[0] * mul, s[1] * mul, s[2] * mul, s[3] * mul, s[4] * mul, s[5] * mul, s[6] * mul,
+                            s[7] * mul);
+    }
+  }
+  uint4* out = reinterpret_cast<uint4*>(dst_codes);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) out[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+  *reinterpret_cast<uint32_t*>(dst_scales) = sc;
 }
 
 // KV4: asymmetric per-vector quantization (true value = v * c * chi).
@@ -614,6 +655,10 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
         if (valid)
           quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
                             p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+      } else if (MODE == kModeMxfp4) {
+        if (valid)
+          quant_mxfp4_store(v, c, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                            p.scales_e4m3 + row * (p.K / 32) + (size_t)b * 4);
       } else if (MODE == kModeF32) {
         if (valid) store_f32_block(v, c, m, p.out_f32 + row * p.ldo + (size_t)b * 128);
       } else if (MODE == kModeAmax) {

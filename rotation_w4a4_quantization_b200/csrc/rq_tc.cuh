@@ -95,6 +95,12 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);    // M >> 4; scale-factor ids 0; K = 64
 }
 
+// Block-scaled FP4 descriptor: NVFP4 (UE4M3 scale per 16) or MXFP4 (UE8M0
+// scale per 32, bit 23).
+__host__ __device__ constexpr uint32_t idesc_fp4(int M, int N, bool mx) {
+  return idesc_nvf4(M, N) | (mx ? (1u << 23) : 0u);
+}
+
 // ---------------------------------------------------------------------------
 // MMAs (issued by one thread)
 // ---------------------------------------------------------------------------
@@ -222,6 +228,18 @@ __device__ __forceinline__ void mma_i8_2cta_ts(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 
+// E2M1 x E2M1 with an E8M0 scale per 32 values (kind::mxf4, scale_vec 2X).
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // TMA 2-D load issued by either CTA of a pair whose completion (transaction
 // bytes) is counted on the even CTA's barrier `bar_cluster` (a shared::cluster
 // address).  No multicast.
@@ -242,6 +260,35 @@ __device__ __forceinline__ void mma_nvf4_2cta(uint32_t d_tmem, uint64_t a_desc, 
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_2cta(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+template <bool MX>
+__device__ __forceinline__ void mma_fp4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                        uint32_t acc) {
+  if (MX)
+    mma_mxf4(d, a, b, idesc, sfa, sfb, acc);
+  else
+    mma_nvf4(d, a, b, idesc, sfa, sfb, acc);
+}
+
+template <bool MX>
+__device__ __forceinline__ void mma_fp4_2cta(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                             uint32_t sfb, uint32_t acc) {
+  if (MX)
+    mma_mxf4_2cta(d, a, b, idesc, sfa, sfb, acc);
+  else
+    mma_nvf4_2cta(d, a, b, idesc, sfa, sfb, acc);
 }
 
 }  // namespace rq

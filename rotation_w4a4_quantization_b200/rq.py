@@ -15,7 +15,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librq.so")
 
-RQ_INT4, RQ_NVFP4 = 0, 1
+RQ_INT4, RQ_NVFP4, RQ_MXFP4 = 0, 1, 2
 RQ_OUT_F32, RQ_OUT_BF16, RQ_OUT_I32_ACC = 0, 1, 2
 RQ_SCALE_DYNAMIC, RQ_SCALE_STATIC = 0, 1
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3: "RQ_ERR_ALIGNMENT",
@@ -75,7 +75,7 @@ def _stream(t=None):
 
 
 def _fmt(fmt):
-    return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4}[fmt] if isinstance(fmt, str) else int(fmt)
+    return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4, "mxfp4": RQ_MXFP4}[fmt] if isinstance(fmt, str) else int(fmt)
 
 
 def init(device=0):
@@ -96,8 +96,10 @@ def _alloc_quant_outputs(rows, k, fmt, device):
     codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=device)
     if fmt == RQ_INT4:
         scales = torch.empty((rows,), dtype=torch.float32, device=device)
-    else:
+    elif fmt == RQ_NVFP4:
         scales = torch.empty((rows, k // 16), dtype=torch.uint8, device=device)
+    else:
+        scales = torch.empty((rows, k // 32), dtype=torch.uint8, device=device)
     return codes, scales
 
 
@@ -106,6 +108,7 @@ def rotate_quantize(x, signs, block=128, fmt="int4", gmode="dynamic", gscale=Non
 
     INT4: codes uint8 [M, K/2], scales fp32 [M], gscale None.
     NVFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/16] (E4M3), gscale fp32 [1].
+    MXFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/32] (E8M0), gscale None.
     """
     _require_cuda(x, signs)
     f = _fmt(fmt)

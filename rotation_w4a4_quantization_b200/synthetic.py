@@ -38,6 +38,7 @@ WORKLOADS = {
     "down_proj_int4": dict(index=3, M=4096, K=12288, N=4096, block=128, fmt="int4"),
     "q_proj_nvfp4": dict(index=4, M=2048, K=4096, N=4096, block=128, fmt="nvfp4"),
     "kv4": dict(index=5, B=16, H=32, S=4096, D=128),
+    "q_proj_mxfp4": dict(index=6, M=2048, K=4096, N=4096, block=128, fmt="mxfp4"),
 }
 
 
@@ -68,7 +69,7 @@ def activations(name, rows=None, device="cpu", seed_offset=0):
     x = torch.randn((m, k), generator=g, device=device, dtype=torch.float32)
     if name == "tiny_int4":
         x[:, [3, 77, 200, 411]] *= 50.0
-    elif name in ("q_proj_int4", "q_proj_nvfp4"):
+    elif name in ("q_proj_int4", "q_proj_nvfp4", "q_proj_mxfp4"):
         gp = _gen(3000 + w["index"], "cpu")
         ch = torch.randperm(k, generator=gp)[:8]
         mult = 20.0 + 40.0 * torch.rand((8,), generator=gp, dtype=torch.float64)

@@ -92,6 +92,33 @@ def check_nvfp4_quant(codes_gpu, sc_gpu, g_gpu, xr, g_ref=None):
     return n_s, n_e
 
 
+def check_mxfp4_quant(codes_gpu, sc_gpu, xr):
+    """MXFP4 parity: E8M0 scales identical except at oracle-flagged
+    power-of-two ties (by one exponent step), whose blocks are then excused
+    from the code comparison; E2M1 codes identical modulo flagged ties."""
+    e, sc, tie_e, tie_s = quant.mxfp4_rows(xr)
+    scg = np.asarray(sc_gpu, dtype=np.int64)
+    bad = scg != sc
+    assert not (bad & ~tie_s).any(), "E8M0 scale mismatch outside tie bands"
+    assert np.all(np.abs(scg - sc) <= 1)
+    excused = np.repeat(bad, 32, axis=1)
+    eg = quant.unpack_nibbles(codes_gpu, signed=False)
+    n_e = check_codes(eg, e, tie_e, rank=e2m1_rank, excused=excused, what="e2m1 codes")
+    return int(bad.sum()), n_e
+
+
+def mxfp4_tie_bounds(e, sc, tie_e, tie_s):
+    """An E2M1 tie moves a value by at most one grid step (<= 2) times the
+    block scale; an E8M0 tie doubles or halves the block scale, moving each
+    value by at most its magnitude plus a grid step at the larger scale."""
+    xhat = quant.mxfp4_dequant(e, sc)
+    sval = np.repeat(formats.e8m0_values(sc), 32, axis=1)
+    d = tie_e * 2.0 * sval
+    blk = np.repeat(tie_s, 32, axis=1)
+    d = d + blk * (np.abs(xhat) + 4.0 * sval)
+    return xhat, d
+
+
 def _fp16_ulp(v):
     h = np.asarray(v, dtype=np.float64).astype(np.float16)
     return np.abs(np.nextafter(h, np.float16(np.inf)).astype(np.float64) - h.astype(np.float64))
