@@ -99,7 +99,9 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
           *reinterpret_cast<int4*>(dst + j) = make_int4((int)r[j] >> 8, (int)r[j + 1] >> 8, (int)r[j + 2] >> 8,
                                                         (int)r[j + 3] >> 8);
       } else {
-        for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = (int)r[j] >> 8;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < p.N) dst[j] = (int)r[j] >> 8;
       }
       continue;
     }
@@ -120,6 +122,7 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
           v[j + 3] *= s.w;
         }
       } else {
+#pragma unroll
         for (int j = 0; j < 32; ++j) v[j] *= (c0 + j < p.N) ? colscale[c0 + j] : 0.f;
       }
     } else {
@@ -133,7 +136,9 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
         for (int j = 0; j < 32; j += 4)
           *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       } else {
-        for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = v[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < p.N) dst[j] = v[j];
       }
     } else {
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + (int64_t)row * p.ldy + c0;
@@ -149,7 +154,9 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
                          *reinterpret_cast<uint32_t*>(&b2), *reinterpret_cast<uint32_t*>(&b3));
         }
       } else {
-        for (int j = 0; j < 32 && c0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < p.N) dst[j] = __float2bfloat16_rn(v[j]);
       }
     }
   }
@@ -417,9 +424,12 @@ done:
 // half of the word.
 template <bool MX>
 __device__ __forceinline__ uint32_t sf_word(const uint4& row16, int j, int kt) {
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(&row16);
+  // j is a compile-time constant in the callers' unrolled loops; the k-tile
+  // parity only selects between two statically indexed words, so the staged
+  // scales stay in registers
+  const uint32_t w[4] = {row16.x, row16.y, row16.z, row16.w};
   if (!MX) return w[j];
-  const uint32_t h = w[2 * (kt & 1) + (j >> 1)];
+  const uint32_t h = (kt & 1) ? w[2 + (j >> 1)] : w[j >> 1];
   return (j & 1) ? (h >> 16) : (h & 0xFFFFu);
 }
 
