@@ -63,17 +63,20 @@ def load_peaks():
 # ncu captures summarised in profiles/, with a fingerprint of the kernel sources
 # they were taken on; a number is reported only while those sources are
 # unchanged.  kv4 was captured on a quarter of one tensor and is scaled by the
-# vectors processed; q_proj_nvfp4 is the mean of its two launches (max pass,
-# quantize pass).
+# vectors processed.
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
+_ROT, _GEM = "96ccf4968826d44e", "c6e805e14224d165"
 TRAFFIC = {
-    ("hadamard_quant", "q_proj_int4"): (16846848, "6171dfa5d6c3486c"),
-    ("hadamard_quant", "down_proj_int4"): (100730880 + 4858368, "6171dfa5d6c3486c"),
-    ("hadamard_quant", "kv4"): ((134337280 + 12498688) * 4, "6171dfa5d6c3486c"),
-    ("hadamard_quant", "q_proj_nvfp4"): ((16825600 + 16836608) // 2, "6171dfa5d6c3486c"),
-    ("gemm", "q_proj_int4"): (12637696 + 8704, "046b718da8bfd820"),
-    ("gemm", "down_proj_int4"): (50567424 + 8494592, "046b718da8bfd820"),
+    ("hadamard_quant", "q_proj_int4"): (16847104, _ROT),
+    ("hadamard_quant", "down_proj_int4"): (100728576 + 5582336, _ROT),
+    ("hadamard_quant", "kv4"): ((134419968 + 12322560) * 4, _ROT),
+    ("hadamard_quant", "q_proj_nvfp4"): (16830464, _ROT),
+    ("hadamard_quant", "q_proj_mxfp4"): (16831744, _ROT),
+    ("gemm", "q_proj_int4"): (12652288, _GEM),
+    ("gemm", "down_proj_int4"): (50722816 + 10223616, _GEM),
+    ("gemm", "q_proj_nvfp4"): (14189056, _GEM),
+    ("gemm", "q_proj_mxfp4"): (13400320, _GEM),
 }
 
 
@@ -155,9 +158,11 @@ class Workload:
         return 1
 
     def quant_kernel(self):
+        if self.kv:
+            return "rotate_kernel<KV4>"
         if self.fmt == "nvfp4" and self.nvfp4_one_pass():
             return "rotate_nvfp4_resident_kernel"
-        return "rotate_kernel<full width>" if (not self.kv and self.block == 0) else "rotate_kernel<128-blocks>"
+        return "rotate_kernel<full width>" if self.block == 0 else "rotate_kernel<128-blocks>"
 
     def gemm_launches(self):
         return 0 if self.kv else 1
@@ -475,13 +480,14 @@ def measure_e2e(wl, rq, dev, stream, K):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
-def workload_config(args, wl):
+def workload_config(args, wl=None):
+    """The `config` object of both arms (the reference arm passes no Workload)."""
     c = dict(syn.WORKLOADS[args.workload])
     c.pop("index", None)
     cfg = {"workload": args.workload}
     cfg.update(c)
-    if not wl.kv:
-        cfg["block"] = "full" if wl.block == 0 else wl.block
+    if args.workload != "kv4":
+        cfg["block"] = "full" if c["block"] == 0 else c["block"]
         cfg["y_dtype"] = args.y_dtype
         cfg["weights"] = "rotated+quantized once before timing (offline side)"
     cfg["l2"] = "flushed between steps (256 MiB memset, outside the kernel events)"
@@ -506,7 +512,7 @@ def run_reference(args, world, rank):
         "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(1e3 * secs / K, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
-        "config": {"workload": args.workload, "sample_rows": rows},
+        "config": workload_config(args),
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
