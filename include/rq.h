@@ -186,6 +186,32 @@ RQ_API rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H,
                                 void* scale_dev, void* zero_dev, rq_stream_t stream);
 
 /*
+ * rq_kv4_decode_attention: one decoding step of attention over the 4-bit KV
+ * cache written by rq_kv_rotate_quantize ("QuaRot", "Activation scheme": the
+ * KV cache is stored rotated; "Rotations for 4-Bit Activations", "A rotation
+ * changes nothing": q.K^T = (q.Q).(K.Q)^T).  For each (b, h): the query is
+ * rotated with the same per-head Q = diag(s).H_128/sqrt(128) as the cache,
+ * the cached vectors dequantize as z + s*q, p = softmax(q~.K~^T * scale) over
+ * the S cached tokens, and o = (p.V~).Q^T is returned in the original basis.
+ *  q_dev       bf16 [B, H, 128] contiguous, 16-byte aligned.
+ *  kcodes_dev, vcodes_dev   uint8 [B, H, S, 64] contiguous, 16-byte aligned;
+ *  kscale_dev, kzero_dev, vscale_dev, vzero_dev   fp16 [B, H, S] contiguous
+ *              (the layouts rq_kv_rotate_quantize writes).
+ *  signs_dev   int8 [128], 16-byte aligned: the signs the cache was rotated with.
+ *  softmax_scale  > 0, or 0 for 1/sqrt(128).
+ *  out_dev     [B, H, 128] fp32 (RQ_OUT_F32) or bf16 (RQ_OUT_BF16).
+ *  workspace_dev  rq_kv4_attention_workspace_bytes(B, H, S) bytes, 16-byte aligned.
+ *  S >= 1 (S = 0 is RQ_ERR_INVALID_ARG); B = 0 or H = 0 is a no-op.
+ * Two kernels: per-chunk partial softmax sums, then a merge that rotates back.
+ */
+RQ_API size_t rq_kv4_attention_workspace_bytes(int64_t B, int64_t H, int64_t S);
+RQ_API rq_status rq_kv4_decode_attention(const void* q_dev, int64_t B, int64_t H, int64_t S, const uint8_t* kcodes_dev,
+                                         const void* kscale_dev, const void* kzero_dev, const uint8_t* vcodes_dev,
+                                         const void* vscale_dev, const void* vzero_dev, const int8_t* signs_dev,
+                                         float softmax_scale, void* out_dev, rq_out out, void* workspace_dev,
+                                         rq_stream_t stream);
+
+/*
  * rq_rotate_f32: the rotation alone, X~ = X.Q as fp32 [M, ldo] (ldo a multiple
  * of 4, out_dev 16-byte aligned).  Same X, K, signs and block rules as
  * rq_rotate_quantize (block 0 allowed for K a power of two in [256, 4096]).

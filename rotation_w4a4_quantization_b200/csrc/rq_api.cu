@@ -16,6 +16,7 @@
 #include "rq_common.cuh"
 #include "rq_rotate.cuh"
 #include "rq_gemm.cuh"
+#include "rq_attn.cuh"
 
 namespace {
 
@@ -407,4 +408,58 @@ rq_status rq_get_device_error(rq_stream_t stream) {
   return v ? RQ_ERR_TIMEOUT : RQ_OK;
 }
 
+// ---------------------------------------------------------------------------
+// KV4 decode attention
+// ---------------------------------------------------------------------------
+size_t rq_kv4_attention_workspace_bytes(int64_t B, int64_t H, int64_t S) {
+  if (B <= 0 || H <= 0 || S <= 0) return 0;
+  const int64_t nchunks = (S + kAttnChunk - 1) / kAttnChunk;
+  return (size_t)(B * H * nchunks) * kAttnPart * sizeof(float);
+}
+
+rq_status rq_kv4_decode_attention(const void* q_dev, int64_t B, int64_t H, int64_t S, const uint8_t* kcodes_dev,
+                                  const void* kscale_dev, const void* kzero_dev, const uint8_t* vcodes_dev,
+                                  const void* vscale_dev, const void* vzero_dev, const int8_t* signs_dev,
+                                  float softmax_scale, void* out_dev, rq_out out, void* workspace_dev,
+                                  rq_stream_t stream) {
+  if (B < 0 || H < 0 || S < 0) return RQ_ERR_INVALID_ARG;
+  if (out != RQ_OUT_F32 && out != RQ_OUT_BF16) return RQ_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.0f) || !std::isfinite(softmax_scale)) return RQ_ERR_INVALID_ARG;
+  if (B == 0 || H == 0) return RQ_OK;
+  if (S == 0) return RQ_ERR_INVALID_ARG;  // softmax over no tokens
+  if (!q_dev || !kcodes_dev || !kscale_dev || !kzero_dev || !vcodes_dev || !vscale_dev || !vzero_dev || !signs_dev ||
+      !out_dev || !workspace_dev)
+    return RQ_ERR_INVALID_ARG;
+  const int64_t BH = B * H;
+  const int64_t nchunks = (S + kAttnChunk - 1) / kAttnChunk;
+  if (BH * nchunks > (int64_t)INT32_MAX || S > ((int64_t)1 << 40) / BH) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(q_dev, 16) || !aligned(kcodes_dev, 16) || !aligned(vcodes_dev, 16) || !aligned(signs_dev, 16) ||
+      !aligned(workspace_dev, 16) || !aligned(kscale_dev, 2) || !aligned(kzero_dev, 2) || !aligned(vscale_dev, 2) ||
+      !aligned(vzero_dev, 2) || !aligned(out_dev, out == RQ_OUT_BF16 ? 2 : 4))
+    return RQ_ERR_ALIGNMENT;
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q_dev);
+  p.kc = kcodes_dev;
+  p.ks = static_cast<const __half*>(kscale_dev);
+  p.kz = static_cast<const __half*>(kzero_dev);
+  p.vc = vcodes_dev;
+  p.vs = static_cast<const __half*>(vscale_dev);
+  p.vz = static_cast<const __half*>(vzero_dev);
+  p.signs = signs_dev;
+  const double sc = softmax_scale > 0.0f ? (double)softmax_scale : 1.0 / std::sqrt(128.0);
+  p.qscale = (float)(sc * 1.4426950408889634 / std::sqrt(128.0));
+  p.S = S;
+  p.nchunks = (int)nchunks;
+  p.part = static_cast<float*>(workspace_dev);
+  p.out = out_dev;
+  p.out_bf16 = out == RQ_OUT_BF16 ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  kv4_attn_partial_kernel<<<(unsigned)(BH * nchunks), 128, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return RQ_ERR_CUDA;
+  kv4_attn_combine_kernel<<<(unsigned)BH, 128, 0, st>>>(p);
+  return last_launch_status();
+}
+
 }  // extern "C"
+

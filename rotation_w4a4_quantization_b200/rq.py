@@ -22,7 +22,7 @@ STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3:
           4: "RQ_ERR_UNSUPPORTED_DEVICE", 5: "RQ_ERR_CUDA", 6: "RQ_ERR_TIMEOUT"}
 EXPORTED = ["rq_init", "rq_status_string", "rq_workspace_bytes", "rq_rotate_quantize", "rq_prepare_weights",
             "rq_w4a4_gemm", "rq_kv_rotate_quantize", "rq_rotate_f32", "rq_get_device_error",
-            "rq_rotate_quantize_nvfp4_noalloc"]
+            "rq_rotate_quantize_nvfp4_noalloc", "rq_kv4_attention_workspace_bytes", "rq_kv4_decode_attention"]
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("librq.so not built: run `python -m rotation_w4a4_quantization_b200.build`")
@@ -49,6 +49,10 @@ lib.rq_rotate_f32.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i64, _p]
 lib.rq_rotate_f32.restype = _i
 lib.rq_rotate_quantize_nvfp4_noalloc.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p]
 lib.rq_rotate_quantize_nvfp4_noalloc.restype = _i
+lib.rq_kv4_attention_workspace_bytes.argtypes = [_i64, _i64, _i64]
+lib.rq_kv4_attention_workspace_bytes.restype = ctypes.c_size_t
+lib.rq_kv4_decode_attention.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, ctypes.c_float, _p, _i, _p, _p]
+lib.rq_kv4_decode_attention.restype = _i
 lib.rq_get_device_error.argtypes = [_p]
 lib.rq_get_device_error.restype = _i
 
@@ -197,6 +201,28 @@ def rotate_quantize_nvfp4_noalloc(x, signs, out=None, gscale=None):
     _check(lib.rq_rotate_quantize_nvfp4_noalloc(_ptr(x), m, k, x.stride(0), _ptr(signs), _ptr(codes), _ptr(scales),
                                                 _ptr(gscale), _stream(x)), "rq_rotate_quantize_nvfp4_noalloc")
     return codes, scales, gscale
+
+
+def kv4_decode_attention(q, kcache, vcache, signs, softmax_scale=0.0, out_dtype="f32", out=None, workspace=None):
+    """One decode step over the KV4 cache.  q bf16 [B, H, 128]; kcache / vcache
+    the (codes [B,H,S,64], scale fp16 [B,H,S], zero fp16 [B,H,S]) triples of
+    kv_rotate_quantize.  Returns o [B, H, 128] (fp32 or bf16) in the original
+    basis."""
+    kc, ks, kz = kcache
+    vc, vs, vz = vcache
+    _require_cuda(q, kc, ks, kz, vc, vs, vz, signs)
+    b, h, d = q.shape
+    s = kc.shape[2]
+    o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16}[out_dtype]
+    if out is None:
+        out = torch.empty((b, h, d), dtype=torch.float32 if o == RQ_OUT_F32 else torch.bfloat16, device=q.device)
+    if workspace is None:
+        nb = int(lib.rq_kv4_attention_workspace_bytes(b, h, s))
+        workspace = torch.empty((max(nb, 16),), dtype=torch.uint8, device=q.device)
+    _check(lib.rq_kv4_decode_attention(_ptr(q), b, h, s, _ptr(kc), _ptr(ks), _ptr(kz), _ptr(vc), _ptr(vs), _ptr(vz),
+                                       _ptr(signs), float(softmax_scale), _ptr(out), o, _ptr(workspace), _stream(q)),
+           "rq_kv4_decode_attention")
+    return out
 
 
 def get_device_error(stream=None):
