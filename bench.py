@@ -107,7 +107,28 @@ class Workload:
         self.cfg = syn.WORKLOADS[name]
         self.y_dtype = y_dtype
         self.kv = name == "kv4"
-        if self.kv:
+        self.kvdec = name == "kv4_decode"
+        if self.kvdec:
+            c = self.cfg
+            self.signs = syn.workload_signs(name).to(device)
+            k = syn.kv(device=device, which=0, seed_offset=seed_offset)
+            self.kcache = rq.kv_rotate_quantize(k, self.signs)
+            del k
+            v = syn.kv(device=device, which=1, seed_offset=seed_offset)
+            self.vcache = rq.kv_rotate_quantize(v, self.signs)
+            del v
+            g = torch.Generator(device=device)
+            g.manual_seed(4000 + c["index"] + seed_offset)
+            self.q = torch.randn((c["B"], c["H"], c["D"]), generator=g, device=device).to(torch.bfloat16)
+            self.out = torch.empty((c["B"], c["H"], c["D"]), dtype=torch.float32, device=device)
+            nws = int(rq.lib.rq_kv4_attention_workspace_bytes(c["B"], c["H"], c["S"]))
+            self.attn_ws = torch.empty((nws,), dtype=torch.uint8, device=device)
+            bh = c["B"] * c["H"]
+            # the whole cache (K and V: 64 B of codes + fp16 scale and zero per token and head), q and o
+            self.quant_bytes = bh * c["S"] * 2 * (64 + 4) + bh * c["D"] * (2 + 4)
+            self.gemm_ops = 0
+            self.h2d_bytes = self.q.numel() * 2
+        elif self.kv:
             c = self.cfg
             self.k = syn.kv(device=device, which=0, seed_offset=seed_offset)
             self.v = syn.kv(device=device, which=1, seed_offset=seed_offset)
@@ -142,6 +163,8 @@ class Workload:
         self.d2h_bytes = 0
 
     def nvfp4_one_pass(self):
+        if self.kv or self.kvdec:
+            return False
         # librq quantizes dynamic NVFP4 in one launch when each SM's share of
         # the rows (plus the sign table) fits its 220 KiB of shared memory;
         # otherwise a max launch precedes the quantize launch
@@ -151,13 +174,15 @@ class Workload:
         return rpc * k * 2 + (k // 128) * 256 + 32 <= 220 * 1024
 
     def quant_launches(self):
-        if self.kv:
+        if self.kv or self.kvdec:
             return 2
         if self.fmt == "nvfp4":
             return 1 if self.nvfp4_one_pass() else 2
         return 1
 
     def quant_kernel(self):
+        if self.kvdec:
+            return "kv4_attn_partial_kernel + kv4_attn_combine_kernel"
         if self.kv:
             return "rotate_kernel<KV4>"
         if self.fmt == "nvfp4" and self.nvfp4_one_pass():
@@ -165,10 +190,14 @@ class Workload:
         return "rotate_kernel<full width>" if self.block == 0 else "rotate_kernel<128-blocks>"
 
     def gemm_launches(self):
-        return 0 if self.kv else 1
+        return 0 if (self.kv or self.kvdec) else 1
 
     def quant(self):
         rq = self.rq
+        if self.kvdec:
+            rq.kv4_decode_attention(self.q, self.kcache, self.vcache, self.signs, out=self.out,
+                                    workspace=self.attn_ws)
+            return None
         if self.kv:
             rq.kv_rotate_quantize(self.k, self.signs, out=self.outs[0])
             rq.kv_rotate_quantize(self.v, self.signs, out=self.outs[1])
@@ -177,11 +206,13 @@ class Workload:
                                   out=self.xq_out, workspace=self.ws)
 
     def gemm(self, xq):
-        if self.kv:
+        if self.kv or self.kvdec:
             return None
         return self.rq.w4a4_gemm(xq, self.wq, self.fmt, self.y_dtype, y=self.y)
 
     def result(self):
+        if self.kvdec:
+            return self.out
         return self.outs[0][0] if self.kv else self.y
 
 
@@ -253,6 +284,22 @@ def oracle_sample(name, rows):
     """Time the oracle (as it stands) on `rows` rows of the workload; returns (GB/s, TOPS, seconds, desc, threads)."""
     from oracle import gemm as ogemm, hadamard as ohad, quant as oquant
     c = syn.WORKLOADS[name]
+    if name == "kv4_decode":
+        # rows = heads of one batch entry over the full sequence length
+        from oracle import attention as oattn
+        s = syn.workload_signs(name).numpy()
+        k = syn.kv(batch=1, heads=rows, which=0).to(torch.float64).numpy()
+        v = syn.kv(batch=1, heads=rows, which=1).to(torch.float64).numpy()
+        caches = []
+        for x in (k, v):
+            q4, sh, zh, _, _ = oquant.kv4_vectors(oattn.rotate_heads(x, s).reshape(-1, 128))
+            caches += [q4.reshape(x.shape), sh.reshape(x.shape[:-1]), zh.reshape(x.shape[:-1])]
+        qv = np.random.default_rng(0).standard_normal((1, rows, 128))
+        t0 = time.perf_counter()
+        oattn.kv4_decode_attention(qv, *caches, s)
+        dt = time.perf_counter() - t0
+        nbytes = rows * c["S"] * 2 * (64 + 4)
+        return nbytes / dt / 1e9, None, dt, "1 x %d heads x %d tokens of the cache" % (rows, c["S"])
     if name == "kv4":
         kv = syn.kv(batch=1, heads=4, seq=rows)
         s = syn.workload_signs(name).numpy()
@@ -314,7 +361,7 @@ def blas_threads():
 
 def sample_rows(name):
     return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096,
-            "q_proj_mxfp4": 256}[name]
+            "q_proj_mxfp4": 256, "kv4_decode": 32}[name]
 
 
 # --------------------------------------------------------------------------- main
@@ -454,7 +501,10 @@ def measure_e2e(wl, rq, dev, stream, K):
     """Same metric through the public API with host buffers: the timed region holds,
     per step, the pinned host -> device copy of the step's input, the path, and the
     device -> host copy of its result."""
-    if wl.kv:
+    if wl.kvdec:
+        host_in = [wl.q.cpu().pin_memory()]
+        dev_in = [wl.q]
+    elif wl.kv:
         host_in = [wl.k.cpu().pin_memory(), wl.v.cpu().pin_memory()]
         dev_in = [wl.k, wl.v]
     else:
@@ -486,7 +536,7 @@ def workload_config(args, wl=None):
     c.pop("index", None)
     cfg = {"workload": args.workload}
     cfg.update(c)
-    if args.workload != "kv4":
+    if args.workload not in ("kv4", "kv4_decode"):
         cfg["block"] = "full" if c["block"] == 0 else c["block"]
         cfg["y_dtype"] = args.y_dtype
         cfg["weights"] = "rotated+quantized once before timing (offline side)"

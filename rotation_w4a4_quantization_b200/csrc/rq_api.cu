@@ -40,8 +40,10 @@ int num_sms_of_current_device() {
   return v;
 }
 
-// Raise a kernel's dynamic shared memory limit once per (kernel, device).
-bool ensure_smem(const void* kernel) {
+// Raise a kernel's dynamic shared memory limit once per (kernel, device).  The
+// default is the whole per-CTA budget; kernels with static shared memory pass
+// what they need (static + dynamic must stay within the per-CTA maximum).
+bool ensure_smem(const void* kernel, int bytes = (int)kSmemBudget + 7 * 1024) {
   static std::mutex mu;
   static std::vector<std::pair<const void*, uint64_t>> done;
   int dev = 0;
@@ -50,9 +52,7 @@ bool ensure_smem(const void* kernel) {
   std::lock_guard<std::mutex> lock(mu);
   for (auto& e : done)
     if (e.first == kernel && bit && (e.second & bit)) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget + 7 * 1024) !=
-      cudaSuccess)
-    return false;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
   for (auto& e : done)
     if (e.first == kernel) {
       e.second |= bit;
@@ -455,7 +455,8 @@ rq_status rq_kv4_decode_attention(const void* q_dev, int64_t B, int64_t H, int64
   p.out = out_dev;
   p.out_bf16 = out == RQ_OUT_BF16 ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  kv4_attn_partial_kernel<<<(unsigned)(BH * nchunks), 128, 0, st>>>(p);
+  if (!ensure_smem(reinterpret_cast<const void*>(kv4_attn_partial_kernel), (int)kAttnSmem)) return RQ_ERR_CUDA;
+  kv4_attn_partial_kernel<<<(unsigned)(BH * nchunks), 128, kAttnSmem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return RQ_ERR_CUDA;
   kv4_attn_combine_kernel<<<(unsigned)BH, 128, 0, st>>>(p);
   return last_launch_status();

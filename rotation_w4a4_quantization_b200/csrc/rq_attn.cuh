@@ -10,15 +10,20 @@
 // back at the end.  The cache is what rq_kv_rotate_quantize writes.
 //
 // Split-S ("flash-decoding") in two kernels:
-// * kv4_attn_partial_kernel: one CTA (4 warps) per 256 cached tokens of one
-//   (batch, head).  Warp 0 rotates q with shuffles (two butterfly stages in
+// * kv4_attn_partial_kernel: one CTA (4 warps) per 1024 cached tokens of one
+//   (batch, head); the code rows stream through a three-stage shared-memory
+//   ring of 128-token stages (cp.async.bulk; a "full" and a per-warp "read"
+//   mbarrier per stage, bounded waits, no CTA-wide barrier in the loop), the
+//   per-token fp16 scales and zeros through registers one stage ahead.  Warp 0
+//   rotates q with shuffles (two butterfly stages in
 //   registers, five across lanes) and folds 1/sqrt(128), the softmax scale and
 //   log2(e) into it, so scores come out in the log2 domain for exp2.  Lane l
 //   keeps the quarter l mod 4 of q~ (32 values) and, for each group of 32
 //   tokens, reads the same quarter of 4 tokens' 64-byte code rows with
-//   coalesced 16-byte loads.  A score is s.(q~ . c) + z.sum(q~): the codes are
-//   never dequantized; a nibble becomes a float through PRMT into the
-//   exponent of 2^23 and one packed subtraction.  The four lanes of a token add
+//   16-byte shared-memory loads.  A score is s.(q~ . c) + z.sum(q~): the codes are
+//   never dequantized; a nibble's own bit pattern is read as an fp32
+//   subnormal and multiplied by an operand pre-scaled by 2^100 (one PRMT per
+//   nibble, no conversion arithmetic).  The four lanes of a token add
 //   their partial dots with two shuffles.  Online softmax per warp; the value
 //   side accumulates w.c with w = p.s_v in the same lane layout, plus sum p.z_v.
 //   The CTA merges its warps and writes (max, sum, o~[128]) per chunk.
@@ -31,7 +36,11 @@
 
 namespace rq {
 
-constexpr int kAttnChunk = 256;     // cached tokens per CTA
+constexpr int kAttnChunk = 1024;    // cached tokens per CTA
+constexpr int kAttnStageTok = 128;  // tokens per shared-memory stage (32 per warp)
+constexpr int kAttnStages = 3;
+constexpr int kAttnStageBytes = kAttnStageTok * 64 * 2;  // K codes | V codes
+constexpr size_t kAttnSmem = (size_t)kAttnStages * kAttnStageBytes + 2 * kAttnStages * 8;
 constexpr int kAttnPart = 132;      // floats per chunk record: max, sum, 128 values, pad
 
 struct AttnParams {
@@ -51,49 +60,51 @@ struct AttnParams {
   int out_bf16;
 };
 
-// 4 nibbles of a 16-bit group -> float2 pairs, via PRMT into the low byte of
-// 2^23's bit pattern and one packed subtraction of 2^23.
-__device__ __forceinline__ float2 nib_pair(uint32_t e, int k) {
-  // e holds one nibble per byte; byte k and byte k+1 -> (float, float)
-  const uint32_t magic = 0x4B000000u;
-  const uint32_t a = __byte_perm(e, magic, 0x7540 | k);          // [e.b_k, 0, 0, 0x4B]
-  const uint32_t b = __byte_perm(e, magic, 0x7540 | (k + 1));
-  return __fadd2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)),
-                    make_float2(-8388608.0f, -8388608.0f));
+// A code nibble n is turned into a float for free: its bit pattern n is the
+// fp32 subnormal n * 2^-149.  Multiplied by an operand pre-scaled by 2^100
+// (kNibScale) the product x * n * 2^-49 is a normal number, exact up to the
+// product's own rounding, and the sums are scaled back by 2^49 (kNibUnscale)
+// once.  (The kernels are built without flush-to-zero, so the subnormal inputs
+// are honoured; the pre-scaled operands stay far below the fp32 range.)
+constexpr float kNibScale = 1.2676506002282294e30f;   // 2^100
+constexpr float kNibUnscale = 562949953421312.0f;     // 2^49
+
+// The nibbles of one 32-bit word as subnormal floats, paired for packed math:
+// pair j = (element 2j, element 2j + 1) of the word (low nibble first).
+__device__ __forceinline__ void word_nibbles(uint32_t w, float2 (&f)[4]) {
+  const uint32_t ev = w & 0x0F0F0F0Fu;          // elements 0, 2, 4, 6
+  const uint32_t od = (w >> 4) & 0x0F0F0F0Fu;   // elements 1, 3, 5, 7
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    f[j] = make_float2(__uint_as_float(__byte_perm(ev, 0u, 0x4440 | j)),
+                       __uint_as_float(__byte_perm(od, 0u, 0x4440 | j)));
 }
 
-// acc (float2) += sum over the 32 nibbles of c (byte j: element 2j low, 2j+1
-// high) times x[0..31], as packed pairs (x[2i], x[2i+1]).
+// sum over the 32 nibbles of c (word i: elements 8i..8i+7) times x[0..31],
+// with x pre-scaled by 2^100; the result carries the 2^-49 factor.
 __device__ __forceinline__ float dot32_nibbles(const uint4 c, const float (&x)[32]) {
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // word i = elements 8i..8i+7; even ones in the low nibbles, odd in the high
-    const uint32_t ev = w[i] & 0x0F0F0F0Fu;         // elements 8i, 8i+2, 8i+4, 8i+6
-    const uint32_t od = (w[i] >> 4) & 0x0F0F0F0Fu;  // elements 8i+1, 8i+3, 8i+5, 8i+7
-    const uint32_t lo = __byte_perm(ev, od, 0x5140);  // bytes: e0 o0 e1 o1 -> elements 8i..8i+3
-    const uint32_t hi = __byte_perm(ev, od, 0x7362);  // elements 8i+4..8i+7
-    const float2 f0 = nib_pair(lo, 0), f1 = nib_pair(lo, 2), f2 = nib_pair(hi, 0), f3 = nib_pair(hi, 2);
-    acc0 = __ffma2_rn(f0, make_float2(x[8 * i], x[8 * i + 1]), acc0);
-    acc1 = __ffma2_rn(f1, make_float2(x[8 * i + 2], x[8 * i + 3]), acc1);
-    acc0 = __ffma2_rn(f2, make_float2(x[8 * i + 4], x[8 * i + 5]), acc0);
-    acc1 = __ffma2_rn(f3, make_float2(x[8 * i + 6], x[8 * i + 7]), acc1);
+    float2 f[4];
+    word_nibbles(w[i], f);
+    acc0 = __ffma2_rn(f[0], make_float2(x[8 * i], x[8 * i + 1]), acc0);
+    acc1 = __ffma2_rn(f[1], make_float2(x[8 * i + 2], x[8 * i + 3]), acc1);
+    acc0 = __ffma2_rn(f[2], make_float2(x[8 * i + 4], x[8 * i + 5]), acc0);
+    acc1 = __ffma2_rn(f[3], make_float2(x[8 * i + 6], x[8 * i + 7]), acc1);
   }
   return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
 
-// o[0..31] += w * (the 32 nibbles of c), packed.
+// o[0..31] += w * (the 32 nibbles of c), w pre-scaled by 2^100 (o carries 2^-49).
 __device__ __forceinline__ void axpy32_nibbles(const uint4 c, float wgt, float (&o)[32]) {
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
   const float2 ww = make_float2(wgt, wgt);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t ev = w[i] & 0x0F0F0F0Fu;
-    const uint32_t od = (w[i] >> 4) & 0x0F0F0F0Fu;
-    const uint32_t lo = __byte_perm(ev, od, 0x5140);
-    const uint32_t hi = __byte_perm(ev, od, 0x7362);
-    const float2 f[4] = {nib_pair(lo, 0), nib_pair(lo, 2), nib_pair(hi, 0), nib_pair(hi, 2)};
+    float2 f[4];
+    word_nibbles(w[i], f);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 t = __ffma2_rn(f[k], ww, make_float2(o[8 * i + 2 * k], o[8 * i + 2 * k + 1]));
@@ -103,7 +114,26 @@ __device__ __forceinline__ void axpy32_nibbles(const uint4 c, float wgt, float (
   }
 }
 
+// Bulk-copy the K and V code rows of stage-iteration n (tokens g0 + 128 n ...,
+// at most 128, clipped at S) into stage buffer `buf`; one elected thread.
+__device__ __forceinline__ void attn_issue(const AttnParams& p, int64_t row0, int64_t t, uint8_t* buf, uint64_t* bar) {
+  const int64_t cnt = min((int64_t)kAttnStageTok, p.S - t);
+  const unsigned bytes = (unsigned)(cnt * 64);
+  mbar_arrive_expect_tx(bar, 2 * bytes);
+  bulk_g2s(buf, p.kc + (row0 + t) * 64, bytes, bar);
+  bulk_g2s(buf + kAttnStageTok * 64, p.vc + (row0 + t) * 64, bytes, bar);
+}
+
+__device__ __forceinline__ float4 attn_scales(const AttnParams& p, int64_t row0, int64_t t) {
+  const int64_t tt = t < p.S ? t : p.S - 1;
+  return make_float4(__half2float(p.ks[row0 + tt]), __half2float(p.kz[row0 + tt]), __half2float(p.vs[row0 + tt]),
+                     __half2float(p.vz[row0 + tt]));
+}
+
 __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams p) {
+  extern __shared__ __align__(128) uint8_t attn_smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(attn_smem + kAttnStages * kAttnStageBytes);
+  uint64_t* empty = full + kAttnStages;  // one arrival per warp once it has read the stage
   __shared__ float qs[128];
   __shared__ float qsum_s;
   __shared__ float wm[4], wl[4];
@@ -112,6 +142,23 @@ __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams 
   const int64_t bh = blockIdx.x / p.nchunks;   // one CTA per (batch*head, chunk)
   const int chunk = (int)(blockIdx.x - bh * p.nchunks);
   const float kNegInf = -__int_as_float(0x7f800000);
+  const int64_t S = p.S;
+  const int64_t row0 = bh * S;
+  const int64_t g0 = (int64_t)chunk * kAttnChunk;
+  const int n_iter = (int)((min((int64_t)kAttnChunk, S - g0) + kAttnStageTok - 1) / kAttnStageTok);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kAttnStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)  // the cache starts streaming before q is rotated
+    for (int n = 0; n < kAttnStages && n < n_iter; ++n)
+      attn_issue(p, row0, g0 + (int64_t)kAttnStageTok * n, attn_smem + n * kAttnStageBytes, &full[n]);
+  float4 scl = attn_scales(p, row0, g0 + 32 * warp + lane);
 
   if (warp == 0) {
     // q~ = (q . diag(s) . H_128) * qscale; lane l holds elements 4l..4l+3
@@ -153,7 +200,7 @@ __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams 
   const int quarter = lane & 3;
   float qq[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) qq[j] = qs[32 * quarter + j];
+  for (int j = 0; j < 32; ++j) qq[j] = qs[32 * quarter + j] * kNibScale;
   const float qsum = qsum_s;
 
   float m = kNegInf, l = 0.f, zacc = 0.f;
@@ -161,63 +208,103 @@ __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams 
 #pragma unroll
   for (int j = 0; j < 32; ++j) o[j] = 0.f;
 
-  const int64_t S = p.S;
-  const int64_t row0 = bh * S;
+  bool timed_out = false;
+  int n_stop = 0;
 #pragma unroll 1
-  for (int g = 0; g < 2; ++g) {
-    const int64_t t0 = (int64_t)chunk * kAttnChunk + warp * 64 + 32 * g;
-    if (t0 >= S) break;
-    // scale / zero of the group's tokens, one per lane
-    const int64_t tl = t0 + lane < S ? t0 + lane : S - 1;
-    const float ksl = __half2float(p.ks[row0 + tl]), kzl = __half2float(p.kz[row0 + tl]);
-    const float vsl = __half2float(p.vs[row0 + tl]), vzl = __half2float(p.vz[row0 + tl]);
-    uint4 kq[4], vq[4];
-    int tok[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      tok[i] = 8 * i + (lane >> 2);  // token within the group
-      const int64_t t = t0 + tok[i] < S ? t0 + tok[i] : S - 1;
-      kq[i] = *reinterpret_cast<const uint4*>(p.kc + (row0 + t) * 64 + 16 * quarter);
-      vq[i] = *reinterpret_cast<const uint4*>(p.vc + (row0 + t) * 64 + 16 * quarter);
+  for (int n = 0; n < n_iter; ++n) {
+    const int st = n % kAttnStages;
+    // warps drift apart by up to a stage; a warp that gives up on a wait
+    // leaves the loop, the device error word records the timeout and the
+    // CTA's partial result is not to be used
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[st], (unsigned)((n / kAttnStages) & 1)))) {
+      timed_out = true;
+      n_stop = n;
+      break;
     }
-    float sc[4];
-    float gmax = kNegInf;
+    const float4 cur = scl;
+    if (n + 1 < n_iter) scl = attn_scales(p, row0, g0 + (int64_t)kAttnStageTok * (n + 1) + 32 * warp + lane);
+    const int64_t t0 = g0 + (int64_t)kAttnStageTok * n + 32 * warp;  // this warp's 32 tokens
+    if (t0 < S) {
+      const uint8_t* kb = attn_smem + st * kAttnStageBytes + 32 * warp * 64;
+      const uint8_t* vb = kb + kAttnStageTok * 64;
+      uint4 kq[4], vq[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float dsum = dot32_nibbles(kq[i], qq);
-      dsum += __shfl_xor_sync(0xFFFFFFFFu, dsum, 1);
-      dsum += __shfl_xor_sync(0xFFFFFFFFu, dsum, 2);
-      const float s_k = __shfl_sync(0xFFFFFFFFu, ksl, tok[i]);
-      const float z_k = __shfl_sync(0xFFFFFFFFu, kzl, tok[i]);
-      sc[i] = (t0 + tok[i] < S) ? fmaf(s_k, dsum, z_k * qsum) : kNegInf;
-      gmax = fmaxf(gmax, sc[i]);
+      for (int i = 0; i < 4; ++i) {
+        // lane l: quarter l mod 4 of token 8i + l/4 -- the 512 bytes at 512 i + 16 l
+        kq[i] = *reinterpret_cast<const uint4*>(kb + 512 * i + 16 * lane);
+        vq[i] = *reinterpret_cast<const uint4*>(vb + 512 * i + 16 * lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
+      float sc[4];
+      float gmax = kNegInf;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = 8 * i + (lane >> 2);
+        float dsum = dot32_nibbles(kq[i], qq);
+        dsum += __shfl_xor_sync(0xFFFFFFFFu, dsum, 1);
+        dsum += __shfl_xor_sync(0xFFFFFFFFu, dsum, 2);
+        dsum *= kNibUnscale;
+        const float s_k = __shfl_sync(0xFFFFFFFFu, cur.x, tok);
+        const float z_k = __shfl_sync(0xFFFFFFFFu, cur.y, tok);
+        sc[i] = (t0 + tok < S) ? fmaf(s_k, dsum, z_k * qsum) : kNegInf;
+        gmax = fmaxf(gmax, sc[i]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xFFFFFFFFu, gmax, off));
+      const float m_new = fmaxf(m, gmax);               // finite: token t0 is valid
+      const float corr = exp2f(m - m_new);              // 0 on the first group (m = -inf)
+      float psum = 0.f, zsum = 0.f;
+      float w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = 8 * i + (lane >> 2);
+        const float pi = exp2f(sc[i] - m_new);          // 0 for masked tokens
+        const float s_v = __shfl_sync(0xFFFFFFFFu, cur.z, tok);
+        const float z_v = __shfl_sync(0xFFFFFFFFu, cur.w, tok);
+        psum += pi;
+        zsum = fmaf(pi, z_v, zsum);
+        w[i] = pi * s_v * kNibScale;
+      }
+      // each token is held by the four lanes of its quarter group: count it once
+      psum = quarter == 0 ? psum : 0.f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xFFFFFFFFu, psum, off);
+      l = fmaf(l, corr, psum);
+      zacc = fmaf(zacc, corr, zsum);
+      m = m_new;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) o[j] *= corr;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) axpy32_nibbles(vq[i], w[i], o);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xFFFFFFFFu, gmax, off));
-    const float m_new = fmaxf(m, gmax);               // finite: the group has a valid token
-    const float corr = exp2f(m - m_new);              // 0 on the first group (m = -inf)
-    float psum = 0.f, zsum = 0.f;
-    float w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float pi = exp2f(sc[i] - m_new);          // 0 for masked tokens
-      const float s_v = __shfl_sync(0xFFFFFFFFu, vsl, tok[i]);
-      const float z_v = __shfl_sync(0xFFFFFFFFu, vzl, tok[i]);
-      psum += pi;
-      zsum = fmaf(pi, z_v, zsum);
-      w[i] = pi * s_v;
+    else if (lane == 0) {
+      mbar_arrive(&empty[st]);  // no tokens of this warp in the stage
     }
-    // each token is held by the four lanes of its quarter group: count it once
-    psum = quarter == 0 ? psum : 0.f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xFFFFFFFFu, psum, off);
-    l = fmaf(l, corr, psum);
-    zacc = fmaf(zacc, corr, zsum);
-    m = m_new;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) o[j] *= corr;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) axpy32_nibbles(vq[i], w[i], o);
+    if (warp == 0 && n + kAttnStages < n_iter) {
+      // lane 0 refills stage st once every warp has read it; the warp leaves
+      // the loop together if that wait gives up
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait_bounded(&empty[st], (unsigned)((n / kAttnStages) & 1));
+        if (ok) {
+          fence_proxy_async_smem();
+          attn_issue(p, row0, g0 + (int64_t)kAttnStageTok * (n + kAttnStages), attn_smem + st * kAttnStageBytes,
+                     &full[st]);
+        }
+      }
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+        timed_out = true;
+        n_stop = n;
+        break;
+      }
+    }
+  }
+  if (timed_out && threadIdx.x == 0) {
+    // stages n_stop+1 .. n_stop+kAttnStages-1 may still be in flight: let
+    // them land before the CTA finishes (stage n_stop landed or gave up)
+    for (int j = n_stop + 1; j < n_stop + kAttnStages && j < n_iter; ++j)
+      (void)mbar_wait_bounded(&full[j % kAttnStages], (unsigned)((j / kAttnStages) & 1));
   }
   // merge the lanes of the same quarter (lane bits 2..4) and the z terms
 #pragma unroll
@@ -225,6 +312,8 @@ __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams 
 #pragma unroll
     for (int j = 0; j < 32; ++j) o[j] += __shfl_xor_sync(0xFFFFFFFFu, o[j], off);
   }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) o[j] *= kNibUnscale;
   float zs = quarter == 0 ? zacc : 0.f;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) zs += __shfl_xor_sync(0xFFFFFFFFu, zs, off);

@@ -39,6 +39,8 @@ WORKLOADS = {
     "q_proj_nvfp4": dict(index=4, M=2048, K=4096, N=4096, block=128, fmt="nvfp4"),
     "kv4": dict(index=5, B=16, H=32, S=4096, D=128),
     "q_proj_mxfp4": dict(index=6, M=2048, K=4096, N=4096, block=128, fmt="mxfp4"),
+    # a decode step over the kv4 workload's cache (written once by the KV4 kernel)
+    "kv4_decode": dict(index=7, B=16, H=32, S=4096, D=128),
 }
 
 
@@ -56,7 +58,7 @@ def signs(k, seed, device="cpu"):
 
 def workload_signs(name, device="cpu"):
     w = WORKLOADS[name]
-    k = w["D"] if name == "kv4" else w["K"]
+    k = w["D"] if "D" in w else w["K"]
     return signs(k, 2000 + w["index"], device)
 
 
