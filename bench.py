@@ -66,6 +66,7 @@ def load_peaks():
 # vectors processed.
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
+ATTN_SOURCES = ("rq_common.cuh", "rq_attn.cuh")
 _ROT, _GEM = "96ccf4968826d44e", "c6e805e14224d165"
 TRAFFIC = {
     ("hadamard_quant", "q_proj_int4"): (16847104, _ROT),
@@ -93,7 +94,10 @@ def traffic(kind, workload):
     entry = TRAFFIC.get((kind, workload))
     if entry is None:
         return None
-    files = ROTATE_SOURCES if kind == "hadamard_quant" else GEMM_SOURCES
+    if workload == "kv4_decode":
+        files = ATTN_SOURCES
+    else:
+        files = ROTATE_SOURCES if kind == "hadamard_quant" else GEMM_SOURCES
     return entry[0] if source_fingerprint(files) == entry[1] else None
 
 
@@ -285,21 +289,25 @@ def oracle_sample(name, rows):
     from oracle import gemm as ogemm, hadamard as ohad, quant as oquant
     c = syn.WORKLOADS[name]
     if name == "kv4_decode":
-        # rows = heads of one batch entry over the full sequence length
+        # rows = (batch entry, head) pairs over the full sequence length: the
+        # cache of one batch entry is built once and attended rows / H times
         from oracle import attention as oattn
         s = syn.workload_signs(name).numpy()
-        k = syn.kv(batch=1, heads=rows, which=0).to(torch.float64).numpy()
-        v = syn.kv(batch=1, heads=rows, which=1).to(torch.float64).numpy()
+        heads = min(rows, c["H"])
+        reps = max(1, rows // heads)
+        k = syn.kv(batch=1, heads=heads, which=0).to(torch.float64).numpy()
+        v = syn.kv(batch=1, heads=heads, which=1).to(torch.float64).numpy()
         caches = []
         for x in (k, v):
             q4, sh, zh, _, _ = oquant.kv4_vectors(oattn.rotate_heads(x, s).reshape(-1, 128))
             caches += [q4.reshape(x.shape), sh.reshape(x.shape[:-1]), zh.reshape(x.shape[:-1])]
-        qv = np.random.default_rng(0).standard_normal((1, rows, 128))
+        qv = np.random.default_rng(0).standard_normal((1, heads, 128))
         t0 = time.perf_counter()
-        oattn.kv4_decode_attention(qv, *caches, s)
+        for _ in range(reps):
+            oattn.kv4_decode_attention(qv, *caches, s)
         dt = time.perf_counter() - t0
-        nbytes = rows * c["S"] * 2 * (64 + 4)
-        return nbytes / dt / 1e9, None, dt, "1 x %d heads x %d tokens of the cache" % (rows, c["S"])
+        nbytes = reps * heads * c["S"] * 2 * (64 + 4)
+        return nbytes / dt / 1e9, None, dt, "%d x %d heads x %d tokens of the cache" % (reps, heads, c["S"])
     if name == "kv4":
         kv = syn.kv(batch=1, heads=4, seq=rows)
         s = syn.workload_signs(name).numpy()
@@ -361,7 +369,7 @@ def blas_threads():
 
 def sample_rows(name):
     return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096,
-            "q_proj_mxfp4": 256, "kv4_decode": 32}[name]
+            "q_proj_mxfp4": 256, "kv4_decode": 1024}[name]
 
 
 # --------------------------------------------------------------------------- main
