@@ -14,6 +14,11 @@ Sources on the pages:
 * MXFP4 -- E2M1 values whose scales are powers of two shared by 32 values:
   same article, section "The full model in NVFP4, on vLLM" (the FP4 study it
   cites) and section "When to rotate".
+* 6- and 8-bit symmetric round to nearest (W8A8, W6A6) and W4A8:
+  "QuaRot (rotation-based outlier removal, W4A4KV4)", field "Bits" (lossless
+  6-bit and 8-bit round-to-nearest, no calibration data) and "SpinQuant
+  (learned rotations + W4A4KV4)", field "Activation scheme" (also reported
+  at W4A8).
 * KV cache at 4 bits, asymmetric: "SpinQuant (learned rotations + W4A4KV4)",
   field "Activation scheme" (per-group INT4 asymmetric for the KV cache), and
   "QuaRot (rotation-based outlier removal, W4A4KV4)", field "Activation scheme"
@@ -23,6 +28,10 @@ Readings where the pages are silent (each also listed in the design notes):
 
 * INT4: s = fp32(fp32(amax)/7); q = clamp(rint(x/s), -8, 7) with rint
   half-to-even; so -8 is never produced.  amax = 0 -> s = 0, q = 0.
+* INT6 / INT8: the INT4 rule with qmax = 2^(b-1) - 1 = 31 / 127 in place
+  of 7: s = fp32(fp32(amax)/qmax), q = clamp(rint(x/s), -qmax-1, qmax), one
+  scale per token (activations) or output channel (weights); the codes are
+  stored one per byte (two's complement).
 * NVFP4: g = fp32(fp32(amax(X~)) / (6*448)) over the whole rotated tensor
   (dynamic) or given by the caller (static).  Per block b of 16 along K:
   S_b = E4M3_rn_satfinite(amax_b / (6 g)); e = E2M1_rn_satfinite(x / (S_b g));
@@ -84,6 +93,26 @@ def int4_sym_rows(xr):
     with np.errstate(divide="ignore", invalid="ignore"):
         v = np.where(s64 > 0, xr / np.where(s64 > 0, s64, 1.0), 0.0)
     q = np.clip(np.rint(v), -8, INT4_QMAX).astype(np.int64)
+    tie = _near_half(v) & (s64 > 0)
+    return q, scale, tie
+
+
+def int_sym_rows(xr, bits):
+    """Per-row symmetric round-to-nearest with b-bit signed codes, b in 4..8.
+
+    qmax = 2^(b-1) - 1.  xr: fp64 [rows, K].  Returns (q int64 [rows, K] in
+    [-qmax-1, qmax], scale fp32 [rows], tie bool [rows, K]).
+    """
+    if not 4 <= bits <= 8:
+        raise ValueError("bits must be in 4..8")
+    qmax = 2 ** (bits - 1) - 1
+    xr = np.asarray(xr, dtype=np.float64)
+    amax = np.abs(xr).max(axis=1).astype(np.float32)
+    scale = amax / np.float32(qmax)                          # fp32 / fp32, correctly rounded
+    s64 = scale.astype(np.float64)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s64 > 0, xr / np.where(s64 > 0, s64, 1.0), 0.0)
+    q = np.clip(np.rint(v), -qmax - 1, qmax).astype(np.int64)
     tie = _near_half(v) & (s64 > 0)
     return q, scale, tie
 

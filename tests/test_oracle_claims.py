@@ -13,6 +13,10 @@ stand-ins (CPU only).
   section "When to rotate": rotations help MXFP4, whose scales are powers of
   two shared by 32 values.
 
+"QuaRot (rotation-based outlier removal, W4A4KV4)", field "Bits": 6- and
+8-bit round to nearest are lossless after rotation; "SpinQuant (learned
+rotations + W4A4KV4)": W4A8 narrows the gap that W4A4 leaves.
+
 The exact figures came from real Qwen3-8B layers and are not reproducible here
 (parity unpinned); the tests check the direction and a margin.
 """
@@ -101,3 +105,28 @@ def test_rotation_helps_mxfp4(which, request):
     y = x @ w.T
     m0, m1 = _mx_err(y, x, w), _mx_err(y, xr, wr)
     assert m1 < 0.95 * m0
+
+
+def _int_err(y, a, b, bx, bw):
+    qa, sa, _ = quant.int_sym_rows(a, bx)
+    qb, sb, _ = quant.int_sym_rows(b, bw)
+    return metrics.rel_product_error(y, gemm.int4_y(gemm.int_acc(qa, qb), sa, sb))
+
+
+@pytest.mark.parametrize("case", ["qproj", "downproj"])
+def test_more_bits_after_rotation(case, request):
+    """After rotation: W8A8 < W6A6 < W4A8 < W4A4 in product error; the rotation
+    cuts the 6- and 8-bit errors by more than 4x, leaving W8A8 near 1-2% and
+    W6A6 under 10% on these outlier-heavy stand-ins (their max/median ratios
+    exceed the article's layers'); W4A8 clearly better than W4A4."""
+    x, w, s, xr, wr = request.getfixturevalue(case)
+    y = x @ w.T
+    e44 = _int_err(y, xr, wr, 4, 4)
+    e48 = _int_err(y, xr, wr, 8, 4)
+    e66 = _int_err(y, xr, wr, 6, 6)
+    e88 = _int_err(y, xr, wr, 8, 8)
+    assert e88 < e66 < e48 < e44
+    assert e88 < 0.025 and e66 < 0.1
+    assert e48 < 0.8 * e44
+    assert _int_err(y, x, w, 8, 8) > 4 * e88
+    assert _int_err(y, x, w, 6, 6) > 4 * e66

@@ -1,6 +1,7 @@
 """Pins for the oracle's W4A4 product (CPU only): triple loops on tiny inputs."""
 
 import numpy as np
+import pytest
 
 from oracle import formats, gemm, quant
 
@@ -81,3 +82,21 @@ def test_mxfp4_y_matches_blockwise_sum():
                             for t in range(32 * b, 32 * b + 32))
                 tot += math.ldexp(inner, int(sx[i, b]) - 127 + int(sw[j, b]) - 127)
             assert y[i, j] == tot
+
+
+@pytest.mark.parametrize("bx,bw", [(8, 4), (8, 8), (6, 6)])
+def test_int_acc_matches_triple_loop(bx, bw):
+    rng = np.random.default_rng(bx * 10 + bw)
+    m, n, k = 4, 5, 48
+    qx = rng.integers(-(2 ** (bx - 1)), 2 ** (bx - 1), size=(m, k))
+    qw = rng.integers(-(2 ** (bw - 1)), 2 ** (bw - 1), size=(n, k))
+    acc = gemm.int_acc(qx, qw)
+    for i in range(m):
+        for j in range(n):
+            assert acc[i, j] == sum(int(qx[i, t]) * int(qw[j, t]) for t in range(k))
+
+
+def test_int_acc_extreme_8bit_fits_int32():
+    k = 65536
+    acc = gemm.int_acc(np.full((1, k), -128), np.full((1, k), -128))
+    assert acc[0, 0] == 16384 * k and acc[0, 0] < 2 ** 31

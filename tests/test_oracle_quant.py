@@ -221,3 +221,77 @@ def test_mxfp4_power_of_two_amax_is_a_scale_tie():
     assert s[0, 0] == 127 and tie_s[0, 0]
     _, _, _, tie_s = quant.mxfp4_rows(_mx_block([5.0, 1.0]))
     assert not tie_s[0, 0]
+
+
+# ---------------------------------------------------------------- 6- and 8-bit RTN
+def _int_bruteforce(x, s, bits):
+    qmax = 2 ** (bits - 1) - 1
+    codes = np.arange(-qmax - 1, qmax + 1)
+    d = np.abs(x[..., None] - codes * s)
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    even = (codes % 2) == 0
+    pick = np.where((cand & even).any(axis=-1), np.argmax(cand & even, axis=-1), np.argmax(cand, axis=-1))
+    return codes[pick]
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_int_sym_bruteforce_and_bound(bits):
+    """Each code is the nearest of all 2^b codes to x / s (argmin search, half to even)."""
+    qmax = 2 ** (bits - 1) - 1
+    rng = np.random.default_rng(40 + bits)
+    x = rng.standard_normal((24, 128))
+    x[:, 5] *= 30
+    q, s, tie = quant.int_sym_rows(x, bits)
+    assert q.min() >= -qmax and q.max() <= qmax   # -qmax-1 never produced (s = amax / qmax)
+    for r in range(x.shape[0]):
+        bf = _int_bruteforce(x[r], float(s[r]), bits)
+        assert ((bf == q[r]) | tie[r]).all()
+    err = np.abs(x - quant.int4_dequant(q, s))
+    assert np.all(err <= s.astype(np.float64)[:, None] * (0.5 + 1e-6))
+    arg = np.abs(x).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(24), arg]) == qmax)
+
+
+def test_int8_and_int6_hand_worked_row():
+    """x = [2.54, -1, 0.5, 0.071]: s = 2.54/127 = 0.02 -> codes 127, -50, 25, 3.55 -> 4;
+    s = 2.54/31 = 0.08193548 -> 31, -12.20 -> -12, 6.10 -> 6, 0.867 -> 1."""
+    x = np.array([[2.54, -1.0, 0.5, 0.071]])
+    q8, s8, _ = quant.int_sym_rows(x, 8)
+    assert s8[0] == np.float32(np.float32(2.54) / np.float32(127.0))
+    assert list(q8[0]) == [127, -50, 25, 4]
+    q6, s6, _ = quant.int_sym_rows(x, 6)
+    assert s6[0] == np.float32(np.float32(2.54) / np.float32(31.0))
+    assert list(q6[0]) == [31, -12, 6, 1]
+
+
+def test_int_sym_zero_row_and_half_even():
+    q, s, tie = quant.int_sym_rows(np.zeros((2, 8)), 8)
+    assert np.all(q == 0) and np.all(s == 0) and not tie.any()
+    # scale 1 (amax = 127): k + 0.5 rounds to the even neighbour
+    x = np.array([[127.0, 0.5, 1.5, 2.5, -0.5, -1.5, -126.5, 3.5]])
+    q, s, tie = quant.int_sym_rows(x, 8)
+    assert s[0] == 1.0
+    assert list(q[0]) == [127, 0, 2, 2, 0, -2, -126, 4]
+    assert list(tie[0]) == [False] + [True] * 7
+
+
+def test_int_sym_at_4_bits_is_the_int4_rule():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((8, 64))
+    a = quant.int_sym_rows(x, 4)
+    b = quant.int4_sym_rows(x)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+def test_more_bits_lower_error():
+    """Round to nearest with b bits: the worst error is s/2 = amax / (2 (2^(b-1) - 1)),
+    so each extra bit roughly halves it."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((32, 256))
+    errs = []
+    for bits in (4, 6, 8):
+        q, s, _ = quant.int_sym_rows(x, bits)
+        errs.append(np.linalg.norm(x - quant.int4_dequant(q, s)) / np.linalg.norm(x))
+    assert errs[0] > 3.5 * errs[1] > 3.5 * 3.5 * errs[2]
