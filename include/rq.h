@@ -63,13 +63,15 @@ typedef enum {
 typedef enum {
   RQ_INT4 = 0,  /* symmetric INT4, one fp32 scale per row */
   RQ_NVFP4 = 1, /* E2M1, one E4M3 scale per 16 values, fp32 per-tensor scale */
-  RQ_MXFP4 = 2  /* E2M1, one E8M0 (power-of-two) scale per 32 values */
+  RQ_MXFP4 = 2, /* E2M1, one E8M0 (power-of-two) scale per 32 values */
+  RQ_INT8 = 3,  /* symmetric 8-bit, one int8 code per byte, one fp32 scale per row */
+  RQ_INT6 = 4   /* symmetric 6-bit (codes in [-31, 31]), one int8 byte each, one fp32 scale per row */
 } rq_format;
 
 typedef enum {
   RQ_OUT_F32 = 0,     /* Y as fp32 */
   RQ_OUT_BF16 = 1,    /* Y as bf16 (round to nearest even) */
-  RQ_OUT_I32_ACC = 2  /* INT4 only: the raw int32 accumulators sum_k qx*qw, no scales */
+  RQ_OUT_I32_ACC = 2  /* integer formats only: the raw int32 accumulators sum_k qx*qw, no scales */
 } rq_out;
 
 typedef enum {
@@ -86,7 +88,7 @@ RQ_API rq_status rq_init(int device);
 RQ_API const char* rq_status_string(rq_status status);
 
 /* Bytes of device workspace rq_rotate_quantize / rq_prepare_weights need:
- * 16 for NVFP4 (the dynamic-scale max word), 0 for INT4 and MXFP4.  The workspace must
+ * 16 for NVFP4 (the dynamic-scale max word), 0 for the other formats.  The workspace must
  * be 16-byte aligned; its contents need not be initialised. */
 RQ_API size_t rq_workspace_bytes(rq_format fmt);
 
@@ -103,7 +105,7 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *  signs_dev  int8 [K], 16-byte aligned, each +1 or -1 (the random sign diagonal;
  *             any other value is read as -1 if negative and +1 otherwise).
  *  block      128 for 128-wide blocks, or 0 for a full-width rotation (then K
- *             must be a power of two in [256, 4096]; INT4 only).
+ *             must be a power of two in [256, 4096]; INT4, INT6 and INT8 only).
  *  fmt        RQ_INT4:
  *               codes_dev  uint8 [M, K/2], scales_dev float [M]:
  *               s = amax/7 (fp32, amax = max |x~| of the row); q = rint(x~/s).
@@ -123,6 +125,12 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *               rule; the pages name only powers of two); e = E2M1_rn_satfinite(x~ / 2^e_b).
  *               amax_b = 0 gives scale code 0 and e = 0.  gscale_dev and
  *               workspace_dev are unused (may be NULL).
+ *             RQ_INT8 / RQ_INT6 (6- and 8-bit round to nearest: "QuaRot", field
+ *             "Bits"; the 8-bit activations of W4A8: "SpinQuant", field
+ *             "Activation scheme"):
+ *               codes_dev  int8 [M, K], scales_dev float [M]:
+ *               s = amax/qmax with qmax = 127 / 31; q = rint(x~/s).  gscale_dev
+ *               and workspace_dev are unused (may be NULL).
  *  workspace_dev  rq_workspace_bytes(fmt) bytes (may be NULL when that is 0).
  *  codes_dev and scales_dev 16-byte aligned (8 for NVFP4 scales).
  * Values that sit within a few fp32 ulps of a rounding boundary may round
@@ -166,6 +174,26 @@ RQ_API rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev
                        const uint8_t* wcodes_dev, const void* wscales_dev, const float* wgscale_dev, int64_t M,
                        int64_t N, int64_t K, rq_format fmt, void* Y_dev, int64_t ldy, rq_out out,
                        rq_stream_t stream);
+
+/*
+ * rq_int_gemm: Y[M, N] = deq(X codes) . deq(W codes)^T for integer codes of
+ * different widths on the two sides: W4A8 ("SpinQuant", field "Activation
+ * scheme"), W8A8 and W6A6 ("QuaRot", field "Bits"), and W4A4.
+ *  xfmt  RQ_INT4 (xcodes uint8 [M, K/2], packed nibbles), RQ_INT6 or RQ_INT8
+ *        (xcodes int8 [M, K]); xscales float [M].
+ *  wfmt  the same for W [N, K]; wscales float [N].
+ *  Supported pairs (xfmt, wfmt): (INT4, INT4) -- the rq_w4a4_gemm INT4 path --
+ *  (INT6/INT8, INT4) and (INT6/INT8, INT6/INT8).  (INT4, INT6/INT8) returns
+ *  RQ_ERR_UNSUPPORTED_SHAPE.
+ *  acc = sum_k qx[m,k] qw[n,k] exactly in int32 (|acc| < 2^31 for K <= 65536);
+ *  Y = float(acc) * sx[m] * sw[n] (float(acc) rounds to nearest above 2^24).
+ *  Codes 16-byte aligned, xscales 4-byte and wscales 16-byte aligned; K a
+ *  multiple of 128, at most 65536; M, N >= 0; Y_dev, ldy and `out` as for
+ *  rq_w4a4_gemm (RQ_OUT_I32_ACC gives the raw accumulators).
+ */
+RQ_API rq_status rq_int_gemm(const uint8_t* xcodes_dev, const float* xscales_dev, rq_format xfmt,
+                             const uint8_t* wcodes_dev, const float* wscales_dev, rq_format wfmt, int64_t M,
+                             int64_t N, int64_t K, void* Y_dev, int64_t ldy, rq_out out, rq_stream_t stream);
 
 /*
  * rq_kv_rotate_quantize: 4-bit KV cache entries ("QuaRot", "Activation

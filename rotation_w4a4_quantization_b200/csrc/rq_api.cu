@@ -202,9 +202,11 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
                                void* workspace, cudaStream_t st) {
   rq_status s = check_rotation_args(X, M, K, ldx, signs, block);
   if (s != RQ_OK) return s;
-  if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4) return RQ_ERR_INVALID_ARG;
+  if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4 && fmt != RQ_INT8 && fmt != RQ_INT6)
+    return RQ_ERR_INVALID_ARG;
   if (gmode != RQ_SCALE_DYNAMIC && gmode != RQ_SCALE_STATIC) return RQ_ERR_INVALID_ARG;
-  if (fmt != RQ_INT4 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  const bool int_fmt = fmt == RQ_INT4 || fmt == RQ_INT8 || fmt == RQ_INT6;
+  if (!int_fmt && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return RQ_OK;
   if (!codes || !scales) return RQ_ERR_INVALID_ARG;
   if (!aligned(codes, 16)) return RQ_ERR_ALIGNMENT;
@@ -224,6 +226,12 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
     p.scales_f32 = static_cast<float*>(scales);
     if (block == 0) return launch_full<kModeInt4>(p, st);
     return launch_block<kModeInt4>(p, st);
+  }
+  if (fmt == RQ_INT8 || fmt == RQ_INT6) {
+    p.scales_f32 = static_cast<float*>(scales);
+    p.qmax = fmt == RQ_INT8 ? 127.0f : 31.0f;
+    if (block == 0) return launch_full<kModeInt8>(p, st);
+    return launch_block<kModeInt8>(p, st);
   }
   if (fmt == RQ_MXFP4) {
     p.scales_e4m3 = static_cast<uint8_t*>(scales);
@@ -398,6 +406,13 @@ rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev, const
                        rq_stream_t stream) {
   return rq::gemm_dispatch(xcodes_dev, xscales_dev, xgscale_dev, wcodes_dev, wscales_dev, wgscale_dev, M, N, K, fmt,
                            Y_dev, ldy, out, static_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_int_gemm(const uint8_t* xcodes_dev, const float* xscales_dev, rq_format xfmt, const uint8_t* wcodes_dev,
+                      const float* wscales_dev, rq_format wfmt, int64_t M, int64_t N, int64_t K, void* Y_dev,
+                      int64_t ldy, rq_out out, rq_stream_t stream) {
+  return rq::int_gemm_dispatch(xcodes_dev, xscales_dev, xfmt, wcodes_dev, wscales_dev, wfmt, M, N, K, Y_dev, ldy, out,
+                               static_cast<cudaStream_t>(stream));
 }
 
 rq_status rq_get_device_error(rq_stream_t stream) {

@@ -60,6 +60,7 @@ struct GemmParams {
   int vec_ok;           // 1: Y rows allow 16-byte vector stores
   int tma_store;        // 1: bf16 Y is written by TMA from a shared-memory staging tile
   int tiles_m, tiles_n, num_tiles;
+  int acc_shift;        // integer accumulators hold 2^acc_shift * sum qx qw (8: W4A4, 4: A8 x W4, 0: A8 x W8)
 };
 
 // Bounded wait used by every role; on timeout the role stops issuing work.
@@ -73,7 +74,7 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, unsigned parity, int
 }
 
 // Epilogue for one 32-row x 256-column slab held by this warp's TMEM lanes.
-// acc_kind 0: int32 accumulators of 256*sum (INT4), 1: fp32 (NVFP4).
+// acc_kind 0: int32 accumulators of 2^p.acc_shift * sum (integer codes), 1: fp32 (FP4).
 // Arrives on `acc_empty` once the slab has been read out of tensor memory.
 template <int ACC_KIND>
 __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tacc, int m0, int n0, int q, int lane,
@@ -91,24 +92,24 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, uint32_t tac
     const int c0 = n0 + 32 * cc;
     if (!row_ok || c0 >= p.N) continue;
     const bool full = (c0 + 32 <= p.N) && p.vec_ok;
-    if (p.out == 2) {  // raw int32 accumulators (INT4 only)
+    if (p.out == 2) {  // raw int32 accumulators (integer codes only)
       int32_t* dst = reinterpret_cast<int32_t*>(p.y) + (int64_t)row * p.ldy + c0;
       if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<int4*>(dst + j) = make_int4((int)r[j] >> 8, (int)r[j + 1] >> 8, (int)r[j + 2] >> 8,
-                                                        (int)r[j + 3] >> 8);
+          *reinterpret_cast<int4*>(dst + j) = make_int4((int)r[j] >> p.acc_shift, (int)r[j + 1] >> p.acc_shift,
+                                                        (int)r[j + 2] >> p.acc_shift, (int)r[j + 3] >> p.acc_shift);
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (c0 + j < p.N) dst[j] = (int)r[j] >> 8;
+          if (c0 + j < p.N) dst[j] = (int)r[j] >> p.acc_shift;
       }
       continue;
     }
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const float a = (ACC_KIND == 0) ? (float)((int)r[j] >> 8) : __uint_as_float(r[j]);
+      const float a = (ACC_KIND == 0) ? (float)((int)r[j] >> p.acc_shift) : __uint_as_float(r[j]);
       v[j] = a * rowscale;
     }
     if (ACC_KIND == 0) {
@@ -809,26 +810,45 @@ done:
 // and stores bf16 through shared memory with TMA.
 //
 // Warps: 0 TMA producer, 1 MMA issuer (even CTA), 2..9 B converters,
-// 10..13 A converters, 14..17 epilogue.
+// 10..13 A converters, 14..21 epilogue.
+//
+// The same kernel serves 8-bit activation codes (A8: W4A8, W6A6, W8A8; the
+// 6-bit codes are int8 bytes in [-31, 31]): the A rows are staged as int8
+// (128B-swizzled) and the A warps copy them into TMEM unchanged.  With 8-bit
+// weight codes (W8) the B tiles need no widening: TMA writes them straight
+// into the 128B-swizzled operand ring, signalling the even CTA's barrier
+// (cta_group::2 copies), and the B converter warps sit idle.  acc holds
+// 2^shift * sum qx qw with shift = 8 (W4A4: both sides widened as 16 q),
+// 4 (A8 x W4) or 0 (A8 x W8).
 // ---------------------------------------------------------------------------
-constexpr int kI3Stg = 6, kI3Ops = 4;
+constexpr int kI3Ops = 4;
 constexpr int kI3BWarps = 8;
 constexpr int kI3AWarp0 = 2 + kI3BWarps;      // 10
 constexpr int kI3EpiWarp0 = kI3AWarp0 + 4;    // 14
 constexpr int kI3EpiWarps = 8;                // two per TMEM lane quadrant, 128 columns each
 constexpr int kI3Threads = 32 * (kI3EpiWarp0 + kI3EpiWarps);
-constexpr int kI3StgA = 128 * 64, kI3StgB = 128 * 64, kI3OpB = 128 * 128;
+constexpr int kI3OpB = 128 * 128;
 constexpr uint32_t kI3ACol0 = 256;
-constexpr size_t kI3Smem =
-    1024 + (size_t)kI3Ops * kI3OpB + (size_t)kI3Stg * (kI3StgA + kI3StgB) + 2 * kEpiStage + 256;
+template <bool A8, bool W8>
+struct I3 {
+  static constexpr int StgA = A8 ? 128 * 128 : 128 * 64;  // A tile per k-tile: int8 or packed nibbles
+  static constexpr int StgB = W8 ? 0 : 128 * 64;          // packed W (W8: straight into the operand ring)
+  static constexpr int Stg = (A8 && !W8) ? 4 : 6;         // staging depth within 227 KB
+  static constexpr int BArr = W8 ? 0 : kI3BWarps;         // B converter arrivals per k-tile and CTA
+  static constexpr int Shift = A8 ? (W8 ? 0 : 4) : 8;
+  static constexpr size_t Smem = 1024 + (size_t)kI3Ops * kI3OpB + (size_t)Stg * (StgA + StgB) + 2 * kEpiStage + 256;
+};
+constexpr size_t kI3Smem = I3<false, false>::Smem;
 
-// INT4 bf16 epilogue through shared memory for one 128-column half `ch` of the
-// CTA's 128 x 256 accumulator, by the four warps (one per lane quadrant) that
-// own that half: y = (acc >> 8) * sx[row] * sw[col], the arithmetic of
-// epilogue_store.  acc >> 8 (|.| < 2^22 for K <= 65536) becomes a float
-// exactly through the 1.5 * 2^23 magic number.  `stage` is this half's 32 KB
+// Integer bf16 epilogue through shared memory for one 128-column half `ch` of
+// the CTA's 128 x 256 accumulator, by the four warps (one per lane quadrant)
+// that own that half: y = (acc >> SHIFT) * sx[row] * sw[col], the arithmetic
+// of epilogue_store.  For W4A4 acc >> 8 (|.| < 2^22 for K <= 65536) becomes a
+// float exactly through the 1.5 * 2^23 magic number; wider codes convert with
+// cvt (exact below 2^24, rounded to nearest above).  `stage` is this half's 32 KB
 // of staging (two 128B-swizzled 64-column boxes); one thread stores it with
 // TMA (which clips rows >= M and columns >= N).  Named barrier 1 + ch.
+template <int SHIFT>
 __device__ __forceinline__ void epilogue_int4_bf16_tma(const GemmParams& p, const CUtensorMap* ytmap, uint32_t tacc,
                                                        int m0, int n0, int q, int ch, int lane, float sx,
                                                        const float* ws, uint8_t* stage,
@@ -870,8 +890,14 @@ __device__ __forceinline__ void epilogue_int4_bf16_tma(const GemmParams& p, cons
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = 8 * k + 2 * e;
-        const float i0 = __int_as_float(((int)r[j] >> 8) + 0x4B400000) - kRoundMagic;
-        const float i1 = __int_as_float(((int)r[j + 1] >> 8) + 0x4B400000) - kRoundMagic;
+        float i0, i1;
+        if (SHIFT == 8) {
+          i0 = __int_as_float(((int)r[j] >> 8) + 0x4B400000) - kRoundMagic;
+          i1 = __int_as_float(((int)r[j + 1] >> 8) + 0x4B400000) - kRoundMagic;
+        } else {
+          i0 = __int2float_rn((int)r[j] >> SHIFT);
+          i1 = __int2float_rn((int)r[j + 1] >> SHIFT);
+        }
         __nv_bfloat162 b = __floats2bfloat162_rn(i0 * sx * sw[j], i1 * sx * sw[j + 1]);
         w[e] = *reinterpret_cast<uint32_t*>(&b);
       }
@@ -888,13 +914,16 @@ __device__ __forceinline__ void epilogue_int4_bf16_tma(const GemmParams& p, cons
   }
 }
 
+template <bool A8, bool W8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
-    gemm_int4_2sm_ts_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                            const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_int_2sm_ts_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  using C = I3<A8, W8>;
+  constexpr int kI3Stg = C::Stg, kI3StgA = C::StgA, kI3StgB = C::StgB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* opb = base;                                         // [kI3Ops][B 16K], 128B-swizzled int8
-  uint8_t* stg = opb + (size_t)kI3Ops * kI3OpB;                // [kI3Stg][A 8K | B 8K], 64B-swizzled nibbles
+  uint8_t* stg = opb + (size_t)kI3Ops * kI3OpB;                // [kI3Stg][A | B]: nibbles 64B-swizzled, int8 128B-swizzled
   uint8_t* epi = stg + (size_t)kI3Stg * (kI3StgA + kI3StgB);   // bf16 output staging, one 32 KB half per column half
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi + 2 * kEpiStage);
   uint64_t* stg_full = bars;
@@ -915,10 +944,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kI3Stg; ++i) {
       mbar_init(&stg_full[i], 1);
-      mbar_init(&stg_empty[i], kI3BWarps + 4);
+      mbar_init(&stg_empty[i], C::BArr + 4);
     }
     for (int i = 0; i < kI3Ops; ++i) {
-      mbar_init(&op_full[i], 2 * (kI3BWarps + 4));
+      // A warps of both CTAs, B converters of both CTAs or (W8) the even
+      // CTA's producer with the transaction bytes of both B copies
+      mbar_init(&op_full[i], 2 * (C::BArr + 4) + (W8 ? 1 : 0));
       mbar_init(&op_empty[i], 1);
     }
     mbar_init(&acc_full[0], 1);
@@ -941,8 +972,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int s = 0;
-      unsigned ph = 0;
+      int s = 0, o = 0;
+      unsigned ph = 0, oph = 0;
       for (int tile = pair; tile < p.num_tiles; tile += npairs) {
         const int m0 = (tile % p.tiles_m) * 256 + 128 * (int)rank;
         const int nb = (tile / p.tiles_m) * 256 + 128 * (int)rank;
@@ -950,8 +981,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
           if (!wait_or_fail(&stg_empty[s], ph ^ 1, abort_flag)) goto done;
           uint8_t* sa = stg + (size_t)s * (kI3StgA + kI3StgB);
           mbar_arrive_expect_tx(&stg_full[s], kI3StgA + kI3StgB);
-          tma_load_2d(sa, &tmap_x, kt * 64, m0, &stg_full[s]);
-          tma_load_2d(sa + kI3StgA, &tmap_w, kt * 64, nb, &stg_full[s]);
+          tma_load_2d(sa, &tmap_x, kt * (A8 ? 128 : 64), m0, &stg_full[s]);
+          if (W8) {
+            // the operand slot is free once the MMAs that read it have completed
+            if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
+            if (leader) mbar_arrive_expect_tx(&op_full[o], 2 * kI3OpB);
+            tma_load_2d_2cta(opb + (size_t)o * kI3OpB, &tmap_w, kt * 128, nb, mapa_u32(&op_full[o], 0));
+            if (++o == kI3Ops) { o = 0; oph ^= 1; }
+          } else {
+            tma_load_2d(sa + kI3StgA, &tmap_w, kt * 64, nb, &stg_full[s]);
+          }
           if (++s == kI3Stg) { s = 0; ph ^= 1; }
         }
       }
@@ -985,7 +1024,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
       }
     }
   } else if (warp < kI3AWarp0) {
-    // B: packed rows -> 128B-swizzled int8 in shared memory
+    // B: packed rows -> 128B-swizzled int8 in shared memory (idle for W8)
+    if (W8) goto done;
     const int t = threadIdx.x - 64;
     int s = 0, o = 0;
     unsigned ph = 0, oph = 0;
@@ -1019,8 +1059,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
         if (!wait_or_fail(&stg_full[s], ph, abort_flag)) goto done;
         if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
         tc_fence_after();
-        const uint8_t* sa = stg + (size_t)s * (kI3StgA + kI3StgB) + row * 64;
         uint32_t w[32];
+        if (A8) {
+          // 128 int8 codes, 16-byte chunk j at 16 (j ^ (row mod 8))
+          const uint8_t* sa = stg + (size_t)s * (kI3StgA + kI3StgB) + row * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 in = *reinterpret_cast<const uint4*>(sa + 16 * (j ^ (row & 7)));
+            w[4 * j + 0] = in.x;
+            w[4 * j + 1] = in.y;
+            w[4 * j + 2] = in.z;
+            w[4 * j + 3] = in.w;
+          }
+        } else {
+        const uint8_t* sa = stg + (size_t)s * (kI3StgA + kI3StgB) + row * 64;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint4 in = *reinterpret_cast<const uint4*>(sa + 16 * (j ^ ((row >> 1) & 3)));
@@ -1034,6 +1086,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
           w[8 * j + 5] = o1.y;
           w[8 * j + 6] = o1.z;
           w[8 * j + 7] = o1.w;
+        }
         }
         tmem_st32(trow + 32u * (uint32_t)o, w);
         tmem_wait_st();
@@ -1061,8 +1114,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
       const int row = m0 + 32 * q + lane;
       const float sx = (row < p.M) ? xs[row] : 0.f;
       if (p.tma_store) {
-        epilogue_int4_bf16_tma(p, &tmap_y, tmem, m0, n0, q, ch, lane, sx, ws, epi + (size_t)ch * kEpiStage,
-                               mapa_u32(&acc_empty[0], 0));
+        epilogue_int4_bf16_tma<C::Shift>(p, &tmap_y, tmem, m0, n0, q, ch, lane, sx, ws,
+                                         epi + (size_t)ch * kEpiStage, mapa_u32(&acc_empty[0], 0));
       } else if (ch == 0) {
         epilogue_store<0>(p, tmem, m0, n0, q, lane, sx, ws, 1.0f, &acc_empty[0], mapa_u32(&acc_empty[0], 0));
       } else {
@@ -1229,6 +1282,7 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
   p.out = (int)out;
   p.vec_ok = ((reinterpret_cast<uintptr_t>(Y) % 16) == 0 && (ldy * (int64_t)esz) % 16 == 0) ? 1 : 0;
   p.tma_store = 0;
+  p.acc_shift = 8;
   p.tiles_m = (int)((M + kBM - 1) / kBM);
   p.tiles_n = (int)((N + kBN - 1) / kBN);
   p.num_tiles = p.tiles_m * p.tiles_n;
@@ -1254,9 +1308,9 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
       std::memset(&ty, 0, sizeof(ty));
       p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
       if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
-      if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int4_2sm_ts_kernel), (int)kI3Smem))
+      if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<false, false>), (int)kI3Smem))
         return RQ_ERR_CUDA;
-      gemm_int4_2sm_ts_kernel<<<grid2, kI3Threads, kI3Smem, st>>>(tx2, tw2, ty, p);
+      gemm_int_2sm_ts_kernel<false, false><<<grid2, kI3Threads, kI3Smem, st>>>(tx2, tw2, ty, p);
       return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
     }
     if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int4_kernel), (int)kI4Smem)) return RQ_ERR_CUDA;
@@ -1264,6 +1318,72 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
   } else {
     return fmt == RQ_MXFP4 ? launch_fp4<true>(p, xc, xs, wc, ws, Y, M, N, K, ldy, out, st)
                            : launch_fp4<false>(p, xc, xs, wc, ws, Y, M, N, K, ldy, out, st);
+  }
+  return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+// Integer GEMM with 8-bit activation codes (W4A8, W6A6, W8A8 and the mixed
+// 6/8-bit pairs): always the two-SM kernel (any M; a pair's second 128 rows
+// are clipped by TMA and the epilogue when M <= 128).  W4A4 goes through
+// gemm_dispatch.
+inline rq_status int_gemm_dispatch(const uint8_t* xc, const float* xs, rq_format xfmt, const uint8_t* wc,
+                                   const float* ws, rq_format wfmt, int64_t M, int64_t N, int64_t K, void* Y,
+                                   int64_t ldy, rq_out out, cudaStream_t st) {
+  auto is_int = [](rq_format f) { return f == RQ_INT4 || f == RQ_INT6 || f == RQ_INT8; };
+  if (!is_int(xfmt) || !is_int(wfmt)) return RQ_ERR_INVALID_ARG;
+  if (xfmt == RQ_INT4 && wfmt == RQ_INT4)
+    return gemm_dispatch(xc, xs, nullptr, wc, ws, nullptr, M, N, K, RQ_INT4, Y, ldy, out, st);
+  if (xfmt == RQ_INT4) return RQ_ERR_UNSUPPORTED_SHAPE;  // 4-bit activations with wider weights
+  const bool w8 = wfmt != RQ_INT4;
+  if (M < 0 || N < 0 || K <= 0 || ldy < N) return RQ_ERR_INVALID_ARG;
+  if (out != RQ_OUT_F32 && out != RQ_OUT_BF16 && out != RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
+  if (M > 0 && N > 0 && (!xc || !xs || !wc || !ws || !Y)) return RQ_ERR_INVALID_ARG;
+  if (K > 65536 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (K % 128 != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return RQ_OK;
+  const size_t esz = out == RQ_OUT_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(xc) | reinterpret_cast<uintptr_t>(wc)) & 15) return RQ_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(Y) % esz != 0) return RQ_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(xs) & 3) || (reinterpret_cast<uintptr_t>(ws) & 15)) return RQ_ERR_ALIGNMENT;
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.xscale = xs;
+  p.wscale = ws;
+  p.y = Y;
+  p.ldy = ldy;
+  p.out = (int)out;
+  p.vec_ok = ((reinterpret_cast<uintptr_t>(Y) % 16) == 0 && (ldy * (int64_t)esz) % 16 == 0) ? 1 : 0;
+  p.acc_shift = w8 ? I3<true, true>::Shift : I3<true, false>::Shift;
+  p.tiles_m = (int)((M + 255) / 256);
+  p.tiles_n = (int)((N + kBN - 1) / kBN);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  const int sms = gemm_num_sms() & ~1;
+  const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
+
+  CUtensorMap tx, tw, ty;
+  std::memset(&ty, 0, sizeof(ty));
+  if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return RQ_ERR_CUDA;
+  if (w8) {
+    if (!make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return RQ_ERR_CUDA;
+  } else {
+    if (!make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return RQ_ERR_CUDA;
+  }
+  p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
+  if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
+  if (w8) {
+    if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<true, true>),
+                          (int)I3<true, true>::Smem))
+      return RQ_ERR_CUDA;
+    gemm_int_2sm_ts_kernel<true, true><<<grid2, kI3Threads, I3<true, true>::Smem, st>>>(tx, tw, ty, p);
+  } else {
+    if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<true, false>),
+                          (int)I3<true, false>::Smem))
+      return RQ_ERR_CUDA;
+    gemm_int_2sm_ts_kernel<true, false><<<grid2, kI3Threads, I3<true, false>::Smem, st>>>(tx, tw, ty, p);
   }
   return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }

@@ -51,7 +51,10 @@ namespace rq {
 #define RQ_FULL_WIDTH_THREADS 256
 #endif
 
-enum RotMode : int { kModeInt4 = 0, kModeNvfp4 = 1, kModeF32 = 2, kModeAmax = 3, kModeKv4 = 4, kModeMxfp4 = 5 };
+enum RotMode : int {
+  kModeInt4 = 0, kModeNvfp4 = 1, kModeF32 = 2, kModeAmax = 3, kModeKv4 = 4, kModeMxfp4 = 5,
+  kModeInt8 = 6  // 6- or 8-bit symmetric codes, one per byte (qmax 31 or 127)
+};
 
 struct RotParams {
   const uint8_t* x;    // bf16 input (bytes)
@@ -64,7 +67,8 @@ struct RotParams {
   int contiguous;      // 1: row r starts at x + r * K * 2
   const int8_t* signs; // [K]
   uint8_t* codes;      // [rows, K/2]
-  float* scales_f32;   // INT4: [rows]
+  float* scales_f32;   // INT4 / INT6 / INT8: [rows]
+  float qmax;          // INT6 / INT8: 31 or 127
   uint8_t* scales_e4m3;// NVFP4: [rows, K/16]; MXFP4: E8M0 [rows, K/32]
   __half* kv_scale;    // KV4: [rows]
   __half* kv_zero;     // KV4: [rows]
@@ -263,6 +267,36 @@ __device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c,
       w[jj] = pack8_magic(q);
     }
     out[j4] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// 6- / 8-bit per-row quantization of v (true value = v * c * chi): codes
+// rint(x * qmax / amax) in [-qmax, qmax], one two's-complement byte each.
+// Writes 128 bytes at dst.
+__device__ __forceinline__ void quant_int8_store(const float (&v)[128], float c, float amax_true, float qmax, int m,
+                                                 uint8_t* dst) {
+  const float r = amax_true > 0.f ? __fdiv_rn(qmax, amax_true) : 0.0f;
+  const float cr = c * r;
+  uint4* out = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j2 = 0; j2 < 8; ++j2) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // chunk j = 8 elements -> two words
+      const int j = 2 * j2 + h;
+      const float mul = with_sign(cr, chi_signbit(j, m));
+      uint32_t q[8];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float2 t = __ffma2_rn(make_float2(v[8 * j + e], v[8 * j + e + 1]), make_float2(mul, mul),
+                                    make_float2(kRoundMagic, kRoundMagic));
+        q[e] = __float_as_uint(t.x);
+        q[e + 1] = __float_as_uint(t.y);
+      }
+      w[2 * h] = gather_low_bytes(q[0], q[1], q[2], q[3]);
+      w[2 * h + 1] = gather_low_bytes(q[4], q[5], q[6], q[7]);
+    }
+    out[j2] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -550,9 +584,48 @@ __device__ __forceinline__ void full_store_int4(const float (&y)[2][NB][64 / NB]
     }
 }
 
+// 6- / 8-bit quantize + store of the full-width layout: COLS bytes per (block, half).
+template <int NB>
+__device__ __forceinline__ void full_store_int8(const float (&y)[2][NB][64 / NB], float rr, uint8_t* crow, int b) {
+  constexpr int COLS = 64 / NB;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int bb = 0; bb < NB; ++bb) {
+      uint32_t q[COLS];
+#pragma unroll
+      for (int cc = 0; cc < COLS; cc += 2) {
+        const float2 t = __ffma2_rn(make_float2(y[h][bb][cc], y[h][bb][cc + 1]), make_float2(rr, rr),
+                                    make_float2(kRoundMagic, kRoundMagic));
+        q[cc] = __float_as_uint(t.x);
+        q[cc + 1] = __float_as_uint(t.y);
+      }
+      uint8_t* dst = crow + bb * 128 + 64 * h + b * COLS;
+      if (COLS == 2) {
+        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)((q[0] & 0xFFu) | ((q[1 % COLS] & 0xFFu) << 8));
+      } else {
+        uint32_t wd[COLS / 4 > 0 ? COLS / 4 : 1];
+#pragma unroll
+        for (int w4 = 0; w4 < COLS / 4; ++w4)
+          wd[w4] = gather_low_bytes(q[(4 * w4) % COLS], q[(4 * w4 + 1) % COLS], q[(4 * w4 + 2) % COLS],
+                                    q[(4 * w4 + 3) % COLS]);
+        if (COLS == 4) {
+          *reinterpret_cast<uint32_t*>(dst) = wd[0];
+        } else if (COLS == 8) {
+          *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1 % (COLS / 4)]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < COLS / 16; ++u)
+            reinterpret_cast<uint4*>(dst)[u] = make_uint4(wd[(4 * u) % (COLS / 4)], wd[(4 * u + 1) % (COLS / 4)],
+                                                          wd[(4 * u + 2) % (COLS / 4)], wd[(4 * u + 3) % (COLS / 4)]);
+        }
+      }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The kernel.  NBF = 0: block-diagonal (B = 128), any mode.  NBF = 2..32:
-// full-width rotation of K = 128*NBF (INT4 and F32 modes).
+// full-width rotation of K = 128*NBF (INT4, INT6/INT8 and F32 modes).
 // ---------------------------------------------------------------------------
 template <int MODE, int NBF>
 __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_kernel(const RotParams p) {
@@ -651,6 +724,13 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
           quant_int4_store(v, c, amax_row, m, p.codes + row * (p.K / 2) + (size_t)b * 64);
           if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
         }
+      } else if (MODE == kModeInt8) {
+        const float a = valid ? absmax128(v) * c : 0.f;
+        const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
+        if (valid) {
+          quant_int8_store(v, c, amax_row, p.qmax, m, p.codes + row * p.K + (size_t)b * 128);
+          if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, p.qmax);
+        }
       } else if (MODE == kModeNvfp4) {
         if (valid)
           quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
@@ -682,7 +762,7 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
           issue_tile_load(p, nt, stage, &full[st]);
         }
       }
-      if (MODE == kModeInt4) {
+      if (MODE == kModeInt4 || MODE == kModeInt8) {
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -694,10 +774,14 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
               a1 = fmaxf(a1, fabsf(y[h][bb][cc + 1]));
             }
         const float amax_row = row_max(valid ? fmaxf(a0, a1) : 0.f, RPS, nb, 1, grp, 0, slots);
-        if (valid) {
+        if (valid && MODE == kModeInt4) {
           const float rr = amax_row > 0.f ? __fdiv_rn(7.0f, amax_row) : 0.0f;
           full_store_int4<NB>(y, rr, p.codes + row * (p.K / 2), b);
           if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
+        } else if (valid) {
+          const float rr = amax_row > 0.f ? __fdiv_rn(p.qmax, amax_row) : 0.0f;
+          full_store_int8<NB>(y, rr, p.codes + row * p.K, b);
+          if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, p.qmax);
         }
       } else if (MODE == kModeF32) {
         if (valid) {

@@ -15,14 +15,15 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librq.so")
 
-RQ_INT4, RQ_NVFP4, RQ_MXFP4 = 0, 1, 2
+RQ_INT4, RQ_NVFP4, RQ_MXFP4, RQ_INT8, RQ_INT6 = 0, 1, 2, 3, 4
 RQ_OUT_F32, RQ_OUT_BF16, RQ_OUT_I32_ACC = 0, 1, 2
 RQ_SCALE_DYNAMIC, RQ_SCALE_STATIC = 0, 1
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3: "RQ_ERR_ALIGNMENT",
           4: "RQ_ERR_UNSUPPORTED_DEVICE", 5: "RQ_ERR_CUDA", 6: "RQ_ERR_TIMEOUT"}
 EXPORTED = ["rq_init", "rq_status_string", "rq_workspace_bytes", "rq_rotate_quantize", "rq_prepare_weights",
             "rq_w4a4_gemm", "rq_kv_rotate_quantize", "rq_rotate_f32", "rq_get_device_error",
-            "rq_rotate_quantize_nvfp4_noalloc", "rq_kv4_attention_workspace_bytes", "rq_kv4_decode_attention"]
+            "rq_rotate_quantize_nvfp4_noalloc", "rq_kv4_attention_workspace_bytes", "rq_kv4_decode_attention",
+            "rq_int_gemm"]
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("librq.so not built: run `python -m rotation_w4a4_quantization_b200.build`")
@@ -43,6 +44,8 @@ lib.rq_prepare_weights.argtypes = [_p, _i64, _i64, _i64, _p, _i, _i, _p, _p, _p,
 lib.rq_prepare_weights.restype = _i
 lib.rq_w4a4_gemm.argtypes = [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i, _p, _i64, _i, _p]
 lib.rq_w4a4_gemm.restype = _i
+lib.rq_int_gemm.argtypes = [_p, _p, _i, _p, _p, _i, _i64, _i64, _i64, _p, _i64, _i, _p]
+lib.rq_int_gemm.restype = _i
 lib.rq_kv_rotate_quantize.argtypes = [_p, _i64, _i64, _i64, _i64, ctypes.POINTER(_i64), _p, _p, _p, _p, _p]
 lib.rq_kv_rotate_quantize.restype = _i
 lib.rq_rotate_f32.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i64, _p]
@@ -79,7 +82,9 @@ def _stream(t=None):
 
 
 def _fmt(fmt):
-    return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4, "mxfp4": RQ_MXFP4}[fmt] if isinstance(fmt, str) else int(fmt)
+    if isinstance(fmt, str):
+        return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4, "mxfp4": RQ_MXFP4, "int8": RQ_INT8, "int6": RQ_INT6}[fmt]
+    return int(fmt)
 
 
 def init(device=0):
@@ -97,6 +102,9 @@ def _require_cuda(*ts):
 
 
 def _alloc_quant_outputs(rows, k, fmt, device):
+    if fmt in (RQ_INT8, RQ_INT6):  # one int8 code per byte
+        return (torch.empty((rows, k), dtype=torch.int8, device=device),
+                torch.empty((rows,), dtype=torch.float32, device=device))
     codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=device)
     if fmt == RQ_INT4:
         scales = torch.empty((rows,), dtype=torch.float32, device=device)
@@ -113,6 +121,7 @@ def rotate_quantize(x, signs, block=128, fmt="int4", gmode="dynamic", gscale=Non
     INT4: codes uint8 [M, K/2], scales fp32 [M], gscale None.
     NVFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/16] (E4M3), gscale fp32 [1].
     MXFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/32] (E8M0), gscale None.
+    INT8 / INT6: codes int8 [M, K] (one code per byte), scales fp32 [M], gscale None.
     """
     _require_cuda(x, signs)
     f = _fmt(fmt)
@@ -157,6 +166,25 @@ def w4a4_gemm(xq, wq, fmt="int4", out="f32", y=None):
         y = torch.empty((m, n), dtype=dt, device=xc.device)
     _check(lib.rq_w4a4_gemm(_ptr(xc), _ptr(xs), _ptr(xg), _ptr(wc), _ptr(ws), _ptr(wg), m, n, 2 * kh, f, _ptr(y),
                             y.stride(0), o, _stream(xc)), "rq_w4a4_gemm")
+    return y
+
+
+def int_gemm(xq, xfmt, wq, wfmt, out="f32", y=None):
+    """Y = deq(xq) . deq(wq)^T for integer codes of different widths (W4A8, W6A6,
+    W8A8, W4A4): xq / wq are (codes, scales, _) triples from rotate_quantize /
+    prepare_weights with formats xfmt / wfmt in {"int4", "int6", "int8"}."""
+    xc, xs = xq[0], xq[1]
+    wc, ws = wq[0], wq[1]
+    _require_cuda(xc, xs, wc, ws)
+    fx, fw = _fmt(xfmt), _fmt(wfmt)
+    o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16, "i32": RQ_OUT_I32_ACC}[out]
+    m, n = xc.shape[0], wc.shape[0]
+    k = xc.shape[1] * (2 if fx == RQ_INT4 else 1)
+    if y is None:
+        dt = {RQ_OUT_F32: torch.float32, RQ_OUT_BF16: torch.bfloat16, RQ_OUT_I32_ACC: torch.int32}[o]
+        y = torch.empty((m, n), dtype=dt, device=xc.device)
+    _check(lib.rq_int_gemm(_ptr(xc), _ptr(xs), fx, _ptr(wc), _ptr(ws), fw, m, n, k, _ptr(y), y.stride(0), o,
+                           _stream(xc)), "rq_int_gemm")
     return y
 
 

@@ -78,6 +78,16 @@ def check_int4_quant(codes_gpu, scales_gpu, xr):
     return check_codes(qg, q, tie, what="int4 codes")
 
 
+def check_int_quant(codes_gpu, scales_gpu, xr, bits):
+    """codes_gpu int8 [M, K] (one 6- or 8-bit code per byte), scales_gpu fp32 [M]
+    against the oracle on rotated fp64 xr."""
+    q, s, tie = quant.int_sym_rows(xr, bits)
+    sg = np.asarray(scales_gpu, dtype=np.float64)
+    so = s.astype(np.float64)
+    assert np.all(np.abs(sg - so) <= SCALE_RTOL * so + 1e-38), np.max(np.abs(sg - so) / np.maximum(so, 1e-38))
+    return check_codes(np.asarray(codes_gpu, dtype=np.int64), q, tie, what="int%d codes" % bits)
+
+
 def check_nvfp4_quant(codes_gpu, sc_gpu, g_gpu, xr, g_ref=None):
     g_o = quant.nvfp4_global_scale(xr) if g_ref is None else np.float32(g_ref)
     if g_ref is None:
