@@ -81,6 +81,13 @@ TRAFFIC = {
 }
 
 
+def code_bytes(fmt, rows, k):
+    """Bytes of codes and scales the rotate kernel writes for `rows` rows of K."""
+    return {"int4": rows * k // 2 + rows * 4, "nvfp4": rows * k // 2 + rows * (k // 16),
+            "mxfp4": rows * k // 2 + rows * (k // 32), "int8": rows * k + rows * 4,
+            "int6": rows * k + rows * 4}[fmt]
+
+
 def source_fingerprint(files):
     import hashlib
     m = hashlib.sha256()
@@ -148,11 +155,12 @@ class Workload:
         else:
             c = self.cfg
             self.fmt = c["fmt"]
+            self.wfmt = c.get("wfmt", self.fmt)
             self.block = c["block"]
             self.x = syn.activations(name, device=device, seed_offset=seed_offset)
             w = syn.weights(name, device=device)
             self.signs = syn.workload_signs(name).to(device)
-            self.wq = rq.prepare_weights(w, self.signs, self.block, self.fmt)
+            self.wq = rq.prepare_weights(w, self.signs, self.block, self.wfmt)
             del w
             m, k, n = c["M"], c["K"], c["N"]
             self.xq_out = rq._alloc_quant_outputs(m, k, rq._fmt(self.fmt), device)
@@ -160,8 +168,7 @@ class Workload:
             self.ws = torch.empty((16,), dtype=torch.uint8, device=device)
             self.y = torch.empty((m, n), dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32,
                                  device=device)
-            scale_bytes = {"int4": m * 4, "nvfp4": m * (k // 16), "mxfp4": m * (k // 32)}[self.fmt]
-            self.quant_bytes = m * k * 2 + m * k // 2 + scale_bytes
+            self.quant_bytes = m * k * 2 + code_bytes(self.fmt, m, k)
             self.gemm_ops = 2 * m * n * k
             self.h2d_bytes = self.x.numel() * 2
         self.d2h_bytes = 0
@@ -191,7 +198,8 @@ class Workload:
             return "rotate_kernel<KV4>"
         if self.fmt == "nvfp4" and self.nvfp4_one_pass():
             return "rotate_nvfp4_resident_kernel"
-        return "rotate_kernel<full width>" if self.block == 0 else "rotate_kernel<128-blocks>"
+        mode = "INT8, " if self.fmt in ("int8", "int6") else ""
+        return "rotate_kernel<%s%s>" % (mode, "full width" if self.block == 0 else "128-blocks")
 
     def gemm_launches(self):
         return 0 if (self.kv or self.kvdec) else 1
@@ -212,12 +220,22 @@ class Workload:
     def gemm(self, xq):
         if self.kv or self.kvdec:
             return None
+        if self.fmt in ("int8", "int6"):
+            return self.rq.int_gemm(xq, self.fmt, self.wq, self.wfmt, self.y_dtype, y=self.y)
         return self.rq.w4a4_gemm(xq, self.wq, self.fmt, self.y_dtype, y=self.y)
 
     def result(self):
         if self.kvdec:
             return self.out
         return self.outs[0][0] if self.kv else self.y
+
+
+def gemm_kernel_name(wl, two_sm):
+    if wl.fmt in ("int8", "int6"):
+        return "gemm_int_2sm_ts_kernel<A8, %s>" % ("W8" if wl.wfmt in ("int8", "int6") else "W4")
+    if wl.fmt == "int4":
+        return "gemm_int_2sm_ts_kernel<A4, W4>" if two_sm else "gemm_int4_kernel"
+    return ("gemm_fp4_2sm_kernel" if two_sm else "gemm_fp4_kernel") + "<%s>" % wl.fmt
 
 
 # --------------------------------------------------------------------------- clocks
@@ -325,7 +343,10 @@ def oracle_sample(name, rows):
     k, n = c["K"], c["N"]
     block = c["block"]
     wr = ohad.rotate(w, s, block)
-    if c["fmt"] == "int4":
+    bits = {"int4": 4, "int6": 6, "int8": 8}
+    if c["fmt"] in ("int8", "int6"):
+        qw, sw, _ = oquant.int_sym_rows(wr, bits[c.get("wfmt", c["fmt"])])
+    elif c["fmt"] == "int4":
         qw, sw, _ = oquant.int4_sym_rows(wr)
     elif c["fmt"] == "nvfp4":
         gw = oquant.nvfp4_global_scale(wr)
@@ -334,7 +355,10 @@ def oracle_sample(name, rows):
         ew, sfw, _, _ = oquant.mxfp4_rows(wr)
     t0 = time.perf_counter()
     xr = ohad.rotate(x, s, block)
-    if c["fmt"] == "int4":
+    if c["fmt"] in ("int8", "int6"):
+        qx, sx, _ = oquant.int_sym_rows(xr, bits[c["fmt"]])
+        qx.astype(np.int8)
+    elif c["fmt"] == "int4":
         qx, sx, _ = oquant.int4_sym_rows(xr)
         oquant.pack_nibbles(qx)
     elif c["fmt"] == "nvfp4":
@@ -345,15 +369,16 @@ def oracle_sample(name, rows):
         ex, sfx, _, _ = oquant.mxfp4_rows(xr)
         oquant.pack_nibbles(ex)
     t1 = time.perf_counter()
-    if c["fmt"] == "int4":
+    if c["fmt"] in ("int8", "int6"):
+        ogemm.int4_y(ogemm.int_acc(qx, qw), sx, sw)
+    elif c["fmt"] == "int4":
         ogemm.int4_y(ogemm.int4_acc(qx, qw), sx, sw)
     elif c["fmt"] == "nvfp4":
         ogemm.nvfp4_y(ex, sfx, gx, ew, sfw, gw)
     else:
         ogemm.mxfp4_y(ex, sfx, ew, sfw)
     t2 = time.perf_counter()
-    scale_bytes = {"int4": rows * 4, "nvfp4": rows * (k // 16), "mxfp4": rows * (k // 32)}[c["fmt"]]
-    nbytes = rows * k * 2 + rows * k // 2 + scale_bytes
+    nbytes = rows * k * 2 + code_bytes(c["fmt"], rows, k)
     return (nbytes / (t1 - t0) / 1e9, 2.0 * rows * n * k / (t2 - t1) / 1e12, t2 - t0,
             "%d of %d rows of X with the full W" % (rows, c["M"]))
 
@@ -369,7 +394,7 @@ def blas_threads():
 
 def sample_rows(name):
     return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096,
-            "q_proj_mxfp4": 256, "kv4_decode": 1024}[name]
+            "q_proj_mxfp4": 256, "kv4_decode": 1024, "q_proj_w4a8": 512, "q_proj_w8a8": 512}[name]
 
 
 # --------------------------------------------------------------------------- main
@@ -476,8 +501,7 @@ def main():
         two_sm = wl.cfg["M"] > 128
         roof_g = {"bound": "tensor", "achieved": round(wl.gemm_ops / (g_mean_ms * 1e-3) / 1e12, 1), "peak": peak_t,
                   "unit": "TFLOP/s", "traffic": traffic("gemm", args.workload),
-                  "kernel": ("gemm_int4_2sm_ts_kernel" if two_sm else "gemm_int4_kernel") if wl.fmt == "int4" else
-                            ("gemm_fp4_2sm_kernel" if two_sm else "gemm_fp4_kernel") + "<%s>" % wl.fmt,
+                  "kernel": gemm_kernel_name(wl, two_sm),
                   "peak_source": "%s bf16 x %g (nominal %s/bf16 ratio)" % (peaks["src"], ratio,
                                                                            "int8" if ratio == 2 else "fp4")}
         roof_g["frac"] = round(roof_g["achieved"] / peak_t, 4)

@@ -36,11 +36,15 @@ def main(argv):
     elif kind == "gemm":
         x = syn.activations(name, device="cuda")
         w = syn.weights(name, device="cuda")
-        wq = rq.prepare_weights(w, s, c["block"], c["fmt"])
+        wfmt = c.get("wfmt", c["fmt"])
+        wq = rq.prepare_weights(w, s, c["block"], wfmt)
         xq = rq.rotate_quantize(x, s, c["block"], c["fmt"])
         y = torch.empty((c["M"], c["N"]), dtype=torch.bfloat16, device="cuda")
         for _ in range(reps):
-            rq.w4a4_gemm(xq, wq, c["fmt"], "bf16", y=y)
+            if c["fmt"] in ("int8", "int6"):
+                rq.int_gemm(xq, c["fmt"], wq, wfmt, "bf16", y=y)
+            else:
+                rq.w4a4_gemm(xq, wq, c["fmt"], "bf16", y=y)
     elif kind == "attention":
         kc = rq.kv_rotate_quantize(syn.kv(batch=4, device="cuda", which=0), s)
         vc = rq.kv_rotate_quantize(syn.kv(batch=4, device="cuda", which=1), s)

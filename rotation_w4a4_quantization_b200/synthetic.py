@@ -41,6 +41,9 @@ WORKLOADS = {
     "q_proj_mxfp4": dict(index=6, M=2048, K=4096, N=4096, block=128, fmt="mxfp4"),
     # a decode step over the kv4 workload's cache (written once by the KV4 kernel)
     "kv4_decode": dict(index=7, B=16, H=32, S=4096, D=128),
+    # 8-bit activations: W4A8 (4-bit weights) and W8A8, q_proj shapes and recipe
+    "q_proj_w4a8": dict(index=8, M=2048, K=4096, N=4096, block=0, fmt="int8", wfmt="int4"),
+    "q_proj_w8a8": dict(index=9, M=2048, K=4096, N=4096, block=0, fmt="int8", wfmt="int8"),
 }
 
 
@@ -71,7 +74,7 @@ def activations(name, rows=None, device="cpu", seed_offset=0):
     x = torch.randn((m, k), generator=g, device=device, dtype=torch.float32)
     if name == "tiny_int4":
         x[:, [3, 77, 200, 411]] *= 50.0
-    elif name in ("q_proj_int4", "q_proj_nvfp4", "q_proj_mxfp4"):
+    elif name in ("q_proj_int4", "q_proj_nvfp4", "q_proj_mxfp4", "q_proj_w4a8", "q_proj_w8a8"):
         gp = _gen(3000 + w["index"], "cpu")
         ch = torch.randperm(k, generator=gp)[:8]
         mult = 20.0 + 40.0 * torch.rand((8,), generator=gp, dtype=torch.float64)
