@@ -118,6 +118,17 @@ rq_status launch_block(RotParams p, cudaStream_t st) {
   return launch_rotate<MODE, 0>(p, st);
 }
 
+// K = 4096: the 64 x 64 two-pass kernel, two CTAs of four row teams per SM.
+template <int MODE>
+rq_status launch_full4096(RotParams p, cudaStream_t st) {
+  const int64_t ctas = (p.rows + kR64Teams - 1) / kR64Teams;
+  const int64_t cap = 2 * (int64_t)num_sms_of_current_device();
+  const int64_t grid = ctas < cap ? ctas : cap;
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_full4096_kernel<MODE>), (int)kR64Smem)) return RQ_ERR_CUDA;
+  rotate_full4096_kernel<MODE><<<(unsigned)grid, kR64Threads, kR64Smem, st>>>(p);
+  return last_launch_status();
+}
+
 template <int MODE>
 rq_status launch_full(RotParams p, cudaStream_t st) {
   switch (p.nb) {
@@ -125,7 +136,7 @@ rq_status launch_full(RotParams p, cudaStream_t st) {
     case 4: return launch_rotate<MODE, 4>(p, st);
     case 8: return launch_rotate<MODE, 8>(p, st);
     case 16: return launch_rotate<MODE, 16>(p, st);
-    case 32: return launch_rotate<MODE, 32>(p, st);
+    case 32: return launch_full4096<MODE>(p, st);
     default: return RQ_ERR_UNSUPPORTED_SHAPE;
   }
 }

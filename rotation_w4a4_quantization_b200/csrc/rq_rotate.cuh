@@ -805,6 +805,183 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
 }
 
 // ---------------------------------------------------------------------------
+// Full-width rotation of K = 4096 as a 64 x 64 two-pass transform.
+//
+// Sylvester's H_4096 is the Kronecker product of twelve H_2, one per bit of
+// the element index n, so the bits can be transformed in any grouping.  The
+// row is read as a 64 x 64 matrix X[a][b] with a = bits 3..8 of n and
+// b = bits 0..2 and 9..11: H_64 along b in every matrix row, then H_64 along a
+// in every column.  A team of 64 threads (two warps) owns one row at a time.
+// Thread a loads matrix row a -- eight 16-byte pieces at elements
+// 8 a + 512 i, so each warp load instruction reads 512 contiguous bytes --
+// signs and transforms it (the next row's loads are issued before this row's
+// arithmetic), writes it to shared memory and, after a team barrier,
+// transforms column b = a.  The codes of its outputs (a = 0..63, b) go back
+// through shared memory as bytes, and thread t stores the codes of outputs
+// 64 t .. 64 t + 63 with 16-byte stores.  Four teams per CTA, two CTAs per SM;
+// a team synchronises on its own named barrier (1..4).  Shared-memory
+// granules are XOR-swizzled so that the row writes, column reads and code
+// transposes are free of bank conflicts (the code reads: two-way).
+// ---------------------------------------------------------------------------
+constexpr int kR64Teams = 4;
+constexpr int kR64Threads = 64 * kR64Teams;
+constexpr size_t kR64TeamBytes = 64 * 64 * 4 + 64 * 64 + 16;  // fp32 transpose | code bytes | amax slots
+constexpr size_t kR64Smem = 2048 * 4 + kR64Teams * kR64TeamBytes;
+
+__device__ __forceinline__ void team_sync(int team) {
+  asm volatile("bar.sync %0, 64;" ::"r"(team + 1) : "memory");
+}
+
+// 64-point fast Walsh-Hadamard transform in registers (unnormalized).
+__device__ __forceinline__ void fwht64(float (&v)[64]) {
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) {
+    const float a = v[i], b = v[i + 1];
+    v[i] = a + b;
+    v[i + 1] = a - b;
+  }
+#pragma unroll
+  for (int h = 2; h < 64; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) {
+      if ((i & h) == 0) {
+        const float2 a = make_float2(v[i], v[i + 1]);
+        const float2 b = make_float2(v[i + h], v[i + h + 1]);
+        const float2 s = __fadd2_rn(a, b);
+        const float2 d = __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+        v[i] = s.x;
+        v[i + 1] = s.y;
+        v[i + h] = d.x;
+        v[i + h + 1] = d.y;
+      }
+    }
+  }
+}
+
+// Matrix row a of `row` -- elements 8 a + 512 i + e, i, e = 0..7 (bf16) -- into
+// registers, bypassing L1.
+__device__ __forceinline__ void load_row64(const RotParams& p, int64_t row, int a, uint4 (&raw)[8]) {
+  const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.sS) + a;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint4 w;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                 : "l"(src + 64 * i));
+    raw[i] = w;
+  }
+}
+
+// Four code bytes (two's complement, element order) -> two packed nibble bytes.
+__device__ __forceinline__ uint32_t nibbles_of(uint32_t w0, uint32_t w1) {
+  const uint32_t a = w0 & 0x0F0F0F0Fu, b = w1 & 0x0F0F0F0Fu;
+  return __byte_perm(a | (a >> 4), b | (b >> 4), 0x6420);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const RotParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw);  // [2048] XOR masks, one per bf16 pair
+  const int team = threadIdx.x >> 6, t = threadIdx.x & 63, lane = threadIdx.x & 31;
+  uint8_t* tb = smem_raw + 2048 * 4 + (size_t)team * kR64TeamBytes;
+  float* tr = reinterpret_cast<float*>(tb);             // [a][b] fp32, 16-byte granule g of row a at g ^ (a mod 16)
+  uint8_t* cb = tb + 64 * 64 * 4;                       // [a][b] code bytes, 8-byte group g of row a at g ^ (a / 8)
+  float* slots = reinterpret_cast<float*>(cb + 64 * 64);
+  const int64_t step = (int64_t)gridDim.x * kR64Teams;
+  int64_t row = (int64_t)blockIdx.x * kR64Teams + team;
+  uint4 raw[8];
+  build_sign_table(p.signs, 32, smask, [&]() {
+    if (row < p.rows) load_row64(p, row, t, raw);
+  });
+  __syncthreads();
+
+#pragma unroll 1
+  for (; row < p.rows; row += step) {
+    float v[64];
+    {
+      const uint4* sm = reinterpret_cast<const uint4*>(smask) + t;  // the pairs of elements 8 t + 512 i + e
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint4 w = raw[i];
+        const uint4 s = sm[64 * i];
+        w.x ^= s.x;
+        w.y ^= s.y;
+        w.z ^= s.z;
+        w.w ^= s.w;
+        v[8 * i + 0] = __uint_as_float(w.x << 16);
+        v[8 * i + 1] = __uint_as_float(w.x & 0xFFFF0000u);
+        v[8 * i + 2] = __uint_as_float(w.y << 16);
+        v[8 * i + 3] = __uint_as_float(w.y & 0xFFFF0000u);
+        v[8 * i + 4] = __uint_as_float(w.z << 16);
+        v[8 * i + 5] = __uint_as_float(w.z & 0xFFFF0000u);
+        v[8 * i + 6] = __uint_as_float(w.w << 16);
+        v[8 * i + 7] = __uint_as_float(w.w & 0xFFFF0000u);
+      }
+    }
+    if (row + step < p.rows) load_row64(p, row + step, t, raw);
+    fwht64(v);
+#pragma unroll
+    for (int g = 0; g < 16; ++g)
+      *reinterpret_cast<float4*>(tr + 64 * t + 4 * (g ^ (t & 15))) =
+          make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    team_sync(team);
+#pragma unroll
+    for (int k = 0; k < 64; ++k) v[k] = tr[64 * k + 4 * ((t >> 2) ^ (k & 15)) + (t & 3)];
+    fwht64(v);
+    // v[k] is output n = (t mod 8) + 8 k + 512 (t / 8)
+    if (MODE == kModeF32) {
+      float* orow = p.out_f32 + row * p.ldo + (t & 7) + 512 * (t >> 3);
+#pragma unroll
+      for (int k = 0; k < 64; ++k) orow[8 * k] = v[k] * 0.015625f;
+      team_sync(team);  // every column read is done before the next row's writes
+      continue;
+    }
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; k += 4) {
+      a0 = fmaxf(a0, fabsf(v[k]));
+      a1 = fmaxf(a1, fabsf(v[k + 1]));
+      a2 = fmaxf(a2, fabsf(v[k + 2]));
+      a3 = fmaxf(a3, fabsf(v[k + 3]));
+    }
+    float a = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    if (lane == 0) slots[t >> 5] = a;
+    team_sync(team);
+    const float amax = fmaxf(slots[0], slots[1]) * 0.015625f;  // max |x~| (x~ = H x / 64, exact scaling)
+    const float qmax = MODE == kModeInt4 ? 7.0f : p.qmax;
+    const float rr = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.0f;
+    const float cr = rr * 0.015625f;
+#pragma unroll
+    for (int k = 0; k < 64; k += 2) {
+      const float2 q = __ffma2_rn(make_float2(v[k], v[k + 1]), make_float2(cr, cr),
+                                  make_float2(kRoundMagic, kRoundMagic));
+      cb[64 * k + (t ^ (8 * (k >> 3)))] = (uint8_t)__float_as_uint(q.x);
+      cb[64 * (k + 1) + (t ^ (8 * ((k + 1) >> 3)))] = (uint8_t)__float_as_uint(q.y);
+    }
+    team_sync(team);
+    // outputs 64 t + 8 r + e sit at a = 8 (t mod 8) + r, b = 8 (t / 8) + e
+    uint2 c[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      c[r] = *reinterpret_cast<const uint2*>(cb + 64 * (8 * (t & 7) + r) + 8 * ((t >> 3) ^ (t & 7)));
+    if (MODE == kModeInt4) {
+      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 2048 + 32 * t);
+      dst[0] = make_uint4(nibbles_of(c[0].x, c[0].y), nibbles_of(c[1].x, c[1].y), nibbles_of(c[2].x, c[2].y),
+                          nibbles_of(c[3].x, c[3].y));
+      dst[1] = make_uint4(nibbles_of(c[4].x, c[4].y), nibbles_of(c[5].x, c[5].y), nibbles_of(c[6].x, c[6].y),
+                          nibbles_of(c[7].x, c[7].y));
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 4096 + 64 * t);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(c[2 * i].x, c[2 * i].y, c[2 * i + 1].x, c[2 * i + 1].y);
+    }
+    if (t == 0) p.scales_f32[row] = __fdiv_rn(amax, qmax);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // NVFP4 with the dynamic per-tensor scale in ONE pass over HBM, for tensors that
 // fit in the SMs' combined shared memory: a cooperative launch (all CTAs
 // resident) where each CTA copies its rows into shared memory once, computes

@@ -197,3 +197,29 @@ def test_rejects_bad_arguments(rq):
     with pytest.raises(rq.RQError):
         rq.rotate_quantize(x[:, 1:], s[1:], 128, "int4")
     rq.get_device_error()
+
+
+# ---------------------------------------------------------------- K = 4096 full width: team edge cases
+@pytest.mark.parametrize("m", [1, 3, 5, 1185, 4097])
+@pytest.mark.parametrize("fmt", ["int4", "int8", "f32"])
+def test_full_width_4096_row_counts(rq, m, fmt):
+    """Fewer rows than a CTA's four row teams, a ragged last team, several rows
+    per team; a zero row; rows of a wider tensor (row stride 4160)."""
+    k = 4096
+    big = _gauss(m, k + 64, 300 + m, outliers=[(11, 60.0)])
+    big[m // 2] = 0
+    x = big[:, :k]
+    s = _signs(k, 77)
+    xr = hadamard.rotate(parity.bf16_to_f64(x), s.numpy(), 0)
+    view = big.cuda()[:, :k]
+    if fmt == "f32":
+        got = rq.rotate_f32(view, s.cuda(), 0)
+        parity.check_rotation(parity.to_np(got), xr)
+        return
+    codes, scales, _ = rq.rotate_quantize(view, s.cuda(), 0, fmt)
+    torch.cuda.synchronize()
+    if fmt == "int4":
+        parity.check_int4_quant(parity.to_np(codes), parity.to_np(scales), xr)
+    else:
+        parity.check_int_quant(parity.to_np(codes), parity.to_np(scales), xr, 8)
+    assert parity.to_np(scales)[m // 2] == 0
