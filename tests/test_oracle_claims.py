@@ -13,6 +13,11 @@ stand-ins (CPU only).
   section "When to rotate": rotations help MXFP4, whose scales are powers of
   two shared by 32 values.
 
+Same article, section "Gotchas" ("Block size matters"): a 128-wide block
+spreads an outlier over eight NVFP4 groups of 16, undoing the isolation the
+small groups give; the FP4 study it cites sizes block-wise rotations to the
+format's groups.
+
 "QuaRot (rotation-based outlier removal, W4A4KV4)", field "Bits": 6- and
 8-bit round to nearest are lossless after rotation; "SpinQuant (learned
 rotations + W4A4KV4)": W4A8 narrows the gap that W4A4 leaves.
@@ -130,3 +135,26 @@ def test_more_bits_after_rotation(case, request):
     assert e48 < 0.8 * e44
     assert _int_err(y, x, w, 8, 8) > 4 * e88
     assert _int_err(y, x, w, 6, 6) > 4 * e66
+
+
+def _mxfp4_err(y, a, b):
+    ea, sa, _, _ = quant.mxfp4_rows(a)
+    eb, sb, _, _ = quant.mxfp4_rows(b)
+    return metrics.rel_product_error(y, gemm.mxfp4_y(ea, sa, eb, sb))
+
+
+@pytest.mark.parametrize("case", ["qproj", "downproj"])
+def test_format_sized_block_rotations(case, request):
+    """NVFP4: a 16-wide rotation (one per scale group) costs less than a 128-wide
+    one (neither beats no rotation); MXFP4: the 32-wide rotation (one per E8M0
+    group) is the best of none / 16 / 32 / 128; per-token INT4 keeps gaining
+    with the block (none > 16 > 32 > 128)."""
+    x, w, s, _, _ = request.getfixturevalue(case)
+    y = x @ w.T
+    rot = {b: (hadamard.rotate(x, s, b), hadamard.rotate(w, s, b)) for b in (16, 32, 128)}
+    nv = {b: _fp4_err(y, *rot[b]) for b in rot}
+    mx = {b: _mxfp4_err(y, *rot[b]) for b in rot}
+    i4 = {b: _int4_err(y, *rot[b]) for b in rot}
+    assert nv[16] < nv[128] and _fp4_err(y, x, w) < nv[16]
+    assert mx[32] < min(mx[16], mx[128], _mxfp4_err(y, x, w))
+    assert _int4_err(y, x, w) > i4[16] > i4[32] > i4[128]

@@ -60,7 +60,8 @@ def test_rejects_non_power_of_two():
         hadamard.sylvester(12)
 
 
-@pytest.mark.parametrize("n,block", [(2, 0), (4, 0), (8, 0), (16, 0), (16, 4), (16, 8), (32, 16), (12, 4)])
+@pytest.mark.parametrize("n,block", [(2, 0), (4, 0), (8, 0), (16, 0), (16, 4), (16, 8), (32, 16), (12, 4),
+                                     (64, 32), (128, 16), (128, 32)])
 def test_rotate_matches_butterfly(n, block):
     rng = np.random.default_rng(7 + n + block)
     x = rng.standard_normal((5, n))
@@ -79,7 +80,7 @@ def test_onehot_outlier_golden(golden):
     assert np.all(np.abs(got) == m / np.sqrt(n))
 
 
-@pytest.mark.parametrize("k,block", [(512, 128), (256, 0), (384, 128)])
+@pytest.mark.parametrize("k,block", [(512, 128), (256, 0), (384, 128), (256, 16), (256, 32)])
 def test_onehot_spreads_to_block(k, block):
     """Each one-hot input maps to a row of Q: +-1/sqrt(B) inside its block, 0 outside."""
     rng = np.random.default_rng(3)
