@@ -19,6 +19,9 @@ Sources on the pages:
   6-bit and 8-bit round-to-nearest, no calibration data) and "SpinQuant
   (learned rotations + W4A4KV4)", field "Activation scheme" (also reported
   at W4A8).
+* Per-group asymmetric INT4 for activations and weights: "SpinQuant (learned
+  rotations + W4A4KV4)", field "Activation scheme" (per-group INT4
+  asymmetric quantization of weights, activations and KV cache).
 * KV cache at 4 bits, asymmetric: "SpinQuant (learned rotations + W4A4KV4)",
   field "Activation scheme" (per-group INT4 asymmetric for the KV cache), and
   "QuaRot (rotation-based outlier removal, W4A4KV4)", field "Activation scheme"
@@ -42,6 +45,9 @@ Readings where the pages are silent (each also listed in the design notes):
   pages give no scale rule; this is the shared-exponent rule of the OCP
   Microscaling formats.  amax_b = 0 -> scale code 0 (2^-127), e = 0.  There
   is no per-tensor scale.
+* Per-group asymmetric INT4 of X / W: the KV4 rule below on every group of
+  128 consecutive channels of a row (the pages give no group width; 128 is
+  the rotation block).
 * KV4 per (batch, head, token) vector of head_dim after the Hadamard:
   z = min, s = (max - min)/15, z_h = fp16(z), s_h = fp16(s);
   q = clamp(rint((x - z_h)/s_h), 0, 15); s_h = 0 -> q = 0.
@@ -231,6 +237,28 @@ def kv4_vectors(xr):
     tie = _near_half(v) & (sh > 0)
     tie_sz = _fp16_tie(lo) | (_fp16_tie(s) & (s > 0))
     return q, s_h, z_h, tie, tie_sz
+
+
+def asym_int4_groups(xr, group=128):
+    """Per-group asymmetric INT4 along the last axis of rotated fp64 xr [rows, K]:
+    each group of `group` channels is quantized by the KV4 rule (z = min,
+    s = (max - min)/15 as fp16, q = clamp(rint((x - z_h)/s_h), 0, 15)).
+
+    Returns (q int64 [rows, K], s_h [rows, K/group], z_h [rows, K/group],
+    tie bool [rows, K], tie_sz bool [rows, K/group]).
+    """
+    xr = np.asarray(xr, dtype=np.float64)
+    rows, k = xr.shape
+    if k % group:
+        raise ValueError("K must be a multiple of the group")
+    q, s_h, z_h, tie, tie_sz = kv4_vectors(xr.reshape(rows, k // group, group))
+    return q.reshape(rows, k), s_h, z_h, tie.reshape(rows, k), tie_sz
+
+
+def asym_int4_dequant(q, s_h, z_h, group=128):
+    rows, k = np.shape(q)
+    qg = np.asarray(q, dtype=np.float64).reshape(rows, k // group, group)
+    return (qg * np.asarray(s_h)[..., None] + np.asarray(z_h)[..., None]).reshape(rows, k)
 
 
 def kv4_dequant(q, s_h, z_h):

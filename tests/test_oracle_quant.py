@@ -295,3 +295,45 @@ def test_more_bits_lower_error():
         q, s, _ = quant.int_sym_rows(x, bits)
         errs.append(np.linalg.norm(x - quant.int4_dequant(q, s)) / np.linalg.norm(x))
     assert errs[0] > 3.5 * errs[1] > 3.5 * 3.5 * errs[2]
+
+
+# ---------------------------------------------------------------- per-group asymmetric INT4
+def test_asym_int4_groups_bruteforce_and_bound():
+    """Each group of 128: codes are the nearest of 0..15 to (x - z_h)/s_h (argmin
+    search), the group's min maps to 0 and max to 15, |x - deq| <= s_h/2 (+ the
+    fp16 rounding of s and z)."""
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((6, 512))
+    x[:, 130] *= 25
+    q, s_h, z_h, tie, tie_sz = quant.asym_int4_groups(x)
+    assert q.shape == x.shape and s_h.shape == (6, 4) and q.min() >= 0 and q.max() <= 15
+    for r in range(6):
+        for g in range(4):
+            sl = slice(128 * g, 128 * (g + 1))
+            d = np.abs((x[r, sl, None] - z_h[r, g]) - np.arange(16) * s_h[r, g])
+            best = d.min(axis=-1, keepdims=True)
+            ok = (d[np.arange(128), q[r, sl]] == best[:, 0]) | tie[r, sl]
+            assert ok.all()
+            assert q[r, sl][np.argmin(x[r, sl])] in (0, 1) and q[r, sl][np.argmax(x[r, sl])] in (14, 15)
+    err = np.abs(x - quant.asym_int4_dequant(q, s_h, z_h))
+    bound = np.repeat(s_h, 128, axis=1) * 0.5 + np.repeat(np.abs(z_h) + 15 * s_h, 128, axis=1) * 2.0 ** -10
+    assert np.all(err <= bound)
+
+
+def test_asym_int4_groups_hand_worked():
+    """A group holding 0, 0.5, ..., 7.5 (eight times): z = min = 0, s = (7.5 - 0)/15
+    = 0.5 exactly, so the codes are x / 0.5 = 0..15 with no rounding."""
+    g = np.tile(np.arange(16) * 0.5, 8)            # 128 values in [0, 7.5], step 0.5
+    q, s_h, z_h, tie, _ = quant.asym_int4_groups(g[None, :])
+    assert s_h[0, 0] == 0.5 and z_h[0, 0] == 0.0
+    assert np.array_equal(q[0], np.tile(np.arange(16), 8)) and not tie.any()
+
+
+def test_asym_int4_groups_equal_kv4_per_group():
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((3, 256))
+    q, s_h, z_h, _, _ = quant.asym_int4_groups(x)
+    for g in range(2):
+        qg, sg, zg, _, _ = quant.kv4_vectors(x[:, 128 * g:128 * (g + 1)])
+        assert np.array_equal(q[:, 128 * g:128 * (g + 1)], qg)
+        assert np.array_equal(s_h[:, g], sg) and np.array_equal(z_h[:, g], zg)
