@@ -85,7 +85,7 @@ def code_bytes(fmt, rows, k):
     """Bytes of codes and scales the rotate kernel writes for `rows` rows of K."""
     return {"int4": rows * k // 2 + rows * 4, "nvfp4": rows * k // 2 + rows * (k // 16),
             "mxfp4": rows * k // 2 + rows * (k // 32), "int8": rows * k + rows * 4,
-            "int6": rows * k + rows * 4}[fmt]
+            "int6": rows * k + rows * 4, "int4_asym": rows * k // 2 + rows * (k // 128) * 4}[fmt]
 
 
 def source_fingerprint(files):
@@ -160,7 +160,7 @@ class Workload:
             self.x = syn.activations(name, device=device, seed_offset=seed_offset)
             w = syn.weights(name, device=device)
             self.signs = syn.workload_signs(name).to(device)
-            self.wq = rq.prepare_weights(w, self.signs, self.block, self.wfmt)
+            self.wq = None if self.fmt == "int4_asym" else rq.prepare_weights(w, self.signs, self.block, self.wfmt)
             del w
             m, k, n = c["M"], c["K"], c["N"]
             self.xq_out = rq._alloc_quant_outputs(m, k, rq._fmt(self.fmt), device)
@@ -198,11 +198,11 @@ class Workload:
             return "rotate_kernel<KV4>"
         if self.fmt == "nvfp4" and self.nvfp4_one_pass():
             return "rotate_nvfp4_resident_kernel"
-        mode = "INT8, " if self.fmt in ("int8", "int6") else ""
-        return "rotate_kernel<%s%s>" % (mode, "full width" if self.block == 0 else "128-blocks")
+        mode = {"int8": "INT8, ", "int6": "INT8, ", "int4_asym": "ASYM4, "}.get(self.fmt, "")
+        return "rotate_kernel<%s%s>" % (mode, "full width" if self.block == 0 else "%d-blocks" % self.block)
 
     def gemm_launches(self):
-        return 0 if (self.kv or self.kvdec) else 1
+        return 0 if (self.kv or self.kvdec or self.fmt == "int4_asym") else 1
 
     def quant(self):
         rq = self.rq
@@ -218,7 +218,7 @@ class Workload:
                                   out=self.xq_out, workspace=self.ws)
 
     def gemm(self, xq):
-        if self.kv or self.kvdec:
+        if self.kv or self.kvdec or self.fmt == "int4_asym":
             return None
         if self.fmt in ("int8", "int6"):
             return self.rq.int_gemm(xq, self.fmt, self.wq, self.wfmt, self.y_dtype, y=self.y)
@@ -227,6 +227,8 @@ class Workload:
     def result(self):
         if self.kvdec:
             return self.out
+        if getattr(self, "fmt", None) == "int4_asym":
+            return self.xq_out[0]
         return self.outs[0][0] if self.kv else self.y
 
 
@@ -337,6 +339,16 @@ def oracle_sample(name, rows):
         dt = time.perf_counter() - t0
         nbytes = x.shape[0] * (128 * 2 + 64 + 4)
         return nbytes / dt / 1e9, None, dt, "%d head_dim vectors (1 x 4 heads x %d tokens)" % (x.shape[0], rows)
+    if c["fmt"] == "int4_asym":
+        # the quantizer alone (no GEMM consumes these codes)
+        x = syn.activations(name, rows=rows).to(torch.float64).numpy()
+        s = syn.workload_signs(name).numpy()
+        t0 = time.perf_counter()
+        q, _, _, _, _ = oquant.asym_int4_groups(ohad.rotate(x, s, c["block"]))
+        oquant.pack_nibbles(q)
+        dt = time.perf_counter() - t0
+        return ((rows * c["K"] * 2 + code_bytes("int4_asym", rows, c["K"])) / dt / 1e9, None, dt,
+                "%d of %d rows of X" % (rows, c["M"]))
     x = syn.activations(name, rows=rows).to(torch.float64).numpy()
     w = syn.weights(name).to(torch.float64).numpy()
     s = syn.workload_signs(name).numpy()
@@ -394,7 +406,8 @@ def blas_threads():
 
 def sample_rows(name):
     return {"tiny_int4": 64, "q_proj_int4": 512, "down_proj_int4": 256, "q_proj_nvfp4": 256, "kv4": 4096,
-            "q_proj_mxfp4": 256, "kv4_decode": 1024, "q_proj_w4a8": 512, "q_proj_w8a8": 512}[name]
+            "q_proj_mxfp4": 256, "kv4_decode": 1024, "q_proj_w4a8": 512, "q_proj_w8a8": 512,
+            "q_proj_nvfp4_b16": 256, "q_proj_mxfp4_b32": 256, "q_proj_int4_asym": 2048}[name]
 
 
 # --------------------------------------------------------------------------- main

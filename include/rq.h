@@ -65,7 +65,8 @@ typedef enum {
   RQ_NVFP4 = 1, /* E2M1, one E4M3 scale per 16 values, fp32 per-tensor scale */
   RQ_MXFP4 = 2, /* E2M1, one E8M0 (power-of-two) scale per 32 values */
   RQ_INT8 = 3,  /* symmetric 8-bit, one int8 code per byte, one fp32 scale per row */
-  RQ_INT6 = 4   /* symmetric 6-bit (codes in [-31, 31]), one int8 byte each, one fp32 scale per row */
+  RQ_INT6 = 4,  /* symmetric 6-bit (codes in [-31, 31]), one int8 byte each, one fp32 scale per row */
+  RQ_INT4_ASYM = 5 /* asymmetric 4-bit per group of 128 along K: fp16 (scale, zero) per group */
 } rq_format;
 
 typedef enum {
@@ -104,8 +105,10 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *  K          channels; a multiple of 128, at most 32768.
  *  signs_dev  int8 [K], 16-byte aligned, each +1 or -1 (the random sign diagonal;
  *             any other value is read as -1 if negative and +1 otherwise).
- *  block      128 for 128-wide blocks, or 0 for a full-width rotation (then K
- *             must be a power of two in [256, 4096]; INT4, INT6 and INT8 only).
+ *  block      128, 32 or 16 for block-diagonal rotations (32 and 16: blocks
+ *             sized to the MXFP4 / NVFP4 scale groups, "Gotchas", "Block size
+ *             matters"), or 0 for a full-width rotation (then K must be a power
+ *             of two in [256, 4096]; INT4, INT6 and INT8 only).
  *  fmt        RQ_INT4:
  *               codes_dev  uint8 [M, K/2], scales_dev float [M]:
  *               s = amax/7 (fp32, amax = max |x~| of the row); q = rint(x~/s).
@@ -131,6 +134,14 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *               codes_dev  int8 [M, K], scales_dev float [M]:
  *               s = amax/qmax with qmax = 127 / 31; q = rint(x~/s).  gscale_dev
  *               and workspace_dev are unused (may be NULL).
+ *             RQ_INT4_ASYM (per-group asymmetric INT4, "SpinQuant", field
+ *             "Activation scheme"; block 16, 32 or 128):
+ *               codes_dev  uint8 [M, K/2], unsigned nibbles q in [0, 15],
+ *               scales_dev fp16 pairs [M, K/128][2] = (s_h, z_h) per group of
+ *               128 channels (4-byte aligned): z = min, s = (max - min)/15 of
+ *               the group's x~, s_h = fp16(s), z_h = fp16(z);
+ *               q = clamp(rint((x~ - z_h)/s_h), 0, 15) (s_h = 0 gives q = 0);
+ *               x^ = z_h + s_h q.  No GEMM in this library consumes these codes.
  *  workspace_dev  rq_workspace_bytes(fmt) bytes (may be NULL when that is 0).
  *  codes_dev and scales_dev 16-byte aligned (8 for NVFP4 scales).
  * Values that sit within a few fp32 ulps of a rounding boundary may round

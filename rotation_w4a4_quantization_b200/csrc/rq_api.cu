@@ -97,7 +97,7 @@ RotCfg rotate_config(int64_t K, bool full, int mode) {
   return c;
 }
 
-template <int MODE, int NBF>
+template <int MODE, int NBF, int LOGB = 7>
 rq_status launch_rotate(RotParams p, cudaStream_t st) {
   const RotCfg c = rotate_config(p.K, NBF != 0, MODE);
   if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
@@ -108,14 +108,20 @@ rq_status launch_rotate(RotParams p, cudaStream_t st) {
   p.num_tiles = (p.rows + c.RPS - 1) / c.RPS;
   const int64_t ctas = (p.num_tiles + c.GPC - 1) / c.GPC;
   const int64_t grid = ctas < num_sms_of_current_device() ? ctas : num_sms_of_current_device();
-  if (!ensure_smem(reinterpret_cast<const void*>(rotate_kernel<MODE, NBF>))) return RQ_ERR_CUDA;
-  rotate_kernel<MODE, NBF><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_kernel<MODE, NBF, LOGB>))) return RQ_ERR_CUDA;
+  rotate_kernel<MODE, NBF, LOGB><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
   return last_launch_status();
 }
 
+// Block-diagonal rotation: blocks of 128, or of 16 / 32 (p.logb 4 / 5, the
+// format-sized blocks; not for KV4, whose block is the head).
 template <int MODE>
 rq_status launch_block(RotParams p, cudaStream_t st) {
-  return launch_rotate<MODE, 0>(p, st);
+  if constexpr (MODE != kModeKv4) {
+    if (p.logb == 4) return launch_rotate<MODE, 0, 4>(p, st);
+    if (p.logb == 5) return launch_rotate<MODE, 0, 5>(p, st);
+  }
+  return launch_rotate<MODE, 0, 7>(p, st);
 }
 
 // K = 4096: the 64 x 64 two-pass kernel, two CTAs of four row teams per SM.
@@ -144,7 +150,8 @@ rq_status launch_full(RotParams p, cudaStream_t st) {
 // Dynamic NVFP4 in one pass (rotate_nvfp4_resident_kernel): every CTA keeps its
 // rows in shared memory; needs all CTAs resident (cooperative launch).  Returns
 // RQ_ERR_UNSUPPORTED_SHAPE (nothing launched) when the rows do not fit.
-rq_status launch_nvfp4_resident(RotParams p, cudaStream_t st) {
+template <int LOGB>
+rq_status launch_nvfp4_resident_b(RotParams p, cudaStream_t st) {
   int dev = 0, coop = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return RQ_ERR_CUDA;
   if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop)
@@ -154,9 +161,9 @@ rq_status launch_nvfp4_resident(RotParams p, cudaStream_t st) {
   const size_t smem = (size_t)rpc * p.K * 2 + (size_t)p.nb * 64 * 4 + 32;
   if (smem > kSmemBudget) return RQ_ERR_UNSUPPORTED_SHAPE;
   const int grid = (int)((p.rows + rpc - 1) / rpc);
-  if (!ensure_smem(reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel))) return RQ_ERR_CUDA;
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel<LOGB>))) return RQ_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_nvfp4_resident_kernel, 384, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_nvfp4_resident_kernel<LOGB>, 384, smem) !=
           cudaSuccess ||
       per_sm < 1 || grid > per_sm * sms)
     return RQ_ERR_UNSUPPORTED_SHAPE;
@@ -173,9 +180,15 @@ rq_status launch_nvfp4_resident(RotParams p, cudaStream_t st) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel), args) != cudaSuccess)
+  if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel<LOGB>), args) != cudaSuccess)
     return RQ_ERR_CUDA;
   return RQ_OK;
+}
+
+rq_status launch_nvfp4_resident(RotParams p, cudaStream_t st) {
+  if (p.logb == 4) return launch_nvfp4_resident_b<4>(p, st);
+  if (p.logb == 5) return launch_nvfp4_resident_b<5>(p, st);
+  return launch_nvfp4_resident_b<7>(p, st);
 }
 
 // Common checks of the X / K / signs / block arguments.
@@ -184,10 +197,17 @@ rq_status check_rotation_args(const void* X, int64_t M, int64_t K, int64_t ldx, 
   if (M > 0 && (!X || !signs)) return RQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || ldx < K) return RQ_ERR_INVALID_ARG;
   if (K % 128 != 0 || K > kMaxKBlock) return RQ_ERR_UNSUPPORTED_SHAPE;
-  if (block != 0 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (block != 0 && block != 16 && block != 32 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (block == 0 && !(is_pow2(K) && K >= 256 && K <= 4096)) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(X, 16) || (ldx * 2) % 16 != 0 || !aligned(signs, 16)) return RQ_ERR_ALIGNMENT;
   return RQ_OK;
+}
+
+// Block-diagonal rotation size (16, 32 or 128; 0 = full width leaves 128).
+void set_block(RotParams& p, int block) {
+  const int b = (block == 16 || block == 32) ? block : 128;
+  p.logb = b == 16 ? 4 : (b == 32 ? 5 : 7);
+  p.cblk = (float)(1.0 / std::sqrt((double)b));
 }
 
 RotParams matrix_params(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* signs) {
@@ -205,6 +225,7 @@ RotParams matrix_params(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.contiguous = (ldx == K) ? 1 : 0;
   p.signs = signs;
   p.cfull = (float)(1.0 / std::sqrt((double)K));
+  set_block(p, 128);
   return p;
 }
 
@@ -213,11 +234,12 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
                                void* workspace, cudaStream_t st) {
   rq_status s = check_rotation_args(X, M, K, ldx, signs, block);
   if (s != RQ_OK) return s;
-  if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4 && fmt != RQ_INT8 && fmt != RQ_INT6)
+  if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4 && fmt != RQ_INT8 && fmt != RQ_INT6 &&
+      fmt != RQ_INT4_ASYM)
     return RQ_ERR_INVALID_ARG;
   if (gmode != RQ_SCALE_DYNAMIC && gmode != RQ_SCALE_STATIC) return RQ_ERR_INVALID_ARG;
   const bool int_fmt = fmt == RQ_INT4 || fmt == RQ_INT8 || fmt == RQ_INT6;
-  if (!int_fmt && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (!int_fmt && block == 0) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return RQ_OK;
   if (!codes || !scales) return RQ_ERR_INVALID_ARG;
   if (!aligned(codes, 16)) return RQ_ERR_ALIGNMENT;
@@ -232,11 +254,16 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
   if (M == 0) return RQ_OK;
 
   RotParams p = matrix_params(X, M, K, ldx, signs);
+  set_block(p, block);
   p.codes = codes;
   if (fmt == RQ_INT4) {
     p.scales_f32 = static_cast<float*>(scales);
     if (block == 0) return launch_full<kModeInt4>(p, st);
     return launch_block<kModeInt4>(p, st);
+  }
+  if (fmt == RQ_INT4_ASYM) {
+    p.kv_scale = static_cast<__half*>(scales);
+    return launch_block<kModeAsym4>(p, st);
   }
   if (fmt == RQ_INT8 || fmt == RQ_INT6) {
     p.scales_f32 = static_cast<float*>(scales);
@@ -368,6 +395,7 @@ rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t ldx, co
   if (!out_dev) return RQ_ERR_INVALID_ARG;
   if (!aligned(out_dev, 16) || ldo % 4 != 0) return RQ_ERR_ALIGNMENT;
   RotParams p = matrix_params(X_dev, M, K, ldx, signs_dev);
+  set_block(p, block);
   p.out_f32 = out_dev;
   p.ldo = ldo;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -408,6 +436,7 @@ rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H, int64_
   p.codes = codes_dev;
   p.kv_scale = static_cast<__half*>(scale_dev);
   p.kv_zero = static_cast<__half*>(zero_dev);
+  set_block(p, 128);
   return launch_block<kModeKv4>(p, static_cast<cudaStream_t>(stream));
 }
 

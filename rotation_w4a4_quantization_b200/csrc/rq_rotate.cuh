@@ -53,7 +53,8 @@ namespace rq {
 
 enum RotMode : int {
   kModeInt4 = 0, kModeNvfp4 = 1, kModeF32 = 2, kModeAmax = 3, kModeKv4 = 4, kModeMxfp4 = 5,
-  kModeInt8 = 6  // 6- or 8-bit symmetric codes, one per byte (qmax 31 or 127)
+  kModeInt8 = 6,  // 6- or 8-bit symmetric codes, one per byte (qmax 31 or 127)
+  kModeAsym4 = 7  // asymmetric 4-bit per group of 128 along K: fp16 (scale, zero) per group
 };
 
 struct RotParams {
@@ -70,7 +71,7 @@ struct RotParams {
   float* scales_f32;   // INT4 / INT6 / INT8: [rows]
   float qmax;          // INT6 / INT8: 31 or 127
   uint8_t* scales_e4m3;// NVFP4: [rows, K/16]; MXFP4: E8M0 [rows, K/32]
-  __half* kv_scale;    // KV4: [rows]
+  __half* kv_scale;    // KV4: [rows]; ASYM4: (scale, zero) pairs [rows, K/128]
   __half* kv_zero;     // KV4: [rows]
   float* out_f32;      // F32: [rows, ldo]
   int64_t ldo;
@@ -79,6 +80,8 @@ struct RotParams {
   unsigned* amax_word; // NVFP4 dynamic: max |X~| as fp32 bits (AMAX writes, NVFP4 reads)
   int nvfp4_dynamic;   // 1: g from amax_word, 0: g from g_in
   float cfull;         // 1/sqrt(K) for full-width rotations (rounded once from the exact value)
+  int logb;            // block-diagonal rotations: log2 of the block, 7 (128), 5 (32) or 4 (16)
+  float cblk;          // 1/sqrt(2^logb), rounded once
   // geometry (host-chosen)
   int G;               // warps per group
   int RPS;             // rows per stage
@@ -194,6 +197,51 @@ __device__ __forceinline__ void fwht128(float (&v)[128]) {
       }
     }
   }
+}
+
+// The same transform over independent blocks of 2^logb consecutive values
+// (logb = 4 or 5: the format-sized blocks of 16 / 32; 7 is fwht128).
+template <int LOGB>
+__device__ __forceinline__ void fwht_blocks(float (&v)[128]) {
+#pragma unroll
+  for (int i = 0; i < 128; i += 2) {
+    const float a = v[i], b = v[i + 1];
+    v[i] = a + b;
+    v[i + 1] = a - b;
+  }
+#pragma unroll
+  for (int h = 2; h < (1 << LOGB); h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 128; i += 2) {
+      if ((i & h) == 0) {
+        const float2 a = make_float2(v[i], v[i + 1]);
+        const float2 b = make_float2(v[i + h], v[i + h + 1]);
+        const float2 s = __fadd2_rn(a, b);
+        const float2 d = __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+        v[i] = s.x;
+        v[i + 1] = s.y;
+        v[i + h] = d.x;
+        v[i + h + 1] = d.y;
+      }
+    }
+  }
+}
+
+template <int LOGB>
+__device__ __forceinline__ void fwht_block_diag(float (&v)[128]) {
+  if constexpr (LOGB == 7)
+    fwht128(v);
+  else
+    fwht_blocks<LOGB>(v);
+}
+
+// XOR key of a thread's chunk order for blocks of 2^logb: only chunk-index
+// bits inside a block may be permuted (the transform then turns the
+// permutation into the sign pattern chi); with 16- or 32-wide blocks that
+// leaves 1 or 2 bits, so the shared-memory reads of those modes keep 4- or
+// 2-way bank conflicts.
+__device__ __forceinline__ int chunk_key(int lane, int logb) {
+  return lane & ((1 << (logb - 3)) - 1) & 7;
 }
 
 // chi for 8-element chunk `chunk` of a thread with XOR key m: +-1 as a sign bit.
@@ -624,10 +672,11 @@ __device__ __forceinline__ void full_store_int8(const float (&y)[2][NB][64 / NB]
 }
 
 // ---------------------------------------------------------------------------
-// The kernel.  NBF = 0: block-diagonal (B = 128), any mode.  NBF = 2..32:
-// full-width rotation of K = 128*NBF (INT4, INT6/INT8 and F32 modes).
+// The kernel.  NBF = 0: block-diagonal with blocks of 2^LOGB (128, 32 or 16),
+// any mode.  NBF = 2..32: full-width rotation of K = 128*NBF (INT4, INT6/INT8
+// and F32 modes).
 // ---------------------------------------------------------------------------
-template <int MODE, int NBF>
+template <int MODE, int NBF, int LOGB = 7>
 __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_kernel(const RotParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -653,9 +702,9 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
     b = wig * 32 + lane;
     active = b < nb;
   }
-  const int m = lane & 7;
+  const int m = chunk_key(lane, NBF ? 7 : LOGB);
   const bool producer = (wig == 0 && lane == 0);
-  const float c = 0.08838834764831845f;  // 1/sqrt(128), rounded once
+  const float c = (NBF || LOGB == 7) ? 0.08838834764831845f : p.cblk;  // 1/sqrt(block), rounded once
   const int64_t TG = (int64_t)gridDim.x * p.GPC;
   const int64_t gg = (int64_t)blockIdx.x * p.GPC + grp;
 
@@ -716,7 +765,7 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
           issue_tile_load(p, nt, stage, &full[st]);
         }
       }
-      fwht128(v);
+      fwht_block_diag<LOGB>(v);
       if (MODE == kModeInt4) {
         const float a = valid ? absmax128(v) * c : 0.f;
         const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
@@ -745,6 +794,11 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
         if (valid) amax_acc = fmaxf(amax_acc, absmax128(v) * c);
       } else if (MODE == kModeKv4) {
         if (valid) quant_kv4_store(v, c, m, p.codes + row * 64, p.kv_scale + row, p.kv_zero + row);
+      } else if (MODE == kModeAsym4) {
+        if (valid) {
+          __half* sz = p.kv_scale + 2 * (row * nb + b);
+          quant_kv4_store(v, c, m, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
+        }
       }
     } else {
       constexpr int NB = NBF ? NBF : 1;
@@ -991,6 +1045,7 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
 // p.amax_word[0] gathers the max, p.amax_word[1] counts arrivals; both are
 // zeroed by the host before the launch.
 // ---------------------------------------------------------------------------
+template <int LOGB>
 __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const RotParams p, int rows_per_cta) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int nb = p.nb;
@@ -1003,8 +1058,8 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
   unsigned* cta_max = reinterpret_cast<unsigned*>(bar + 1);
   int* flag = reinterpret_cast<int*>(cta_max + 1);
   const int tid = threadIdx.x;
-  const int m = tid & 7;
-  const float c = 0.08838834764831845f;  // 1/sqrt(128), rounded once
+  const int m = chunk_key(tid, LOGB);
+  const float c = LOGB == 7 ? 0.08838834764831845f : p.cblk;  // 1/sqrt(block), rounded once
 
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -1035,7 +1090,7 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
       const int r = u / nb, b = u - r * nb;
       float v[128];
       load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
-      fwht128(v);
+      fwht_block_diag<LOGB>(v);
       amax = fmaxf(amax, absmax128(v) * c);
     }
   }
@@ -1075,7 +1130,7 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
     const int64_t row = r0 + r;
     float v[128];
     load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
-    fwht128(v);
+    fwht_block_diag<LOGB>(v);
     quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
                       p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
   }

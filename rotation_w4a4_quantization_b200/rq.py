@@ -15,7 +15,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librq.so")
 
-RQ_INT4, RQ_NVFP4, RQ_MXFP4, RQ_INT8, RQ_INT6 = 0, 1, 2, 3, 4
+RQ_INT4, RQ_NVFP4, RQ_MXFP4, RQ_INT8, RQ_INT6, RQ_INT4_ASYM = 0, 1, 2, 3, 4, 5
 RQ_OUT_F32, RQ_OUT_BF16, RQ_OUT_I32_ACC = 0, 1, 2
 RQ_SCALE_DYNAMIC, RQ_SCALE_STATIC = 0, 1
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3: "RQ_ERR_ALIGNMENT",
@@ -83,7 +83,8 @@ def _stream(t=None):
 
 def _fmt(fmt):
     if isinstance(fmt, str):
-        return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4, "mxfp4": RQ_MXFP4, "int8": RQ_INT8, "int6": RQ_INT6}[fmt]
+        return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4, "mxfp4": RQ_MXFP4, "int8": RQ_INT8, "int6": RQ_INT6,
+                "int4_asym": RQ_INT4_ASYM}[fmt]
     return int(fmt)
 
 
@@ -106,6 +107,8 @@ def _alloc_quant_outputs(rows, k, fmt, device):
         return (torch.empty((rows, k), dtype=torch.int8, device=device),
                 torch.empty((rows,), dtype=torch.float32, device=device))
     codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=device)
+    if fmt == RQ_INT4_ASYM:  # fp16 (scale, zero) per group of 128
+        return codes, torch.empty((rows, k // 128, 2), dtype=torch.float16, device=device)
     if fmt == RQ_INT4:
         scales = torch.empty((rows,), dtype=torch.float32, device=device)
     elif fmt == RQ_NVFP4:
@@ -122,6 +125,7 @@ def rotate_quantize(x, signs, block=128, fmt="int4", gmode="dynamic", gscale=Non
     NVFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/16] (E4M3), gscale fp32 [1].
     MXFP4: codes uint8 [M, K/2] (E2M1), scales uint8 [M, K/32] (E8M0), gscale None.
     INT8 / INT6: codes int8 [M, K] (one code per byte), scales fp32 [M], gscale None.
+    INT4_ASYM: codes uint8 [M, K/2] (unsigned nibbles), scales fp16 [M, K/128, 2] = (scale, zero).
     """
     _require_cuda(x, signs)
     f = _fmt(fmt)

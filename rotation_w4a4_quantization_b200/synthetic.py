@@ -44,6 +44,11 @@ WORKLOADS = {
     # 8-bit activations: W4A8 (4-bit weights) and W8A8, q_proj shapes and recipe
     "q_proj_w4a8": dict(index=8, M=2048, K=4096, N=4096, block=0, fmt="int8", wfmt="int4"),
     "q_proj_w8a8": dict(index=9, M=2048, K=4096, N=4096, block=0, fmt="int8", wfmt="int8"),
+    # format-sized block rotations: one block per NVFP4 (16) or MXFP4 (32) scale group
+    "q_proj_nvfp4_b16": dict(index=10, M=2048, K=4096, N=4096, block=16, fmt="nvfp4"),
+    "q_proj_mxfp4_b32": dict(index=11, M=2048, K=4096, N=4096, block=32, fmt="mxfp4"),
+    # per-group (128) asymmetric INT4 of the activations (quantizer only: no GEMM consumes it)
+    "q_proj_int4_asym": dict(index=12, M=2048, K=4096, N=4096, block=128, fmt="int4_asym"),
 }
 
 
@@ -74,7 +79,7 @@ def activations(name, rows=None, device="cpu", seed_offset=0):
     x = torch.randn((m, k), generator=g, device=device, dtype=torch.float32)
     if name == "tiny_int4":
         x[:, [3, 77, 200, 411]] *= 50.0
-    elif name in ("q_proj_int4", "q_proj_nvfp4", "q_proj_mxfp4", "q_proj_w4a8", "q_proj_w8a8"):
+    elif name.startswith("q_proj"):
         gp = _gen(3000 + w["index"], "cpu")
         ch = torch.randperm(k, generator=gp)[:8]
         mult = 20.0 + 40.0 * torch.rand((8,), generator=gp, dtype=torch.float64)
