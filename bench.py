@@ -59,25 +59,32 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
 
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
-# ncu captures summarised in profiles/, with a fingerprint of the kernel sources
-# they were taken on; a number is reported only while those sources are
-# unchanged.  kv4 was captured on a quarter of one tensor and is scaled by the
-# vectors processed.
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
 ATTN_SOURCES = ("rq_common.cuh", "rq_attn.cuh")
-_ROT, _GEM = "96ccf4968826d44e", "c6e805e14224d165"
+_ROT, _GEM, _ATT = "72f58a0c7fdcb2d8", "6dd5a8abd00b6055", "ef7bba0ae5109f9f"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
+# ncu capture of the kernel (summarised in profiles/), with the fingerprint of
+# the sources it was taken on (reported as null once they change).  kv4 and
+# kv4_decode were captured at B = 4 and are scaled to the bench's B = 16 (traffic
+# grows with the vectors processed); kv4_decode is the partial + combine pair.
 TRAFFIC = {
-    ("hadamard_quant", "q_proj_int4"): (16847104, _ROT),
-    ("hadamard_quant", "down_proj_int4"): (100728576 + 5582336, _ROT),
-    ("hadamard_quant", "kv4"): ((134419968 + 12322560) * 4, _ROT),
-    ("hadamard_quant", "q_proj_nvfp4"): (16830464, _ROT),
+    ("hadamard_quant", "q_proj_int4"): (16807168, _ROT),
+    ("hadamard_quant", "down_proj_int4"): (105399296, _ROT),
+    ("hadamard_quant", "kv4"): (150622720 * 4, _ROT),
+    ("hadamard_quant", "q_proj_nvfp4"): (16830720, _ROT),
     ("hadamard_quant", "q_proj_mxfp4"): (16831744, _ROT),
-    ("gemm", "q_proj_int4"): (12652288, _GEM),
-    ("gemm", "down_proj_int4"): (50722816 + 10223616, _GEM),
-    ("gemm", "q_proj_nvfp4"): (14189056, _GEM),
+    ("hadamard_quant", "q_proj_w4a8"): (16806400, _ROT),
+    ("hadamard_quant", "q_proj_w8a8"): (16806400, _ROT),
+    ("hadamard_quant", "q_proj_nvfp4_b16"): (16824320, _ROT),
+    ("hadamard_quant", "q_proj_int4_asym"): (16840960, _ROT),
+    ("hadamard_quant", "kv4_decode"): (72350976 * 4, _ATT),
+    ("gemm", "q_proj_int4"): (12650240, _GEM),
+    ("gemm", "down_proj_int4"): (62656512, _GEM),
+    ("gemm", "q_proj_nvfp4"): (14189312, _GEM),
     ("gemm", "q_proj_mxfp4"): (13400320, _GEM),
+    ("gemm", "q_proj_w4a8"): (16844032, _GEM),
+    ("gemm", "q_proj_w8a8"): (25229568, _GEM),
 }
 
 
