@@ -12,9 +12,11 @@ For the KV workload a step is rq_kv_rotate_quantize on K and on V.
 The metric is the pair "fused Hadamard+quant GB/s vs HBM peak; W4A4 GEMM TOPS
 vs tensor peak": `value` is the fused rotate+quantize throughput in GB/s
 (algorithmic bytes / device time), and the `gemm` object carries the GEMM's
-TOPS.  Times are CUDA events on the launching stream, L2 is flushed between
-steps, and for N > 1 each rank runs its own batch (weak scaling, no data-path
-collective) and the time is the max over ranks.
+TOPS.  Times are CUDA events on the launching stream around K steps run back
+to back; the inputs cycle through distinct sets that together exceed the L2
+(no flush is needed), the per-kernel figures come from K launches of each
+kernel alone over the same inputs, and for N > 1 each rank runs its own batch
+(weak scaling, no data-path collective) and the time is the max over ranks.
 """
 
 import argparse
@@ -33,14 +35,15 @@ if ROOT not in sys.path:
 from rotation_w4a4_quantization_b200 import synthetic as syn  # noqa: E402
 
 METRIC = "fused Hadamard+quant GB/s vs HBM peak; W4A4 GEMM TOPS vs tensor peak"
-L2_FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20      # B200 L2 (nominal)
+RING_MAX = 16
 DEFAULT_WORKLOAD = "q_proj_int4"
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -95,6 +98,32 @@ def code_bytes(fmt, rows, k):
             "int6": rows * k + rows * 4, "int4_asym": rows * k // 2 + rows * (k // 128) * 4}[fmt]
 
 
+def ring_slots(name):
+    """How many distinct input sets the timed steps cycle through so that a set
+    is out of L2 when it comes round again: the step's distinct inputs (X and
+    the weight codes) times the slot count cover at least twice the L2.  The KV
+    workloads' inputs alone are several times the L2."""
+    c = syn.WORKLOADS[name]
+    if name in ("kv4", "kv4_decode"):
+        return 1
+    per = c["M"] * c["K"] * 2
+    if c["fmt"] != "int4_asym":
+        per += code_bytes(c.get("wfmt", c["fmt"]), c["N"], c["K"])
+    return int(min(RING_MAX, max(1, -(-2 * L2_BYTES // per))))
+
+
+def ring_bytes(name):
+    c = syn.WORKLOADS[name]
+    if name == "kv4":
+        return 2 * c["B"] * c["H"] * c["S"] * c["D"] * 2
+    if name == "kv4_decode":
+        return 2 * c["B"] * c["H"] * c["S"] * 68
+    per = c["M"] * c["K"] * 2
+    if c["fmt"] != "int4_asym":
+        per += code_bytes(c.get("wfmt", c["fmt"]), c["N"], c["K"])
+    return ring_slots(name) * per
+
+
 def source_fingerprint(files):
     import hashlib
     m = hashlib.sha256()
@@ -126,6 +155,7 @@ class Workload:
         self.y_dtype = y_dtype
         self.kv = name == "kv4"
         self.kvdec = name == "kv4_decode"
+        self.R = 1
         if self.kvdec:
             c = self.cfg
             self.signs = syn.workload_signs(name).to(device)
@@ -164,17 +194,28 @@ class Workload:
             self.fmt = c["fmt"]
             self.wfmt = c.get("wfmt", self.fmt)
             self.block = c["block"]
-            self.x = syn.activations(name, device=device, seed_offset=seed_offset)
+            self.R = ring_slots(name)
+            # R distinct input sets (activations from their own seeds, copies of the
+            # weight codes) and outputs, cycled step to step
+            self.xs = [syn.activations(name, device=device, seed_offset=seed_offset * RING_MAX + r)
+                       for r in range(self.R)]
+            self.x = self.xs[0]
             w = syn.weights(name, device=device)
             self.signs = syn.workload_signs(name).to(device)
-            self.wq = None if self.fmt == "int4_asym" else rq.prepare_weights(w, self.signs, self.block, self.wfmt)
+            wq = None if self.fmt == "int4_asym" else rq.prepare_weights(w, self.signs, self.block, self.wfmt)
             del w
+            self.wqs = [None if wq is None else tuple(None if t is None else t.clone() for t in wq)
+                        for _ in range(self.R)]
+            self.wq = self.wqs[0]
             m, k, n = c["M"], c["K"], c["N"]
-            self.xq_out = rq._alloc_quant_outputs(m, k, rq._fmt(self.fmt), device)
-            self.gscale = torch.empty((1,), dtype=torch.float32, device=device)
+            self.xq_outs = [rq._alloc_quant_outputs(m, k, rq._fmt(self.fmt), device) for _ in range(self.R)]
+            self.xq_out = self.xq_outs[0]
+            self.gscales = [torch.empty((1,), dtype=torch.float32, device=device) for _ in range(self.R)]
+            self.gscale = self.gscales[0]
             self.ws = torch.empty((16,), dtype=torch.uint8, device=device)
-            self.y = torch.empty((m, n), dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32,
-                                 device=device)
+            self.ys = [torch.empty((m, n), dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32,
+                                   device=device) for _ in range(self.R)]
+            self.y = self.ys[0]
             self.quant_bytes = m * k * 2 + code_bytes(self.fmt, m, k)
             self.gemm_ops = 2 * m * n * k
             self.h2d_bytes = self.x.numel() * 2
@@ -187,7 +228,7 @@ class Workload:
         # the rows (plus the sign table) fits its 220 KiB of shared memory;
         # otherwise a max launch precedes the quantize launch
         m, k = self.cfg["M"], self.cfg["K"]
-        sms = torch.cuda.get_device_properties(self.x.device).multi_processor_count
+        sms = torch.cuda.get_device_properties(self.xs[0].device).multi_processor_count
         rpc = -(-m // sms)
         return rpc * k * 2 + (k // 128) * 256 + 32 <= 220 * 1024
 
@@ -211,8 +252,9 @@ class Workload:
     def gemm_launches(self):
         return 0 if (self.kv or self.kvdec or self.fmt == "int4_asym") else 1
 
-    def quant(self):
+    def quant(self, i=0):
         rq = self.rq
+        r = i % self.R
         if self.kvdec:
             rq.kv4_decode_attention(self.q, self.kcache, self.vcache, self.signs, out=self.out,
                                     workspace=self.attn_ws)
@@ -221,15 +263,21 @@ class Workload:
             rq.kv_rotate_quantize(self.k, self.signs, out=self.outs[0])
             rq.kv_rotate_quantize(self.v, self.signs, out=self.outs[1])
             return None
-        return rq.rotate_quantize(self.x, self.signs, self.block, self.fmt, "dynamic", gscale=self.gscale,
-                                  out=self.xq_out, workspace=self.ws)
+        return rq.rotate_quantize(self.xs[r], self.signs, self.block, self.fmt, "dynamic", gscale=self.gscales[r],
+                                  out=self.xq_outs[r], workspace=self.ws)
 
-    def gemm(self, xq):
+    def slot_codes(self, i):
+        """The quantized activations of slot i (as the rotate kernel left them)."""
+        r = i % self.R
+        return self.xq_outs[r] + (self.gscales[r] if self.fmt == "nvfp4" else None,)
+
+    def gemm(self, xq, i=0):
         if self.kv or self.kvdec or self.fmt == "int4_asym":
             return None
+        r = i % self.R
         if self.fmt in ("int8", "int6"):
-            return self.rq.int_gemm(xq, self.fmt, self.wq, self.wfmt, self.y_dtype, y=self.y)
-        return self.rq.w4a4_gemm(xq, self.wq, self.fmt, self.y_dtype, y=self.y)
+            return self.rq.int_gemm(xq, self.fmt, self.wqs[r], self.wfmt, self.y_dtype, y=self.ys[r])
+        return self.rq.w4a4_gemm(xq, self.wqs[r], self.fmt, self.y_dtype, y=self.ys[r])
 
     def result(self):
         if self.kvdec:
@@ -439,48 +487,52 @@ def main():
     from rotation_w4a4_quantization_b200 import rq
     rq.init(local)
     wl = Workload(args.workload, rq, dev, seed_offset=rank, y_dtype=args.y_dtype)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    K = args.steps
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        xq = wl.quant()
-        if ev is not None:
-            ev[1].record(stream)
-        wl.gemm(xq)
-        if ev is not None:
-            ev[2].record(stream)
+    def step(i):
+        wl.gemm(wl.quant(i), i)
 
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        step()
+    def timed(fn):
+        """K launches of fn(i) back to back on the stream, between one pair of
+        events; the inputs cycle through the ring (larger than L2 together)."""
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(2_000_000)   # keep the GPU busy while the launches queue up
+        a.record(stream)
+        for i in range(K):
+            fn(i)
+        b.record(stream)
+        return a, b
+
+    for i in range(max(args.warmup, 3, wl.R)):
+        step(i)
     rq.get_device_error()
     torch.cuda.synchronize()
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # the timed region: K steps of the whole path, back to back
     clocks = ClockSampler(local)
     clocks.start()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()           # evict L2 (126 MB) between steps
-        step(events[i])
+    ev_step = timed(step)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clk = clocks.stop()
     rq.get_device_error()
-
-    q_ms = np.array([e[0].elapsed_time(e[1]) for e in events])
-    g_ms = np.array([e[1].elapsed_time(e[2]) for e in events])
-    step_ms = q_ms + g_ms
-    tot = torch.tensor([step_ms.sum(), q_ms.sum(), g_ms.sum()], dtype=torch.float64, device=dev)
+    # per-kernel averages for the roofline: each kernel alone, K launches the same way
+    ev_q = timed(lambda i: wl.quant(i))
+    ev_g = timed(lambda i: wl.gemm(wl.slot_codes(i), i)) if wl.gemm_launches() else None
+    torch.cuda.synchronize()
+    rq.get_device_error()
+    step_tot = ev_step[0].elapsed_time(ev_step[1])
+    q_tot = ev_q[0].elapsed_time(ev_q[1])
+    g_tot = ev_g[0].elapsed_time(ev_g[1]) if ev_g is not None else 0.0
+    tot = torch.tensor([step_tot, q_tot, g_tot], dtype=torch.float64, device=dev)
     if dist is not None:
         dist.all_reduce(tot, op=dist.ReduceOp.MAX)
     tot = tot.cpu().numpy()
-    K = args.steps
     ms_step = tot[0] / K
     q_mean_ms = tot[1] / K
     g_mean_ms = tot[2] / K
@@ -592,7 +644,15 @@ def workload_config(args, wl=None):
         cfg["block"] = "full" if c["block"] == 0 else c["block"]
         cfg["y_dtype"] = args.y_dtype
         cfg["weights"] = "rotated+quantized once before timing (offline side)"
-    cfg["l2"] = "flushed between steps (256 MiB memset, outside the kernel events)"
+    r = ring_slots(args.workload)
+    if r > 1:
+        cfg["l2"] = ("inputs larger than L2: %d distinct input sets (activations and weight codes, %d MB) "
+                     "cycled step to step, steps back to back, no flush" % (r, ring_bytes(args.workload) // 10**6))
+    else:
+        cfg["l2"] = ("inputs larger than L2 (%d MB read per step), steps back to back, no flush"
+                     % (ring_bytes(args.workload) // 10**6))
+    cfg["timing"] = ("K steps between one event pair (max over ranks); per-kernel averages from K launches "
+                     "of each kernel alone over the same inputs")
     return cfg
 
 
