@@ -284,6 +284,19 @@ RQ_API rq_status rq_rotate_quantize_nvfp4_noalloc(const void* X_dev, int64_t M, 
                                                   const int8_t* signs_dev, uint8_t* codes_dev, void* scales_dev,
                                                   float* gscale_dev, rq_stream_t stream);
 
+/*
+ * rq_selftest_wait_timeout: exercises the device-side timeout path (every
+ * wait of this library's kernels on an mbarrier or a flag is bounded).
+ * Launches one tiny kernel that waits on an mbarrier
+ * nobody arrives at, for at most `limit_cycles` SM clock cycles (1 .. the
+ * library's own limit of 2e9 cycles, ~1 s), then records RQ_ERR_TIMEOUT in
+ * the device error word and returns; the context stays usable.  The next
+ * rq_get_device_error on the stream reports RQ_ERR_TIMEOUT (and clears it).
+ * Returns RQ_ERR_INVALID_ARG for a limit out of range, RQ_ERR_CUDA if the
+ * launch fails.
+ */
+RQ_API rq_status rq_selftest_wait_timeout(int64_t limit_cycles, rq_stream_t stream);
+
 /* Synchronizes `stream`, returns RQ_ERR_TIMEOUT if any kernel of this library
  * recorded a device-side timeout since the last call (and clears the record),
  * RQ_ERR_CUDA if the stream reports an error, else RQ_OK. */

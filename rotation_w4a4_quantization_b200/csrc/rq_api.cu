@@ -455,6 +455,12 @@ rq_status rq_int_gemm(const uint8_t* xcodes_dev, const float* xscales_dev, rq_fo
                                static_cast<cudaStream_t>(stream));
 }
 
+rq_status rq_selftest_wait_timeout(int64_t limit_cycles, rq_stream_t stream) {
+  if (limit_cycles <= 0 || limit_cycles > (int64_t)kWaitLimitCycles) return RQ_ERR_INVALID_ARG;
+  rq::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((long long)limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
 rq_status rq_get_device_error(rq_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RQ_ERR_CUDA;
   unsigned v = 0, zero = 0;

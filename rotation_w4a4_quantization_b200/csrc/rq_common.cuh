@@ -65,17 +65,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
 }
 
 // Bounded wait on an mbarrier phase. Returns false (and records a timeout in
-// the device error word) if the phase did not complete within the limit.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
+// the device error word) if the phase did not complete within `limit` SM
+// clock cycles (kWaitLimitCycles, ~1 s, unless given).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity,
+                                                  long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
       return false;
     }
   }
   return true;
+}
+
+// Self-test of the timeout path: one thread waits on an mbarrier that expects
+// an arrival nobody makes, with a short limit, and so records a timeout.
+__global__ void selftest_wait_timeout_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait_bounded(&bar, 0u, limit);
+  }
 }
 
 // 1-D bulk copy global -> shared (TMA engine, no tensor map), completion

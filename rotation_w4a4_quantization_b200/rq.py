@@ -23,7 +23,7 @@ STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3:
 EXPORTED = ["rq_init", "rq_status_string", "rq_workspace_bytes", "rq_rotate_quantize", "rq_prepare_weights",
             "rq_w4a4_gemm", "rq_kv_rotate_quantize", "rq_rotate_f32", "rq_get_device_error",
             "rq_rotate_quantize_nvfp4_noalloc", "rq_kv4_attention_workspace_bytes", "rq_kv4_decode_attention",
-            "rq_int_gemm"]
+            "rq_int_gemm", "rq_selftest_wait_timeout"]
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("librq.so not built: run `python -m rotation_w4a4_quantization_b200.build`")
@@ -56,6 +56,8 @@ lib.rq_kv4_attention_workspace_bytes.argtypes = [_i64, _i64, _i64]
 lib.rq_kv4_attention_workspace_bytes.restype = ctypes.c_size_t
 lib.rq_kv4_decode_attention.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, ctypes.c_float, _p, _i, _p, _p]
 lib.rq_kv4_decode_attention.restype = _i
+lib.rq_selftest_wait_timeout.argtypes = [_i64, _p]
+lib.rq_selftest_wait_timeout.restype = _i
 lib.rq_get_device_error.argtypes = [_p]
 lib.rq_get_device_error.restype = _i
 
@@ -255,6 +257,11 @@ def kv4_decode_attention(q, kcache, vcache, signs, softmax_scale=0.0, out_dtype=
                                        _ptr(signs), float(softmax_scale), _ptr(out), o, _ptr(workspace), _stream(q)),
            "rq_kv4_decode_attention")
     return out
+
+
+def selftest_wait_timeout(limit_cycles=1_000_000):
+    """Launch the self-test kernel whose bounded wait runs out (see rq.h)."""
+    _check(lib.rq_selftest_wait_timeout(int(limit_cycles), _stream()), "rq_selftest_wait_timeout")
 
 
 def get_device_error(stream=None):
