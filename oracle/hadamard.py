@@ -16,23 +16,33 @@ Reading taken where the pages are silent: Q = diag(s) . H_B / sqrt(B) per block
 applied to X and to W, so (X.Q)(W.Q)^T = X.W^T.
 """
 
+import functools
+
 import numpy as np
 
 
 def sylvester(n):
     """Dense Sylvester Hadamard H_n (n a power of two), fp64, entries +-1.
 
-    Closed form H[i, j] = (-1)^popcount(i & j).
+    Closed form H[i, j] = (-1)^popcount(i & j).  The matrix depends on n only;
+    it is built once per n and returned read-only.
     """
     if n < 1 or (n & (n - 1)) != 0:
         raise ValueError("Hadamard order must be a power of two, got %d" % n)
+    return _sylvester_built(n)
+
+
+@functools.lru_cache(maxsize=16)
+def _sylvester_built(n):
     idx = np.arange(n, dtype=np.int64)
     anded = idx[:, None] & idx[None, :]
     parity = np.zeros_like(anded)
     while np.any(anded):
         parity ^= anded & 1
         anded >>= 1
-    return np.where(parity == 0, 1.0, -1.0)
+    h = np.where(parity == 0, 1.0, -1.0)
+    h.setflags(write=False)
+    return h
 
 
 def rotation_block_matrix(signs_blk):
