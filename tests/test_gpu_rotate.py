@@ -223,3 +223,22 @@ def test_full_width_4096_row_counts(rq, m, fmt):
     else:
         parity.check_int_quant(parity.to_np(codes), parity.to_np(scales), xr, 8)
     assert parity.to_np(scales)[m // 2] == 0
+
+
+@pytest.mark.parametrize("block,k", [(128, 512), (32, 256), (16, 256), (0, 4096), (0, 1024)])
+def test_rotate_f32_onehot_is_exact(rq, block, k):
+    """A one-hot row rotates to +-v/sqrt(B) on its block and exact zeros elsewhere
+    (one nonzero term per output: no rounding but the fp32 1/sqrt(B) itself)."""
+    b = k if block == 0 else block
+    rows = [(0, 1.0), (k - 1, -2.0), (k // 2 + 5, 0.5)]
+    x = torch.zeros((len(rows), k), dtype=torch.float32)
+    for r, (ch, val) in enumerate(rows):
+        x[r, ch] = val
+    s = _signs(k, 31)
+    got = parity.to_np(rq.rotate_f32(x.to(torch.bfloat16).cuda(), s.cuda(), block)).astype(np.float64)
+    inv = float(np.float32(1.0 / np.sqrt(b)))
+    for r, (ch, val) in enumerate(rows):
+        blk = ch // b
+        inside = got[r, blk * b:(blk + 1) * b]
+        assert np.all(np.abs(inside) == abs(val) * inv)
+        assert np.all(np.delete(got[r], np.s_[blk * b:(blk + 1) * b]) == 0)
