@@ -235,13 +235,44 @@ __device__ __forceinline__ void fwht_block_diag(float (&v)[128]) {
     fwht_blocks<LOGB>(v);
 }
 
-// XOR key of a thread's chunk order for blocks of 2^logb: only chunk-index
-// bits inside a block may be permuted (the transform then turns the
-// permutation into the sign pattern chi); with 16- or 32-wide blocks that
-// leaves 1 or 2 bits, so the shared-memory reads of those modes keep 4- or
-// 2-way bank conflicts.
-__device__ __forceinline__ int chunk_key(int lane, int logb) {
-  return lane & ((1 << (logb - 3)) - 1) & 7;
+// A lane reads its block's 8-element chunks in the order j ^ m so that the
+// lanes of a shared-memory phase hit distinct banks (m = lane mod 8 makes the
+// reads conflict-free).  The bits of m inside one rotation block (chunk-index
+// bits below log2(B/8)) turn into the output sign pattern chi of the
+// transform; bits above it only swap whole blocks of 16 or 32 values, so
+// register chunk j then holds output chunk j ^ mo with mo = those bits, and
+// the stores put it there (kPermuted).  That is done for 16-wide blocks (a
+// 4-way conflict otherwise); 32-wide blocks keep m inside the block (2-way
+// conflicts), which measured faster than scattering their stores.
+template <int LOGB>
+struct ChunkOrder {
+  static constexpr bool kPermuted = LOGB == 4;
+  static constexpr int T = LOGB >= 7 ? 15 : (1 << (LOGB - 3)) - 1;
+};
+struct ChunkKeys {
+  int m;     // read order key
+  int mchi;  // the part of m inside a block (sign pattern)
+  int mo;    // the part of m above a block (output chunk permutation)
+};
+template <int LOGB>
+__device__ __forceinline__ ChunkKeys chunk_keys(int lane) {
+  constexpr int T = ChunkOrder<LOGB>::T;
+  const int m = ChunkOrder<LOGB>::kPermuted ? (lane & 7) : (lane & T & 7);
+  return ChunkKeys{m, m & T, m & ~T & 7};
+}
+
+// Store the four code words of chunks 4 j4 .. 4 j4 + 3 (4 bytes each) in place,
+// or (PERM) each at chunk j ^ mo.
+template <bool PERM>
+__device__ __forceinline__ void store_words4(uint8_t* dst, int j4, int mo, uint32_t w0, uint32_t w1, uint32_t w2,
+                                             uint32_t w3) {
+  if (!PERM) {
+    reinterpret_cast<uint4*>(dst)[j4] = make_uint4(w0, w1, w2, w3);
+  } else {
+    const uint32_t w[4] = {w0, w1, w2, w3};
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) *reinterpret_cast<uint32_t*>(dst + 4 * ((4 * j4 + jj) ^ mo)) = w[jj];
+  }
 }
 
 // chi for 8-element chunk `chunk` of a thread with XOR key m: +-1 as a sign bit.
@@ -291,7 +322,8 @@ __device__ __forceinline__ float absmax128(const float (&v)[128]) {
 
 // INT4 per-row quantization of v (true value = v * c * chi) and packing.
 // amax_true: the row's max |x~|.  Writes 64 bytes at dst.
-__device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c, float amax_true, int m,
+template <bool PERM = false>
+__device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c, float amax_true, int m, int mo,
                                                  uint8_t* dst) {
   // r = 7/amax; zero rows -> r = 0 -> all codes 0
   const float r = amax_true > 0.f ? __fdiv_rn(7.0f, amax_true) : 0.0f;
@@ -314,15 +346,17 @@ __device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c,
       }
       w[jj] = pack8_magic(q);
     }
-    out[j4] = make_uint4(w[0], w[1], w[2], w[3]);
+    store_words4<PERM>(dst, j4, mo, w[0], w[1], w[2], w[3]);
   }
+  (void)out;
 }
 
 // 6- / 8-bit per-row quantization of v (true value = v * c * chi): codes
 // rint(x * qmax / amax) in [-qmax, qmax], one two's-complement byte each.
 // Writes 128 bytes at dst.
+template <bool PERM = false>
 __device__ __forceinline__ void quant_int8_store(const float (&v)[128], float c, float amax_true, float qmax, int m,
-                                                 uint8_t* dst) {
+                                                 int mo, uint8_t* dst) {
   const float r = amax_true > 0.f ? __fdiv_rn(qmax, amax_true) : 0.0f;
   const float cr = c * r;
   uint4* out = reinterpret_cast<uint4*>(dst);
@@ -344,14 +378,20 @@ __device__ __forceinline__ void quant_int8_store(const float (&v)[128], float c,
       w[2 * h] = gather_low_bytes(q[0], q[1], q[2], q[3]);
       w[2 * h + 1] = gather_low_bytes(q[4], q[5], q[6], q[7]);
     }
-    out[j2] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (!PERM) {
+      out[j2] = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {  // chunk j (8 bytes) at chunk j ^ mo
+      *reinterpret_cast<uint2*>(dst + 8 * ((2 * j2) ^ mo)) = make_uint2(w[0], w[1]);
+      *reinterpret_cast<uint2*>(dst + 8 * ((2 * j2 + 1) ^ mo)) = make_uint2(w[2], w[3]);
+    }
   }
 }
 
 // NVFP4 quantization of v (true value = v * c * chi): 8 groups of 16.
 // Writes 64 bytes of codes and 8 bytes of E4M3 scales.
+template <bool PERM = false>
 __device__ __forceinline__ void quant_nvfp4_store(const float (&v)[128], float c, float g, float inv6g, int m,
-                                                  uint8_t* dst_codes, uint8_t* dst_scales) {
+                                                  int mo, uint8_t* dst_codes, uint8_t* dst_scales) {
   uint32_t words[16];
   uint32_t sc_lo = 0, sc_hi = 0;
 #pragma unroll
@@ -376,15 +416,18 @@ __device__ __forceinline__ void quant_nvfp4_store(const float (&v)[128], float c
       words[j] = pack8_e2m1(s[0] * mul, s[1] * mul, s[2] * mul, s[3] * mul, s[4] * mul, s[5] * mul, s[6] * mul,
                             s[7] * mul);
     }
-    if (gi < 4)
+    if (PERM) {
+      dst_scales[gi ^ (mo >> 1)] = (uint8_t)scode;  // group gi = chunks 2 gi, 2 gi + 1
+    } else if (gi < 4) {
       sc_lo |= scode << (8 * gi);
-    else
+    } else {
       sc_hi |= scode << (8 * (gi - 4));
+    }
   }
-  uint4* out = reinterpret_cast<uint4*>(dst_codes);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) out[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
-  *reinterpret_cast<uint2*>(dst_scales) = make_uint2(sc_lo, sc_hi);
+  for (int j = 0; j < 4; ++j)
+    store_words4<PERM>(dst_codes, j, mo, words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+  if (!PERM) *reinterpret_cast<uint2*>(dst_scales) = make_uint2(sc_lo, sc_hi);
 }
 
 // MXFP4 quantization of v (true value = v * c * chi): 4 groups of 32 with an
@@ -393,7 +436,8 @@ __device__ __forceinline__ void quant_nvfp4_store(const float (&v)[128], float c
 // subnormal amax gives -127 - 2 and clamps to -127).  x / 2^e is exact, so the
 // only rounding left is the E2M1 conversion.  Writes 64 bytes of codes and 4
 // bytes of scales.
-__device__ __forceinline__ void quant_mxfp4_store(const float (&v)[128], float c, int m, uint8_t* dst_codes,
+template <bool PERM = false>
+__device__ __forceinline__ void quant_mxfp4_store(const float (&v)[128], float c, int m, int mo, uint8_t* dst_codes,
                                                   uint8_t* dst_scales) {
   uint32_t words[16];
   uint32_t sc = 0;
@@ -408,7 +452,10 @@ __device__ __forceinline__ void quant_mxfp4_store(const float (&v)[128], float c
     const float amax_b = fmaxf(a0, a1) * c;  // true block max
     int ex = (int)((__float_as_uint(amax_b) >> 23) & 0xFFu) - 127 - 2;
     ex = min(max(ex, -127), 127);
-    sc |= (uint32_t)(ex + 127) << (8 * gi);
+    if (PERM)
+      dst_scales[gi ^ (mo >> 2)] = (uint8_t)(ex + 127);  // group gi = chunks 4 gi .. 4 gi + 3
+    else
+      sc |= (uint32_t)(ex + 127) << (8 * gi);
     // 2^-ex: a normal fp32 for ex <= 126; 2^-127 is the subnormal 0x00400000
     const float inv = ex == 127 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - ex) << 23);
     const float ci = c * inv;
@@ -421,14 +468,15 @@ __device__ __forceinline__ void quant_mxfp4_store(const float (&v)[128], float c
                             s[7] * mul);
     }
   }
-  uint4* out = reinterpret_cast<uint4*>(dst_codes);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) out[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
-  *reinterpret_cast<uint32_t*>(dst_scales) = sc;
+  for (int j = 0; j < 4; ++j)
+    store_words4<PERM>(dst_codes, j, mo, words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+  if (!PERM) *reinterpret_cast<uint32_t*>(dst_scales) = sc;
 }
 
 // KV4: asymmetric per-vector quantization (true value = v * c * chi).
-__device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, int m, uint8_t* dst_codes,
+template <bool PERM = false>
+__device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, int m, int mo, uint8_t* dst_codes,
                                                 __half* dst_scale, __half* dst_zero) {
   float lo = 3.0e38f, hi = -3.0e38f;
 #pragma unroll
@@ -484,19 +532,22 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
       }
       w[jj] = pack8_magic(q);
     }
-    out[j4] = make_uint4(w[0], w[1], w[2], w[3]);
+    store_words4<PERM>(dst_codes, j4, mo, w[0], w[1], w[2], w[3]);
   }
+  (void)out;
   *dst_scale = s_h;
   *dst_zero = z_h;
 }
 
-__device__ __forceinline__ void store_f32_block(const float (&v)[128], float c, int m, float* dst) {
+template <bool PERM = false>
+__device__ __forceinline__ void store_f32_block(const float (&v)[128], float c, int m, int mo, float* dst) {
   float4* out = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float mul = with_sign(c, chi_signbit(j, m));
-    out[2 * j] = make_float4(v[8 * j] * mul, v[8 * j + 1] * mul, v[8 * j + 2] * mul, v[8 * j + 3] * mul);
-    out[2 * j + 1] = make_float4(v[8 * j + 4] * mul, v[8 * j + 5] * mul, v[8 * j + 6] * mul, v[8 * j + 7] * mul);
+    const int d = PERM ? (j ^ mo) : j;
+    out[2 * d] = make_float4(v[8 * j] * mul, v[8 * j + 1] * mul, v[8 * j + 2] * mul, v[8 * j + 3] * mul);
+    out[2 * d + 1] = make_float4(v[8 * j + 4] * mul, v[8 * j + 5] * mul, v[8 * j + 6] * mul, v[8 * j + 7] * mul);
   }
 }
 
@@ -702,7 +753,9 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
     b = wig * 32 + lane;
     active = b < nb;
   }
-  const int m = chunk_key(lane, NBF ? 7 : LOGB);
+  constexpr bool PERM = NBF == 0 && ChunkOrder<LOGB>::kPermuted;
+  const ChunkKeys ck = chunk_keys<NBF ? 7 : LOGB>(lane);
+  const int m = ck.m, mchi = ck.mchi, mo = ck.mo;
   const bool producer = (wig == 0 && lane == 0);
   const float c = (NBF || LOGB == 7) ? 0.08838834764831845f : p.cblk;  // 1/sqrt(block), rounded once
   const int64_t TG = (int64_t)gridDim.x * p.GPC;
@@ -770,34 +823,34 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
         const float a = valid ? absmax128(v) * c : 0.f;
         const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
         if (valid) {
-          quant_int4_store(v, c, amax_row, m, p.codes + row * (p.K / 2) + (size_t)b * 64);
+          quant_int4_store<PERM>(v, c, amax_row, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64);
           if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
         }
       } else if (MODE == kModeInt8) {
         const float a = valid ? absmax128(v) * c : 0.f;
         const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
         if (valid) {
-          quant_int8_store(v, c, amax_row, p.qmax, m, p.codes + row * p.K + (size_t)b * 128);
+          quant_int8_store<PERM>(v, c, amax_row, p.qmax, mchi, mo, p.codes + row * p.K + (size_t)b * 128);
           if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, p.qmax);
         }
       } else if (MODE == kModeNvfp4) {
         if (valid)
-          quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                            p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+          quant_nvfp4_store<PERM>(v, c, g, inv6g, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                                  p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
       } else if (MODE == kModeMxfp4) {
         if (valid)
-          quant_mxfp4_store(v, c, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                            p.scales_e4m3 + row * (p.K / 32) + (size_t)b * 4);
+          quant_mxfp4_store<PERM>(v, c, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                                  p.scales_e4m3 + row * (p.K / 32) + (size_t)b * 4);
       } else if (MODE == kModeF32) {
-        if (valid) store_f32_block(v, c, m, p.out_f32 + row * p.ldo + (size_t)b * 128);
+        if (valid) store_f32_block<PERM>(v, c, mchi, mo, p.out_f32 + row * p.ldo + (size_t)b * 128);
       } else if (MODE == kModeAmax) {
         if (valid) amax_acc = fmaxf(amax_acc, absmax128(v) * c);
       } else if (MODE == kModeKv4) {
-        if (valid) quant_kv4_store(v, c, m, p.codes + row * 64, p.kv_scale + row, p.kv_zero + row);
+        if (valid) quant_kv4_store(v, c, m, 0, p.codes + row * 64, p.kv_scale + row, p.kv_zero + row);
       } else if (MODE == kModeAsym4) {
         if (valid) {
           __half* sz = p.kv_scale + 2 * (row * nb + b);
-          quant_kv4_store(v, c, m, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
+          quant_kv4_store<PERM>(v, c, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
         }
       }
     } else {
@@ -1058,7 +1111,9 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
   unsigned* cta_max = reinterpret_cast<unsigned*>(bar + 1);
   int* flag = reinterpret_cast<int*>(cta_max + 1);
   const int tid = threadIdx.x;
-  const int m = chunk_key(tid, LOGB);
+  constexpr bool PERM = ChunkOrder<LOGB>::kPermuted;
+  const ChunkKeys ck = chunk_keys<LOGB>(tid);
+  const int m = ck.m;
   const float c = LOGB == 7 ? 0.08838834764831845f : p.cblk;  // 1/sqrt(block), rounded once
 
   if (tid == 0) {
@@ -1131,8 +1186,8 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
     float v[128];
     load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
     fwht_block_diag<LOGB>(v);
-    quant_nvfp4_store(v, c, g, inv6g, m, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                      p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+    quant_nvfp4_store<PERM>(v, c, g, inv6g, ck.mchi, ck.mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                            p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
   }
 }
 
