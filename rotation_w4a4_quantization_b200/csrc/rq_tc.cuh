@@ -206,18 +206,9 @@ __device__ __forceinline__ void tc_commit_2cta_mc(uint64_t* bar, uint16_t cta_ma
       "h"(cta_mask)
       : "memory");
 }
-__device__ __forceinline__ void mma_i8_2cta(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Same, with A (M = 256 split over the pair: 128 rows in each CTA's TMEM
-// lanes, K packed 4 int8 per 32-bit column) read from tensor memory.
+// Signed 8-bit MMA on a CTA pair (cta_group::2, issued by the even CTA) with A
+// (M = 256 split over the pair: 128 rows in each CTA's TMEM lanes, K packed 4
+// int8 per 32-bit column) read from tensor memory and B from shared memory.
 __device__ __forceinline__ void mma_i8_2cta_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
