@@ -423,7 +423,10 @@ def oracle_sample(name, rows):
         dt = time.perf_counter() - t0
         return ((rows * c["K"] * 2 + code_bytes("int4_asym", rows, c["K"])) / dt / 1e9, None, dt,
                 "%d of %d rows of X" % (rows, c["M"]))
-    x = syn.activations(name, rows=rows).to(torch.float64).numpy()
+    # rows beyond 4096 are timed as repeats of one 4096-row batch (host memory)
+    chunk = min(rows, 4096)
+    reps = -(-rows // chunk)
+    x = syn.activations(name, rows=chunk).to(torch.float64).numpy()
     s = syn.workload_signs(name).numpy()
     k, n = c["K"], c["N"]
     block = c["block"]
@@ -446,34 +449,39 @@ def oracle_sample(name, rows):
         ew, sfw, gw = _ORACLE_W[name]
     else:
         ew, sfw = _ORACLE_W[name]
-    t0 = time.perf_counter()
-    xr = ohad.rotate(x, s, block)
-    if c["fmt"] in ("int8", "int6"):
-        qx, sx, _ = oquant.int_sym_rows(xr, bits[c["fmt"]])
-        qx.astype(np.int8)
-    elif c["fmt"] == "int4":
-        qx, sx, _ = oquant.int4_sym_rows(xr)
-        oquant.pack_nibbles(qx)
-    elif c["fmt"] == "nvfp4":
-        gx = oquant.nvfp4_global_scale(xr)
-        ex, sfx, _, _ = oquant.nvfp4_rows(xr, gx)
-        oquant.pack_nibbles(ex)
-    else:
-        ex, sfx, _, _ = oquant.mxfp4_rows(xr)
-        oquant.pack_nibbles(ex)
-    t1 = time.perf_counter()
-    if c["fmt"] in ("int8", "int6"):
-        ogemm.int4_y(ogemm.int_acc(qx, qw), sx, sw)
-    elif c["fmt"] == "int4":
-        ogemm.int4_y(ogemm.int4_acc(qx, qw), sx, sw)
-    elif c["fmt"] == "nvfp4":
-        ogemm.nvfp4_y(ex, sfx, gx, ew, sfw, gw)
-    else:
-        ogemm.mxfp4_y(ex, sfx, ew, sfw)
-    t2 = time.perf_counter()
-    nbytes = rows * k * 2 + code_bytes(c["fmt"], rows, k)
-    return (nbytes / (t1 - t0) / 1e9, 2.0 * rows * n * k / (t2 - t1) / 1e12, t2 - t0,
-            "%d of %d rows of X with the full W" % (rows, c["M"]))
+    tq = tg = 0.0
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        xr = ohad.rotate(x, s, block)
+        if c["fmt"] in ("int8", "int6"):
+            qx, sx, _ = oquant.int_sym_rows(xr, bits[c["fmt"]])
+            qx.astype(np.int8)
+        elif c["fmt"] == "int4":
+            qx, sx, _ = oquant.int4_sym_rows(xr)
+            oquant.pack_nibbles(qx)
+        elif c["fmt"] == "nvfp4":
+            gx = oquant.nvfp4_global_scale(xr)
+            ex, sfx, _, _ = oquant.nvfp4_rows(xr, gx)
+            oquant.pack_nibbles(ex)
+        else:
+            ex, sfx, _, _ = oquant.mxfp4_rows(xr)
+            oquant.pack_nibbles(ex)
+        t1 = time.perf_counter()
+        if c["fmt"] in ("int8", "int6"):
+            ogemm.int4_y(ogemm.int_acc(qx, qw), sx, sw)
+        elif c["fmt"] == "int4":
+            ogemm.int4_y(ogemm.int4_acc(qx, qw), sx, sw)
+        elif c["fmt"] == "nvfp4":
+            ogemm.nvfp4_y(ex, sfx, gx, ew, sfw, gw)
+        else:
+            ogemm.mxfp4_y(ex, sfx, ew, sfw)
+        t2 = time.perf_counter()
+        tq += t1 - t0
+        tg += t2 - t1
+    done = reps * chunk
+    nbytes = done * k * 2 + code_bytes(c["fmt"], done, k)
+    return (nbytes / tq / 1e9, 2.0 * done * n * k / tg / 1e12, tq + tg,
+            "%d rows of X (%d x %d) with the full W" % (done, reps, chunk))
 
 
 def blas_threads():
@@ -488,9 +496,9 @@ def blas_threads():
 def sample_rows(name):
     """Rows (tokens, vectors, or head-passes for kv4_decode) of the oracle's timed
     sample: about 5-10 s of host work on the GPU machines' 16 cores."""
-    return {"tiny_int4": 64, "q_proj_int4": 4096, "down_proj_int4": 4096, "q_proj_nvfp4": 2048, "kv4": 102400,
-            "q_proj_mxfp4": 4096, "kv4_decode": 1024, "q_proj_w4a8": 4096, "q_proj_w8a8": 4096,
-            "q_proj_nvfp4_b16": 2048, "q_proj_mxfp4_b32": 4096, "q_proj_int4_asym": 16384}[name]
+    return {"tiny_int4": 64, "q_proj_int4": 40960, "down_proj_int4": 16384, "q_proj_nvfp4": 8192, "kv4": 102400,
+            "q_proj_mxfp4": 16384, "kv4_decode": 1024, "q_proj_w4a8": 40960, "q_proj_w8a8": 40960,
+            "q_proj_nvfp4_b16": 8192, "q_proj_mxfp4_b32": 16384, "q_proj_int4_asym": 16384}[name]
 
 
 def min_rows(name):
