@@ -997,9 +997,10 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
   const int64_t step = (int64_t)gridDim.x * kR64Teams;
   int64_t row = (int64_t)blockIdx.x * kR64Teams + team;
   uint4 raw[8];
-  build_sign_table(p.signs, 32, smask, [&]() {
-    if (row < p.rows) load_row64(p, row, t, raw);
-  });
+  // the sign table first, then the first row: issued together, the 4 KB of
+  // signs every CTA reads queue behind the whole grid's row loads
+  build_sign_table(p.signs, 32, smask, []() {});
+  if (row < p.rows) load_row64(p, row, t, raw);
   __syncthreads();
 
 #pragma unroll 1
