@@ -555,7 +555,9 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed steps")
     ev_step = timed(step)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()

@@ -1,6 +1,7 @@
 // librq: the C ABI declared in include/rq.h.  Host-side argument checks,
 // kernel selection and launches.  All kernels live in the headers included
 // below (one translation unit, so the device error word is a single symbol).
+#include <nvtx3/nvToolsExt.h>
 #include "../../include/rq.h"
 
 #include <cuda_runtime.h>
@@ -322,11 +323,20 @@ rq_status noalloc_scratch_address(void** out) {
 
 }  // namespace
 
+
+// An NVTX range around each public call (a no-op unless a profiler such as
+// Nsight Systems or Nsight Compute with NVTX filtering is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 extern "C" {
 
 rq_status rq_rotate_quantize_nvfp4_noalloc(const void* X_dev, int64_t M, int64_t K, int64_t ldx,
                                            const int8_t* signs_dev, uint8_t* codes_dev, void* scales_dev,
                                            float* gscale_dev, rq_stream_t stream) {
+  NvtxRange nvtx_("rq_rotate_quantize_nvfp4_noalloc");
   // The scratch this path needs does not grow with M or K; the check keeps the
   // static array's stated size honest if that ever changes.
   if (rq_workspace_bytes(RQ_NVFP4) > sizeof(g_noalloc_scratch)) return RQ_ERR_UNSUPPORTED_SHAPE;
@@ -375,6 +385,7 @@ size_t rq_workspace_bytes(rq_format fmt) { return fmt == RQ_NVFP4 ? 16 : 0; }
 rq_status rq_rotate_quantize(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev,
                              int block, rq_format fmt, rq_gscale gmode, uint8_t* codes_dev, void* scales_dev,
                              float* gscale_dev, void* workspace_dev, rq_stream_t stream) {
+  NvtxRange nvtx_("rq_rotate_quantize");
   return rotate_quantize_impl(X_dev, M, K, ldx, signs_dev, block, fmt, gmode, codes_dev, scales_dev, gscale_dev,
                               workspace_dev, static_cast<cudaStream_t>(stream));
 }
@@ -382,12 +393,14 @@ rq_status rq_rotate_quantize(const void* X_dev, int64_t M, int64_t K, int64_t ld
 rq_status rq_prepare_weights(const void* W_dev, int64_t N, int64_t K, int64_t ldw, const int8_t* signs_dev,
                              int block, rq_format fmt, uint8_t* codes_dev, void* scales_dev, float* gscale_dev,
                              void* workspace_dev, rq_stream_t stream) {
+  NvtxRange nvtx_("rq_prepare_weights");
   return rotate_quantize_impl(W_dev, N, K, ldw, signs_dev, block, fmt, RQ_SCALE_DYNAMIC, codes_dev, scales_dev,
                               gscale_dev, workspace_dev, static_cast<cudaStream_t>(stream));
 }
 
 rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t ldx, const int8_t* signs_dev, int block,
                         float* out_dev, int64_t ldo, rq_stream_t stream) {
+  NvtxRange nvtx_("rq_rotate_f32");
   rq_status s = check_rotation_args(X_dev, M, K, ldx, signs_dev, block);
   if (s != RQ_OK) return s;
   if (ldo < K) return RQ_ERR_INVALID_ARG;
@@ -406,6 +419,7 @@ rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t ldx, co
 rq_status rq_kv_rotate_quantize(const void* KV_dev, int64_t B, int64_t H, int64_t S, int64_t D,
                                 const int64_t* strides_host, const int8_t* signs_dev, uint8_t* codes_dev,
                                 void* scale_dev, void* zero_dev, rq_stream_t stream) {
+  NvtxRange nvtx_("rq_kv_rotate_quantize");
   if (B < 0 || H < 0 || S < 0) return RQ_ERR_INVALID_ARG;
   if (D != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (B * H * S == 0) return RQ_OK;
@@ -444,6 +458,7 @@ rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev, const
                        const uint8_t* wcodes_dev, const void* wscales_dev, const float* wgscale_dev, int64_t M,
                        int64_t N, int64_t K, rq_format fmt, void* Y_dev, int64_t ldy, rq_out out,
                        rq_stream_t stream) {
+  NvtxRange nvtx_("rq_w4a4_gemm");
   return rq::gemm_dispatch(xcodes_dev, xscales_dev, xgscale_dev, wcodes_dev, wscales_dev, wgscale_dev, M, N, K, fmt,
                            Y_dev, ldy, out, static_cast<cudaStream_t>(stream));
 }
@@ -451,6 +466,7 @@ rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev, const
 rq_status rq_int_gemm(const uint8_t* xcodes_dev, const float* xscales_dev, rq_format xfmt, const uint8_t* wcodes_dev,
                       const float* wscales_dev, rq_format wfmt, int64_t M, int64_t N, int64_t K, void* Y_dev,
                       int64_t ldy, rq_out out, rq_stream_t stream) {
+  NvtxRange nvtx_("rq_int_gemm");
   return rq::int_gemm_dispatch(xcodes_dev, xscales_dev, xfmt, wcodes_dev, wscales_dev, wfmt, M, N, K, Y_dev, ldy, out,
                                static_cast<cudaStream_t>(stream));
 }
@@ -483,6 +499,7 @@ rq_status rq_kv4_decode_attention(const void* q_dev, int64_t B, int64_t H, int64
                                   const void* vscale_dev, const void* vzero_dev, const int8_t* signs_dev,
                                   float softmax_scale, void* out_dev, rq_out out, void* workspace_dev,
                                   rq_stream_t stream) {
+  NvtxRange nvtx_("rq_kv4_decode_attention");
   if (B < 0 || H < 0 || S < 0) return RQ_ERR_INVALID_ARG;
   if (out != RQ_OUT_F32 && out != RQ_OUT_BF16) return RQ_ERR_INVALID_ARG;
   if (!(softmax_scale >= 0.0f) || !std::isfinite(softmax_scale)) return RQ_ERR_INVALID_ARG;
