@@ -537,7 +537,9 @@ def main():
         """K launches of fn(i) back to back on the stream, between one pair of
         events; the inputs cycle through the ring (larger than L2 together)."""
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda._sleep(2_000_000)   # keep the GPU busy while the launches queue up
+        # keep the GPU busy until all K launches are queued (~50 us of host time
+        # each at most), so the timed region measures the GPU, not the host
+        torch.cuda._sleep(min(100_000 * K, 2_000_000_000))
         a.record(stream)
         for i in range(K):
             fn(i)
