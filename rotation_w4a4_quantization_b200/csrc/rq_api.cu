@@ -98,8 +98,10 @@ RotCfg rotate_config(int64_t K, bool full, int mode) {
   return c;
 }
 
+// pdl = false for a launch that directly follows a non-kernel stream operation
+// (a memset), which programmatic launch must not overlap.
 template <int MODE, int NBF, int LOGB = 7>
-rq_status launch_rotate(RotParams p, cudaStream_t st) {
+rq_status launch_rotate(RotParams p, cudaStream_t st, bool pdl = true) {
   const RotCfg c = rotate_config(p.K, NBF != 0, MODE);
   if (c.stages < 2) return RQ_ERR_UNSUPPORTED_SHAPE;
   p.G = c.G;
@@ -110,19 +112,22 @@ rq_status launch_rotate(RotParams p, cudaStream_t st) {
   const int64_t ctas = (p.num_tiles + c.GPC - 1) / c.GPC;
   const int64_t grid = ctas < num_sms_of_current_device() ? ctas : num_sms_of_current_device();
   if (!ensure_smem(reinterpret_cast<const void*>(rotate_kernel<MODE, NBF, LOGB>))) return RQ_ERR_CUDA;
-  rotate_kernel<MODE, NBF, LOGB><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
+  if (pdl)
+    (void)launch_pdl(rotate_kernel<MODE, NBF, LOGB>, dim3((unsigned)grid), dim3(c.threads), c.smem, st, p);
+  else
+    rotate_kernel<MODE, NBF, LOGB><<<(unsigned)grid, c.threads, c.smem, st>>>(p);
   return last_launch_status();
 }
 
 // Block-diagonal rotation: blocks of 128, or of 16 / 32 (p.logb 4 / 5, the
 // format-sized blocks; not for KV4, whose block is the head).
 template <int MODE>
-rq_status launch_block(RotParams p, cudaStream_t st) {
+rq_status launch_block(RotParams p, cudaStream_t st, bool pdl = true) {
   if constexpr (MODE != kModeKv4) {
-    if (p.logb == 4) return launch_rotate<MODE, 0, 4>(p, st);
-    if (p.logb == 5) return launch_rotate<MODE, 0, 5>(p, st);
+    if (p.logb == 4) return launch_rotate<MODE, 0, 4>(p, st, pdl);
+    if (p.logb == 5) return launch_rotate<MODE, 0, 5>(p, st, pdl);
   }
-  return launch_rotate<MODE, 0, 7>(p, st);
+  return launch_rotate<MODE, 0, 7>(p, st, pdl);
 }
 
 // K = 4096: the 64 x 64 two-pass kernel, two CTAs of four row teams per SM.
@@ -132,7 +137,7 @@ rq_status launch_full4096(RotParams p, cudaStream_t st) {
   const int64_t cap = 2 * (int64_t)num_sms_of_current_device();
   const int64_t grid = ctas < cap ? ctas : cap;
   if (!ensure_smem(reinterpret_cast<const void*>(rotate_full4096_kernel<MODE>), (int)kR64Smem)) return RQ_ERR_CUDA;
-  rotate_full4096_kernel<MODE><<<(unsigned)grid, kR64Threads, kR64Smem, st>>>(p);
+  (void)launch_pdl(rotate_full4096_kernel<MODE>, dim3((unsigned)grid), dim3(kR64Threads), kR64Smem, st, p);
   return last_launch_status();
 }
 
@@ -284,7 +289,7 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
     // one pass over HBM when the whole tensor fits in the SMs' shared memory
     s = launch_nvfp4_resident(p, st);
     if (s != RQ_ERR_UNSUPPORTED_SHAPE) return s;
-    s = launch_block<kModeAmax>(p, st);
+    s = launch_block<kModeAmax>(p, st, /*pdl=*/false);  // follows the memset
     if (s != RQ_OK) return s;
     p.nvfp4_dynamic = 1;
     p.g_out = gscale;
@@ -534,9 +539,9 @@ rq_status rq_kv4_decode_attention(const void* q_dev, int64_t B, int64_t H, int64
   p.out_bf16 = out == RQ_OUT_BF16 ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!ensure_smem(reinterpret_cast<const void*>(kv4_attn_partial_kernel), (int)kAttnSmem)) return RQ_ERR_CUDA;
-  kv4_attn_partial_kernel<<<(unsigned)(BH * nchunks), 128, kAttnSmem, st>>>(p);
+  (void)launch_pdl(kv4_attn_partial_kernel, dim3((unsigned)(BH * nchunks)), dim3(128), kAttnSmem, st, p);
   if (cudaGetLastError() != cudaSuccess) return RQ_ERR_CUDA;
-  kv4_attn_combine_kernel<<<(unsigned)BH, 128, 0, st>>>(p);
+  (void)launch_pdl(kv4_attn_combine_kernel, dim3((unsigned)BH), dim3(128), 0, st, p);
   return last_launch_status();
 }
 

@@ -131,6 +131,8 @@ __device__ __forceinline__ float4 attn_scales(const AttnParams& p, int64_t row0,
 }
 
 __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams p) {
+  griddep_wait();
+  griddep_trigger();
   extern __shared__ __align__(128) uint8_t attn_smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(attn_smem + kAttnStages * kAttnStageBytes);
   uint64_t* empty = full + kAttnStages;  // one arrival per warp once it has read the stage
@@ -347,6 +349,8 @@ __global__ void __launch_bounds__(128) kv4_attn_partial_kernel(const AttnParams 
 }
 
 __global__ void __launch_bounds__(128) kv4_attn_combine_kernel(const AttnParams p) {
+  griddep_wait();
+  griddep_trigger();
   __shared__ float buf[128];
   const int64_t bh = blockIdx.x;
   const int d = threadIdx.x, lane = d & 31, warp = d >> 5;

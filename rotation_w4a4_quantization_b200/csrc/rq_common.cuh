@@ -64,6 +64,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
+// Programmatic dependent launch.  Kernels launched with launch_pdl may start
+// while the previous kernel in the stream is still finishing; each kernel
+// first waits (griddep_wait) until every earlier grid has completed and its
+// memory is visible -- before it touches any global memory -- and then lets
+// the next kernel launch early (griddep_trigger).  What overlaps is the
+// launch, the CTA start-up and the previous kernel's tail; not one memory
+// access.  Without the launch attribute both instructions do nothing.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Bounded wait on an mbarrier phase. Returns false (and records a timeout in
 // the device error word) if the phase did not complete within `limit` SM
 // clock cycles (kWaitLimitCycles, ~1 s, unless given).

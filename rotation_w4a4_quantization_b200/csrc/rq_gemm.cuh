@@ -449,6 +449,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_sx, const __grid_constant__ CUtensorMap tmap_sw,
                       const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  griddep_wait();
+  griddep_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* op = base;
@@ -624,6 +626,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
     gemm_fp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                           const __grid_constant__ CUtensorMap tmap_sx, const __grid_constant__ CUtensorMap tmap_sw,
                           const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  griddep_wait();
+  griddep_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* op = base;
@@ -918,6 +922,8 @@ template <bool A8, bool W8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
     gemm_int_2sm_ts_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                            const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  griddep_wait();
+  griddep_trigger();
   using C = I3<A8, W8>;
   constexpr int kI3Stg = C::Stg, kI3StgA = C::StgA, kI3StgB = C::StgB;
   extern __shared__ uint8_t smem_raw[];
@@ -1231,7 +1237,7 @@ rq_status launch_fp4(GemmParams p, const uint8_t* xc, const void* xs, const uint
     const int sms = gemm_num_sms() & ~1;
     const int grid2 = 2 * p.num_tiles < sms ? 2 * p.num_tiles : sms;
     if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_fp4_2sm_kernel<MX>), (int)kN2Smem)) return RQ_ERR_CUDA;
-    gemm_fp4_2sm_kernel<MX><<<grid2, kN2Threads, kN2Smem, st>>>(tx, tw, tsx, tsw, ty, p);
+    (void)launch_pdl(gemm_fp4_2sm_kernel<MX>, dim3(grid2), dim3(kN2Threads), kN2Smem, st, tx, tw, tsx, tsw, ty, p);
     return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
   }
   if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1241,7 +1247,7 @@ rq_status launch_fp4(GemmParams p, const uint8_t* xc, const void* xs, const uint
     return RQ_ERR_CUDA;
   const int grid = p.num_tiles < gemm_num_sms() ? p.num_tiles : gemm_num_sms();
   if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_fp4_kernel<MX>), (int)kF4Smem)) return RQ_ERR_CUDA;
-  gemm_fp4_kernel<MX><<<grid, kGemmThreads, kF4Smem, st>>>(tx, tw, tsx, tsw, ty, p);
+  (void)launch_pdl(gemm_fp4_kernel<MX>, dim3(grid), dim3(kGemmThreads), kF4Smem, st, tx, tw, tsx, tsw, ty, p);
   return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 
@@ -1310,7 +1316,7 @@ inline rq_status gemm_dispatch(const uint8_t* xc, const void* xs, const float* x
       if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
       if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<false, false>), (int)kI3Smem))
         return RQ_ERR_CUDA;
-      gemm_int_2sm_ts_kernel<false, false><<<grid2, kI3Threads, kI3Smem, st>>>(tx2, tw2, ty, p);
+      (void)launch_pdl(gemm_int_2sm_ts_kernel<false, false>, dim3(grid2), dim3(kI3Threads), kI3Smem, st, tx2, tw2, ty, p);
       return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
     }
     if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int4_kernel), (int)kI4Smem)) return RQ_ERR_CUDA;
@@ -1378,12 +1384,12 @@ inline rq_status int_gemm_dispatch(const uint8_t* xc, const float* xs, rq_format
     if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<true, true>),
                           (int)I3<true, true>::Smem))
       return RQ_ERR_CUDA;
-    gemm_int_2sm_ts_kernel<true, true><<<grid2, kI3Threads, I3<true, true>::Smem, st>>>(tx, tw, ty, p);
+    (void)launch_pdl(gemm_int_2sm_ts_kernel<true, true>, dim3(grid2), dim3(kI3Threads), I3<true, true>::Smem, st, tx, tw, ty, p);
   } else {
     if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<true, false>),
                           (int)I3<true, false>::Smem))
       return RQ_ERR_CUDA;
-    gemm_int_2sm_ts_kernel<true, false><<<grid2, kI3Threads, I3<true, false>::Smem, st>>>(tx, tw, ty, p);
+    (void)launch_pdl(gemm_int_2sm_ts_kernel<true, false>, dim3(grid2), dim3(kI3Threads), I3<true, false>::Smem, st, tx, tw, ty, p);
   }
   return cudaGetLastError() == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }

@@ -729,6 +729,8 @@ __device__ __forceinline__ void full_store_int8(const float (&y)[2][NB][64 / NB]
 // ---------------------------------------------------------------------------
 template <int MODE, int NBF, int LOGB = 7>
 __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_kernel(const RotParams p) {
+  griddep_wait();
+  griddep_trigger();
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G, RPS = p.RPS, nb = p.nb;
@@ -987,6 +989,8 @@ __device__ __forceinline__ uint32_t nibbles_of(uint32_t w0, uint32_t w1) {
 
 template <int MODE>
 __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const RotParams p) {
+  griddep_wait();
+  griddep_trigger();
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw);  // [2048] XOR masks, one per bf16 pair
   const int team = threadIdx.x >> 6, t = threadIdx.x & 63, lane = threadIdx.x & 31;
