@@ -825,7 +825,6 @@ done:
 // 2^shift * sum qx qw with shift = 8 (W4A4: both sides widened as 16 q),
 // 4 (A8 x W4) or 0 (A8 x W8).
 // ---------------------------------------------------------------------------
-constexpr int kI3Ops = 4;
 constexpr int kI3BWarps = 8;
 constexpr int kI3AWarp0 = 2 + kI3BWarps;      // 10
 constexpr int kI3EpiWarp0 = kI3AWarp0 + 4;    // 14
@@ -837,10 +836,12 @@ template <bool A8, bool W8>
 struct I3 {
   static constexpr int StgA = A8 ? 128 * 128 : 128 * 64;  // A tile per k-tile: int8 or packed nibbles
   static constexpr int StgB = W8 ? 0 : 128 * 64;          // packed W (W8: straight into the operand ring)
-  static constexpr int Stg = (A8 && !W8) ? 4 : 6;         // staging depth within 227 KB
+  static constexpr int Stg = A8 ? 4 : 6;                  // staging depth within 227 KB
+  static constexpr int Ops = (A8 && W8) ? 6 : 4;           // operand ring: B in smem, A in TMEM (32 columns each)
   static constexpr int BArr = W8 ? 0 : kI3BWarps;         // B converter arrivals per k-tile and CTA
   static constexpr int Shift = A8 ? (W8 ? 0 : 4) : 8;
-  static constexpr size_t Smem = 1024 + (size_t)kI3Ops * kI3OpB + (size_t)Stg * (StgA + StgB) + 2 * kEpiStage + 256;
+  static constexpr size_t Smem = 1024 + (size_t)Ops * kI3OpB + (size_t)Stg * (StgA + StgB) + 2 * kEpiStage + 256;
+  static_assert(Smem <= 232448, "fits the 227 KB of shared memory a CTA may use");
 };
 constexpr size_t kI3Smem = I3<false, false>::Smem;
 
@@ -925,7 +926,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
   griddep_wait();
   griddep_trigger();
   using C = I3<A8, W8>;
-  constexpr int kI3Stg = C::Stg, kI3StgA = C::StgA, kI3StgB = C::StgB;
+  constexpr int kI3Stg = C::Stg, kI3StgA = C::StgA, kI3StgB = C::StgB, kI3Ops = C::Ops;
+  static_assert(kI3ACol0 + 32 * kI3Ops <= 512, "A stages fit the TMEM allocation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* opb = base;                                         // [kI3Ops][B 16K], 128B-swizzled int8
