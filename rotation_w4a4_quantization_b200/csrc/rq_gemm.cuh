@@ -270,6 +270,21 @@ __device__ __forceinline__ void convert_chunk(const uint8_t* stg, uint8_t* op, i
   *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j + 1) ^ sw_out)) = o1;
 }
 
+// The same widening split in two: job jb = 4 r + j reads chunk j of packed
+// row r, and writes its two widened chunks.
+__device__ __forceinline__ uint4 load_chunk(const uint8_t* stg, int jb) {
+  const int r = jb >> 2, j = jb & 3;
+  return *reinterpret_cast<const uint4*>(stg + r * 64 + 16 * (j ^ ((r >> 1) & 3)));
+}
+__device__ __forceinline__ void store_widened(uint8_t* op, int jb, uint4 in) {
+  const int r = jb >> 2, j = jb & 3;
+  uint4 o0, o1;
+  widen16(in, o0, o1);
+  const int sw_out = r & 7;
+  *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j) ^ sw_out)) = o0;
+  *reinterpret_cast<uint4*>(op + r * 128 + 16 * ((2 * j + 1) ^ sw_out)) = o1;
+}
+
 __global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const GemmParams p) {
@@ -1043,8 +1058,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
         if (!wait_or_fail(&op_empty[o], oph ^ 1, abort_flag)) goto done;
         const uint8_t* sb = stg + (size_t)s * (kI3StgA + kI3StgB) + kI3StgA;
         uint8_t* ob = opb + (size_t)o * kI3OpB;
+static_assert(128 * 4 == 2 * 32 * kI3BWarps, "two widening jobs per thread");
+        uint4 in[2];  // both reads issued before the first store
 #pragma unroll
-        for (int jb = t; jb < 128 * 4; jb += 32 * kI3BWarps) convert_chunk(sb, ob, jb >> 2, jb & 3);
+        for (int u = 0; u < 2; ++u) in[u] = load_chunk(sb, t + 32 * kI3BWarps * u);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) store_widened(ob, t + 32 * kI3BWarps * u, in[u]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
