@@ -495,7 +495,7 @@ def blas_threads():
 
 def sample_rows(name):
     """Rows (tokens, vectors, or head-passes for kv4_decode) of the oracle's timed
-    sample: about 5-10 s of host work on the GPU machines' 16 cores."""
+    sample: about 5-10 s of host work on a 16-core host."""
     return {"tiny_int4": 64, "q_proj_int4": 40960, "down_proj_int4": 16384, "q_proj_nvfp4": 8192, "kv4": 102400,
             "q_proj_mxfp4": 16384, "kv4_decode": 1024, "q_proj_w4a8": 40960, "q_proj_w8a8": 40960,
             "q_proj_nvfp4_b16": 8192, "q_proj_mxfp4_b32": 16384, "q_proj_int4_asym": 16384}[name]
