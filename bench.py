@@ -65,7 +65,7 @@ def load_peaks():
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
 ATTN_SOURCES = ("rq_common.cuh", "rq_attn.cuh")
-_ROT, _GEM, _ATT = "d77923a9a24c886e", "18a623aa73ccc565", "80b39046d2c3159b"
+_ROT, _GEM, _ATT = "d77923a9a24c886e", "bbf648be1c99fde4", "80b39046d2c3159b"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
 # ncu capture of the kernel (summarised in profiles/), with the fingerprint of
 # the sources it was taken on (reported as null once they change).  kv4 and
@@ -82,12 +82,12 @@ TRAFFIC = {
     ("hadamard_quant", "q_proj_nvfp4_b16"): (16825600, _ROT),
     ("hadamard_quant", "q_proj_int4_asym"): (16841216, _ROT),
     ("hadamard_quant", "kv4_decode"): (72926720 * 4, _ATT),
-    ("gemm", "q_proj_int4"): (12651264, _GEM),
-    ("gemm", "down_proj_int4"): (61594880, _GEM),
-    ("gemm", "q_proj_nvfp4"): (14189312, _GEM),
-    ("gemm", "q_proj_mxfp4"): (13400832, _GEM),
-    ("gemm", "q_proj_w4a8"): (16844544, _GEM),
-    ("gemm", "q_proj_w8a8"): (25274880, _GEM),
+    ("gemm", "q_proj_int4"): (12649984, _GEM),
+    ("gemm", "down_proj_int4"): (59483904, _GEM),
+    ("gemm", "q_proj_nvfp4"): (14189568, _GEM),
+    ("gemm", "q_proj_mxfp4"): (13400320, _GEM),
+    ("gemm", "q_proj_w4a8"): (16844032, _GEM),
+    ("gemm", "q_proj_w8a8"): (25233920, _GEM),
 }
 
 
