@@ -20,6 +20,11 @@
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and never synchronizes, except
  *    rq_get_device_error and rq_init.
+ *  - The rotate, GEMM and attention kernels are launched with programmatic
+ *    dependent launch: a kernel may be scheduled while the previous kernel on
+ *    the stream drains, but it reads and writes no global memory before that
+ *    kernel has completed, so stream order is kept.  Calls may be captured
+ *    into CUDA graphs.
  *  - Arguments are validated on the host before anything is launched; a
  *    rejected call returns a status other than RQ_OK and leaves every output
  *    untouched.  RQ_ERR_CUDA reports a launch failure (cudaGetLastError).
