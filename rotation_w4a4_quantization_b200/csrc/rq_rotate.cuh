@@ -998,17 +998,19 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
   float* tr = reinterpret_cast<float*>(tb);             // [a][b] fp32, 16-byte granule g of row a at g ^ (a mod 16)
   uint8_t* cb = tb + 64 * 64 * 4;                       // [a][b] code bytes, 8-byte group g of row a at g ^ (a / 8)
   float* slots = reinterpret_cast<float*>(cb + 64 * 64);
-  const int64_t step = (int64_t)gridDim.x * kR64Teams;
-  int64_t row = (int64_t)blockIdx.x * kR64Teams + team;
+  // each CTA a contiguous run of M / grid rows (rounded down or up), dealt to
+  // its teams in turn: no SM carries a whole team-round more rows than another
+  const int64_t row_end = ((int64_t)blockIdx.x + 1) * p.rows / gridDim.x;
+  int64_t row = (int64_t)blockIdx.x * p.rows / gridDim.x + team;
   uint4 raw[8];
   // the sign table first, then the first row: issued together, the 4 KB of
   // signs every CTA reads queue behind the whole grid's row loads
   build_sign_table(p.signs, 32, smask, []() {});
-  if (row < p.rows) load_row64(p, row, t, raw);
+  if (row < row_end) load_row64(p, row, t, raw);
   __syncthreads();
 
 #pragma unroll 1
-  for (; row < p.rows; row += step) {
+  for (; row < row_end; row += kR64Teams) {
     float v[64];
     {
       const uint4* sm = reinterpret_cast<const uint4*>(smask) + t;  // the pairs of elements 8 t + 512 i + e
@@ -1030,7 +1032,7 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
         v[8 * i + 7] = __uint_as_float(w.w & 0xFFFF0000u);
       }
     }
-    if (row + step < p.rows) load_row64(p, row + step, t, raw);
+    if (row + kR64Teams < row_end) load_row64(p, row + kR64Teams, t, raw);
     fwht64(v);
 #pragma unroll
     for (int g = 0; g < 16; ++g)
