@@ -65,20 +65,20 @@ def load_peaks():
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
 ATTN_SOURCES = ("rq_common.cuh", "rq_attn.cuh")
-_ROT, _GEM, _ATT = "d77923a9a24c886e", "bbf648be1c99fde4", "80b39046d2c3159b"
+_ROT, _GEM, _ATT = "ca3beeb8c0e87f73", "bbf648be1c99fde4", "80b39046d2c3159b"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
 # ncu capture of the kernel (summarised in profiles/), with the fingerprint of
 # the sources it was taken on (reported as null once they change).  kv4 and
 # kv4_decode were captured at B = 4 and are scaled to the bench's B = 16 (traffic
 # grows with the vectors processed); kv4_decode is the partial + combine pair.
 TRAFFIC = {
-    ("hadamard_quant", "q_proj_int4"): (16807424, _ROT),
+    ("hadamard_quant", "q_proj_int4"): (16809984, _ROT),
     ("hadamard_quant", "down_proj_int4"): (105441792, _ROT),
     ("hadamard_quant", "kv4"): (146989312 * 4, _ROT),
     ("hadamard_quant", "q_proj_nvfp4"): (16830464, _ROT),
     ("hadamard_quant", "q_proj_mxfp4"): (16832000, _ROT),
-    ("hadamard_quant", "q_proj_w4a8"): (16806912, _ROT),
-    ("hadamard_quant", "q_proj_w8a8"): (16806912, _ROT),
+    ("hadamard_quant", "q_proj_w4a8"): (16809216, _ROT),
+    ("hadamard_quant", "q_proj_w8a8"): (16809216, _ROT),
     ("hadamard_quant", "q_proj_nvfp4_b16"): (16825600, _ROT),
     ("hadamard_quant", "q_proj_int4_asym"): (16841216, _ROT),
     ("hadamard_quant", "kv4_decode"): (72926720 * 4, _ATT),
