@@ -127,3 +127,75 @@ def test_init_without_gpu_reports_unsupported_device():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert lib.rq_init(0) == 4
+
+
+def igemm(xc=A16, xs=A16, xf=3, wc=A16, ws=A16, wf=0, m=256, n=256, k=512, y=A16, ldy=256, out=0):
+    return lib.rq_int_gemm(xc, xs, xf, wc, ws, wf, m, n, k, y, ldy, out, None)
+
+
+def test_int_gemm_rejections():
+    assert igemm(xf=1) == INVALID                  # NVFP4 is not an integer format
+    assert igemm(wf=5) == INVALID                  # per-group asymmetric codes have no GEMM
+    assert igemm(xf=0, wf=3) == SHAPE              # 4-bit activations with wider weights
+    assert igemm(xf=0, wf=0, k=192) == SHAPE       # W4A4 goes through the W4A4 GEMM's checks
+    assert igemm(ldy=100) == INVALID
+    assert igemm(out=9) == INVALID
+    assert igemm(xc=None) == INVALID
+    assert igemm(k=192) == SHAPE
+    assert igemm(k=65536 + 128) == SHAPE
+    assert igemm(xc=A8) == ALIGN
+    assert igemm(y=P(0x10002)) == ALIGN            # fp32 Y 4-byte aligned
+    assert igemm(ws=P(0x10004)) == ALIGN           # weight scales read 16 bytes at a time
+    assert igemm(m=0) == 0 and igemm(n=0) == 0
+
+
+def attn(q=A16, b=2, h=4, s=1500, kc=A16, ks=A16, kz=A16, vc=A16, vs=A16, vz=A16, signs=A16, scale=0.0, o=A16,
+         out=0, ws=A16):
+    return lib.rq_kv4_decode_attention(q, b, h, s, kc, ks, kz, vc, vs, vz, signs, scale, o, out, ws, None)
+
+
+def test_decode_attention_rejections():
+    assert attn(b=-1) == INVALID
+    assert attn(out=2) == INVALID                  # fp32 or bf16 output only
+    assert attn(scale=-1.0) == INVALID
+    assert attn(scale=float("inf")) == INVALID
+    assert attn(scale=float("nan")) == INVALID
+    assert attn(b=0) == 0 and attn(h=0) == 0       # nothing to do
+    assert attn(s=0) == INVALID                    # a softmax over no tokens
+    assert attn(q=None) == INVALID
+    assert attn(ws=None) == INVALID
+    assert attn(vz=None) == INVALID
+    assert attn(q=A8) == ALIGN
+    assert attn(ks=P(0x10001)) == ALIGN
+    assert attn(o=P(0x10002)) == ALIGN             # fp32 output 4-byte aligned
+    assert attn(o=P(0x10001), out=1) == ALIGN      # bf16 output 2-byte aligned
+    assert attn(b=1 << 20, h=1 << 11, s=1024) == SHAPE   # more partial records than a grid holds
+
+
+def test_decode_attention_workspace_bytes():
+    wsb = lib.rq_kv4_attention_workspace_bytes
+    assert wsb(0, 4, 100) == 0 and wsb(2, 0, 100) == 0 and wsb(2, 4, 0) == 0
+    one = wsb(1, 1, 1)
+    assert one > 0 and one % 16 == 0
+    assert wsb(1, 1, 1024) == one                  # one record per 1024 cached tokens
+    assert wsb(1, 1, 1025) == 2 * one
+    assert wsb(2, 4, 1500) == 2 * 4 * 2 * one
+
+
+def test_noalloc_and_selftest_rejections():
+    f = lib.rq_rotate_quantize_nvfp4_noalloc
+    assert f(None, 4, 512, 512, A16, A16, A16, A16, None) == INVALID
+    assert f(A16, 4, 500, 500, A16, A16, A16, A16, None) == SHAPE
+    assert f(A16, 0, 512, 512, A16, A16, A16, A16, None) == 0
+    assert lib.rq_selftest_wait_timeout(0, None) == INVALID
+    assert lib.rq_selftest_wait_timeout(-5, None) == INVALID
+    assert lib.rq_selftest_wait_timeout(1 << 40, None) == INVALID    # above the kernels' own limit
+
+
+def test_rotate_quantize_format_rules():
+    assert rotq(fmt=6) == INVALID                  # no such format
+    assert rotq(fmt=2, block=0) == SHAPE           # MXFP4 needs block-diagonal rotation
+    assert rotq(fmt=5, block=0) == SHAPE           # so do per-group asymmetric codes
+    assert rotq(fmt=3, block=64) == SHAPE          # blocks of 16, 32, 128 or the full width
+    assert rotq(fmt=3, m=0) == 0 and rotq(fmt=4, m=0) == 0 and rotq(fmt=5, m=0) == 0
+    assert rotq(fmt=3, scales=P(0x10002)) == ALIGN  # fp32 scales
