@@ -113,11 +113,15 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *  block      128, 32 or 16 for block-diagonal rotations (32 and 16: blocks
  *             sized to the MXFP4 / NVFP4 scale groups, "Gotchas", "Block size
  *             matters"), or 0 for a full-width rotation (then K must be a power
- *             of two in [256, 4096]; INT4, INT6 and INT8 only).
+ *             of two in [256, 4096]; INT4, INT6 and INT8 only), or 1 for no
+ *             rotation: blocks of one channel, Q = diag(s).  With all signs +1
+ *             that quantizes X itself -- the unrotated arm that section "What
+ *             it buys in 4 bits, and what it doesn't" compares the rotated
+ *             product error against.  Every format takes 1, 16, 32 or 128.
  *  fmt        RQ_INT4:
  *               codes_dev  uint8 [M, K/2], scales_dev float [M]:
  *               s = amax/7 (fp32, amax = max |x~| of the row); q = rint(x~/s).
- *             RQ_NVFP4 (block must be 128):
+ *             RQ_NVFP4:
  *               codes_dev  uint8 [M, K/2] E2M1 codes,
  *               scales_dev uint8 [M, K/16] E4M3 block scales,
  *               gscale_dev float scalar g:
@@ -125,7 +129,7 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *                 RQ_SCALE_STATIC : read.
  *               S_b = E4M3_rn_satfinite(amax_b / (6 g));
  *               e = E2M1_rn_satfinite(x~ / (S_b g)); S_b = 0 gives e = 0.
- *             RQ_MXFP4 (block must be 128):
+ *             RQ_MXFP4:
  *               codes_dev  uint8 [M, K/2] E2M1 codes,
  *               scales_dev uint8 [M, K/32] E8M0 block scales (4-byte aligned):
  *               per block b of 32, 2^e_b with e_b = floor(log2(amax_b)) - 2
@@ -147,6 +151,10 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *               the group's x~, s_h = fp16(s), z_h = fp16(z);
  *               q = clamp(rint((x~ - z_h)/s_h), 0, 15) (s_h = 0 gives q = 0);
  *               x^ = z_h + s_h q.  No GEMM in this library consumes these codes.
+ *               z and s are rounded to fp16 from the exact min and max: a
+ *               group whose fp32 min or scale lies near an fp16 rounding
+ *               midpoint has both re-evaluated in fp64 (as in
+ *               rq_kv_rotate_quantize).
  *  workspace_dev  rq_workspace_bytes(fmt) bytes (may be NULL when that is 0).
  *  codes_dev and scales_dev 16-byte aligned (8 for NVFP4 scales).
  * Values that sit within a few fp32 ulps of a rounding boundary may round
@@ -217,7 +225,10 @@ RQ_API rq_status rq_int_gemm(const uint8_t* xcodes_dev, const float* xscales_dev
  * "Activation scheme": asymmetric INT4 for the KV cache).  Each head_dim
  * vector v of K or V [B, H, S, D] (D = 128) becomes v~ = v.diag(s).H_128/sqrt(128),
  * then z = min(v~), s = (max(v~) - min(v~))/15, stored as fp16 z_h, s_h, and
- * q = clamp(rint((v~ - z_h)/s_h), 0, 15) (s_h = 0 gives q = 0).
+ * q = clamp(rint((v~ - z_h)/s_h), 0, 15) (s_h = 0 gives q = 0).  z_h and s_h
+ * are the fp16 roundings of the exact min and scale: the rotation runs in
+ * fp32, and a vector whose fp32 min or scale lies near an fp16 rounding
+ * midpoint has its min and max re-evaluated in fp64 (about 1 % of vectors).
  *  KV_dev      bf16, element (b,h,t,d) at KV_dev + b*strides_host[0] + h*strides_host[1]
  *              + t*strides_host[2] + d (strides in elements; d contiguous; each
  *              vector 16-byte aligned).
@@ -280,7 +291,9 @@ RQ_API rq_status rq_rotate_f32(const void* X_dev, int64_t M, int64_t K, int64_t 
  *    RQ_ERR_UNSUPPORTED_SHAPE before anything runs.
  *  - The first call on a device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    stream capture.  The cached address belongs to the device's primary
+ *    context: after cudaDeviceReset on that device, do not call this entry
+ *    point again in the same process.
  *  - Every call clears the scratch it uses before use, but all calls share the
  *    one array: calls that may overlap on the GPU (different streams, or
  *    different host threads) race on it and must be serialized by the caller.

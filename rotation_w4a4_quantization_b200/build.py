@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librq.so")
 SOURCES = ["rq_api.cu"]
-HEADERS = ["rq_common.cuh", "rq_rotate.cuh", "rq_gemm.cuh", "rq_tc.cuh"]
+HEADERS = ["rq_common.cuh", "rq_rotate.cuh", "rq_gemm.cuh", "rq_tc.cuh", "rq_attn.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

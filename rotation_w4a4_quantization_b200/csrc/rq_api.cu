@@ -120,10 +120,12 @@ rq_status launch_rotate(RotParams p, cudaStream_t st, bool pdl = true) {
 }
 
 // Block-diagonal rotation: blocks of 128, or of 16 / 32 (p.logb 4 / 5, the
-// format-sized blocks; not for KV4, whose block is the head).
+// format-sized blocks), or of one channel (p.logb 0: no rotation, signs only);
+// not for KV4, whose block is the head.
 template <int MODE>
 rq_status launch_block(RotParams p, cudaStream_t st, bool pdl = true) {
   if constexpr (MODE != kModeKv4) {
+    if (p.logb == 0) return launch_rotate<MODE, 0, 0>(p, st, pdl);
     if (p.logb == 4) return launch_rotate<MODE, 0, 4>(p, st, pdl);
     if (p.logb == 5) return launch_rotate<MODE, 0, 5>(p, st, pdl);
   }
@@ -192,6 +194,7 @@ rq_status launch_nvfp4_resident_b(RotParams p, cudaStream_t st) {
 }
 
 rq_status launch_nvfp4_resident(RotParams p, cudaStream_t st) {
+  if (p.logb == 0) return launch_nvfp4_resident_b<0>(p, st);
   if (p.logb == 4) return launch_nvfp4_resident_b<4>(p, st);
   if (p.logb == 5) return launch_nvfp4_resident_b<5>(p, st);
   return launch_nvfp4_resident_b<7>(p, st);
@@ -203,16 +206,16 @@ rq_status check_rotation_args(const void* X, int64_t M, int64_t K, int64_t ldx, 
   if (M > 0 && (!X || !signs)) return RQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || ldx < K) return RQ_ERR_INVALID_ARG;
   if (K % 128 != 0 || K > kMaxKBlock) return RQ_ERR_UNSUPPORTED_SHAPE;
-  if (block != 0 && block != 16 && block != 32 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
+  if (block != 0 && block != 1 && block != 16 && block != 32 && block != 128) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (block == 0 && !(is_pow2(K) && K >= 256 && K <= 4096)) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(X, 16) || (ldx * 2) % 16 != 0 || !aligned(signs, 16)) return RQ_ERR_ALIGNMENT;
   return RQ_OK;
 }
 
-// Block-diagonal rotation size (16, 32 or 128; 0 = full width leaves 128).
+// Block-diagonal rotation size (1, 16, 32 or 128; 0 = full width leaves 128).
 void set_block(RotParams& p, int block) {
-  const int b = (block == 16 || block == 32) ? block : 128;
-  p.logb = b == 16 ? 4 : (b == 32 ? 5 : 7);
+  const int b = (block == 1 || block == 16 || block == 32) ? block : 128;
+  p.logb = b == 1 ? 0 : (b == 16 ? 4 : (b == 32 ? 5 : 7));
   p.cblk = (float)(1.0 / std::sqrt((double)b));
 }
 

@@ -227,11 +227,13 @@ __device__ __forceinline__ void fwht_blocks(float (&v)[128]) {
   }
 }
 
+// LOGB = 0 is the identity: blocks of one channel, Q = diag(s) (the
+// unrotated arm, signs only).
 template <int LOGB>
 __device__ __forceinline__ void fwht_block_diag(float (&v)[128]) {
   if constexpr (LOGB == 7)
     fwht128(v);
-  else
+  else if constexpr (LOGB > 0)
     fwht_blocks<LOGB>(v);
 }
 
@@ -244,10 +246,12 @@ __device__ __forceinline__ void fwht_block_diag(float (&v)[128]) {
 // the stores put it there (kPermuted).  That is done for 16-wide blocks (a
 // 4-way conflict otherwise); 32-wide blocks keep m inside the block (2-way
 // conflicts), which measured faster than scattering their stores.
+// With no rotation (LOGB = 0) a block is one channel: every bit of m lies
+// above it, so the whole key permutes the stores, as for 16-wide blocks.
 template <int LOGB>
 struct ChunkOrder {
-  static constexpr bool kPermuted = LOGB == 4;
-  static constexpr int T = LOGB >= 7 ? 15 : (1 << (LOGB - 3)) - 1;
+  static constexpr bool kPermuted = LOGB <= 4;
+  static constexpr int T = LOGB >= 7 ? 15 : (LOGB <= 3 ? 0 : (1 << (LOGB - 3)) - 1);
 };
 struct ChunkKeys {
   int m;     // read order key
@@ -474,9 +478,96 @@ __device__ __forceinline__ void quant_mxfp4_store(const float (&v)[128], float c
   if (!PERM) *reinterpret_cast<uint32_t*>(dst_scales) = sc;
 }
 
-// KV4: asymmetric per-vector quantization (true value = v * c * chi).
-template <bool PERM = false>
-__device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, int m, int mo, uint8_t* dst_codes,
+// Global address of row `row`'s first input element.
+__device__ __forceinline__ const uint8_t* row_src(const RotParams& p, int64_t row) {
+  if (p.contiguous) return p.x + row * (int64_t)p.K * 2;
+  const int64_t t = row % p.S, bh = row / p.S;
+  return p.x + (bh / p.H) * p.sB + (bh % p.H) * p.sH + t * p.sS;
+}
+
+// True when the fp16 rounding of v could change within +-band, i.e. v lies
+// that close to the midpoint between two neighbouring fp16 values.
+__device__ __forceinline__ bool near_fp16_midpoint(float v, float band) {
+  return __half2float(__float2half_rn(v - band)) != __half2float(__float2half_rn(v + band));
+}
+
+// 1 / sqrt(2^LOGB) in fp64 (LOGB = 0, 4, 5, 7).
+template <int LOGB>
+__device__ __forceinline__ double inv_sqrt_block_f64() {
+  if constexpr (LOGB == 0) return 1.0;
+  else if constexpr (LOGB == 4) return 0.25;
+  else if constexpr (LOGB == 5) return 0.125 * 1.4142135623730951;   // 2^-2.5 = 2^-3 sqrt(2)
+  else return 0.0625 * 1.4142135623730951;                            // 2^-3.5 = 2^-4 sqrt(2)
+}
+
+// The rotated min and max of one group of 128 channels, in fp64, by the whole
+// warp: lane l takes channels 4l .. 4l+3 of the group's bf16 inputs at `src`
+// (global memory) and of its sign masks, and the fast Walsh-Hadamard
+// butterflies of the 2^LOGB-wide blocks run in fp64 (the first two stages
+// within a lane, the others across lanes), scaled by 1/sqrt(2^LOGB).  The sum
+// of a block's +-x is exact in fp64 for any inputs whose magnitudes span less
+// than 2^45, so the result is the true min / max to within one fp64 rounding.
+template <int LOGB>
+__device__ __forceinline__ void rotated_minmax_f64(const uint8_t* src, const uint32_t* smask_grp, int lane, double& lo,
+                                                   double& hi) {
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src) + lane);
+  const uint2 mk = *reinterpret_cast<const uint2*>(smask_grp + 2 * lane);
+  const uint32_t a = raw.x ^ mk.x, b = raw.y ^ mk.y;
+  double v[4] = {(double)__uint_as_float(a << 16), (double)__uint_as_float(a & 0xFFFF0000u),
+                 (double)__uint_as_float(b << 16), (double)__uint_as_float(b & 0xFFFF0000u)};
+  if constexpr (LOGB >= 1) {  // h = 1
+    const double t0 = v[0], t2 = v[2];
+    v[0] = t0 + v[1];
+    v[1] = t0 - v[1];
+    v[2] = t2 + v[3];
+    v[3] = t2 - v[3];
+  }
+  if constexpr (LOGB >= 2) {  // h = 2
+    const double t0 = v[0], t1 = v[1];
+    v[0] = t0 + v[2];
+    v[2] = t0 - v[2];
+    v[1] = t1 + v[3];
+    v[3] = t1 - v[3];
+  }
+#pragma unroll
+  for (int j = 0; j + 2 < LOGB; ++j) {  // h = 4 * 2^j: the partner is lane ^ 2^j
+    const bool upper = (lane >> j) & 1;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double o = __shfl_xor_sync(0xFFFFFFFFu, v[e], 1 << j);
+      v[e] = upper ? o - v[e] : v[e] + o;
+    }
+  }
+  double mn = fmin(fmin(v[0], v[1]), fmin(v[2], v[3]));
+  double mx = fmax(fmax(v[0], v[1]), fmax(v[2], v[3]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fmin(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+    mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  }
+  const double c = inv_sqrt_block_f64<LOGB>();
+  lo = mn * c;
+  hi = mx * c;
+}
+
+// KV4 and per-group asymmetric INT4: asymmetric quantization of one group of
+// 128 channels (true value = v * c * chi): z = min, s = (max - min)/15, both
+// stored as fp16, q = clamp(rint((x - z)/s), 0, 15).
+//
+// The fp32 butterflies leave the group's min and max within about 2^-23 of
+// its largest magnitude (measured; the bound of a 7-level summation is a few
+// times that), which can decide the fp16 rounding of z or s when either lies
+// that close to a midpoint between two fp16 values.  The lanes for which that
+// is possible (a band of 2^-20 of the largest magnitude around z, 2^-22 around
+// s: about 1 % of groups) have their group's min and max re-evaluated in fp64
+// by the whole warp (rotated_minmax_f64), so z and s are the fp16 roundings of
+// the exact values.  Every lane of the warp must call this function together;
+// `valid` marks lanes that hold a real group (only they store), and `src_of()`
+// gives the group's global input address (called only by lanes that need the
+// re-evaluation).
+template <bool PERM, int LOGB, typename SrcFn>
+__device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, int m, int mo, bool valid,
+                                                SrcFn src_of, const uint32_t* smask_grp, uint8_t* dst_codes,
                                                 __half* dst_scale, __half* dst_zero) {
   float lo = 3.0e38f, hi = -3.0e38f;
 #pragma unroll
@@ -498,8 +589,31 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
   lo *= c;
   hi *= c;
   const float s = __fdiv_rn(hi - lo, 15.0f);
-  const __half s_h = __float2half_rn(s);
-  const __half z_h = __float2half_rn(lo);
+  __half s_h = __float2half_rn(s);
+  __half z_h = __float2half_rn(lo);
+  {
+    const float am = fmaxf(fabsf(lo), fabsf(hi));
+    const bool unsure = valid && (near_fp16_midpoint(lo, am * 0x1p-20f) || near_fp16_midpoint(s, am * 0x1p-22f));
+    unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
+    if (pending) {
+      const int lane = threadIdx.x & 31;
+      const uint8_t* src = unsure ? src_of() : nullptr;
+      while (pending) {
+        const int L = __ffs(pending) - 1;
+        pending &= pending - 1;
+        const uint8_t* srcL =
+            reinterpret_cast<const uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(src), L));
+        const uint32_t* mskL = reinterpret_cast<const uint32_t*>(
+            __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(smask_grp), L));
+        double dlo, dhi;
+        rotated_minmax_f64<LOGB>(srcL, mskL, lane, dlo, dhi);
+        if (lane == L) {
+          z_h = __double2half(dlo);
+          s_h = __double2half((dhi - dlo) / 15.0);
+        }
+      }
+    }
+  }
   const float sf = __half2float(s_h);
   const float zf = __half2float(z_h);
   const float inv = sf > 0.f ? __frcp_rn(sf) : 0.0f;
@@ -509,7 +623,6 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
   // whether clamping to [0, 15] can be needed for this vector.
   const float tlo = fmaf(lo, inv, off), thi = fmaf(hi, inv, off);
   const bool need_clamp = !(tlo > -0.5f && thi < 15.5f);
-  uint4* out = reinterpret_cast<uint4*>(dst_codes);
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
     uint32_t w[4];
@@ -532,11 +645,12 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
       }
       w[jj] = pack8_magic(q);
     }
-    store_words4<PERM>(dst_codes, j4, mo, w[0], w[1], w[2], w[3]);
+    if (valid) store_words4<PERM>(dst_codes, j4, mo, w[0], w[1], w[2], w[3]);
   }
-  (void)out;
-  *dst_scale = s_h;
-  *dst_zero = z_h;
+  if (valid) {
+    *dst_scale = s_h;
+    *dst_zero = z_h;
+  }
 }
 
 template <bool PERM = false>
@@ -759,7 +873,8 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
   const ChunkKeys ck = chunk_keys<NBF ? 7 : LOGB>(lane);
   const int m = ck.m, mchi = ck.mchi, mo = ck.mo;
   const bool producer = (wig == 0 && lane == 0);
-  const float c = (NBF || LOGB == 7) ? 0.08838834764831845f : p.cblk;  // 1/sqrt(block), rounded once
+  // 1/sqrt(block), rounded once; 1 without a rotation
+  const float c = (NBF || LOGB == 7) ? 0.08838834764831845f : (LOGB == 0 ? 1.0f : p.cblk);
   const int64_t TG = (int64_t)gridDim.x * p.GPC;
   const int64_t gg = (int64_t)blockIdx.x * p.GPC + grp;
 
@@ -848,12 +963,12 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
       } else if (MODE == kModeAmax) {
         if (valid) amax_acc = fmaxf(amax_acc, absmax128(v) * c);
       } else if (MODE == kModeKv4) {
-        if (valid) quant_kv4_store(v, c, m, 0, p.codes + row * 64, p.kv_scale + row, p.kv_zero + row);
+        quant_kv4_store<false, 7>(v, c, m, 0, valid, [&]() { return row_src(p, row); }, smask, p.codes + row * 64,
+                                  p.kv_scale + row, p.kv_zero + row);
       } else if (MODE == kModeAsym4) {
-        if (valid) {
-          __half* sz = p.kv_scale + 2 * (row * nb + b);
-          quant_kv4_store<PERM>(v, c, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
-        }
+        __half* sz = p.kv_scale + 2 * (row * nb + b);
+        quant_kv4_store<PERM, LOGB>(v, c, mchi, mo, valid, [&]() { return row_src(p, row) + (size_t)b * 256; },
+                                    smask + bl * 64, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
       }
     } else {
       constexpr int NB = NBF ? NBF : 1;
@@ -1121,7 +1236,7 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
   constexpr bool PERM = ChunkOrder<LOGB>::kPermuted;
   const ChunkKeys ck = chunk_keys<LOGB>(tid);
   const int m = ck.m;
-  const float c = LOGB == 7 ? 0.08838834764831845f : p.cblk;  // 1/sqrt(block), rounded once
+  const float c = LOGB == 7 ? 0.08838834764831845f : (LOGB == 0 ? 1.0f : p.cblk);  // 1/sqrt(block), rounded once
 
   if (tid == 0) {
     mbar_init(bar, 1);

@@ -104,6 +104,72 @@ def _require_cuda(*ts):
             raise ValueError("librq takes CUDA tensors only")
 
 
+# Host-side checks of what the C ABI cannot see (dtypes, inner strides and the
+# sizes of caller-passed buffers), so that a mismatch raises ValueError here
+# instead of making a kernel read or write out of bounds.
+def _expect(t, shape, dtype, name, contiguous=True):
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if contiguous and not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _expect_matrix_bf16(x, name):
+    if x.dim() != 2:
+        raise ValueError("%s must be 2-D [rows, K], got %d-D" % (name, x.dim()))
+    if x.dtype != torch.bfloat16:
+        raise ValueError("%s must be torch.bfloat16, got %s" % (name, x.dtype))
+    if x.shape[0] > 0 and x.stride(1) != 1:
+        raise ValueError("%s rows must be contiguous (stride(1) == 1)" % name)
+
+
+def _expect_signs(signs, k):
+    _expect(signs, (k,), torch.int8, "signs")
+
+
+def _expect_bytes(t, nbytes, name):
+    if not t.is_contiguous() or t.numel() * t.element_size() < nbytes:
+        raise ValueError("%s must be a contiguous buffer of at least %d bytes" % (name, nbytes))
+
+
+def _quant_shapes(rows, k, fmt):
+    """(codes shape, codes dtype, scales shape, scales dtype) that a format writes."""
+    if fmt in (RQ_INT8, RQ_INT6):
+        return (rows, k), torch.int8, (rows,), torch.float32
+    if fmt == RQ_INT4_ASYM:
+        return (rows, k // 2), torch.uint8, (rows, k // 128, 2), torch.float16
+    if fmt == RQ_INT4:
+        return (rows, k // 2), torch.uint8, (rows,), torch.float32
+    if fmt == RQ_NVFP4:
+        return (rows, k // 2), torch.uint8, (rows, k // 16), torch.uint8
+    if fmt == RQ_MXFP4:
+        return (rows, k // 2), torch.uint8, (rows, k // 32), torch.uint8
+    raise ValueError("unknown format %r" % fmt)
+
+
+def _expect_quant_outputs(out, rows, k, fmt):
+    cs, cd, ss, sd = _quant_shapes(rows, k, fmt)
+    codes, scales = out
+    _expect(codes, cs, cd, "codes")
+    _expect(scales, ss, sd, "scales")
+
+
+def _expect_quantized(q, rows, k, fmt, name):
+    """A (codes, scales, gscale) triple as rotate_quantize / prepare_weights return it."""
+    _expect_quant_outputs((q[0], q[1]), rows, k, fmt)
+    if fmt == RQ_NVFP4:
+        if q[2] is None:
+            raise ValueError("%s: NVFP4 needs its per-tensor scale (gscale)" % name)
+        _expect(q[2].reshape(-1)[:1], (1,), torch.float32, name + " gscale", contiguous=False)
+
+
+def _expect_output_matrix(y, m, n, dtype):
+    if y.dtype != dtype or y.dim() != 2 or y.shape[0] != m or y.shape[1] < n or (m > 0 and y.stride(1) != 1):
+        raise ValueError("y must be %s [M, >= N] with contiguous rows" % dtype)
+
+
 def _alloc_quant_outputs(rows, k, fmt, device):
     if fmt in (RQ_INT8, RQ_INT6):  # one int8 code per byte
         return (torch.empty((rows, k), dtype=torch.int8, device=device),
@@ -129,11 +195,25 @@ def rotate_quantize(x, signs, block=128, fmt="int4", gmode="dynamic", gscale=Non
     INT8 / INT6: codes int8 [M, K] (one code per byte), scales fp32 [M], gscale None.
     INT4_ASYM: codes uint8 [M, K/2] (unsigned nibbles), scales fp16 [M, K/128, 2] = (scale, zero).
     """
-    _require_cuda(x, signs)
     f = _fmt(fmt)
+    _expect_matrix_bf16(x, "x")
     m, k = x.shape
-    codes, scales = out if out is not None else _alloc_quant_outputs(m, k, f, x.device)
+    _expect_signs(signs, k)
+    if out is not None:
+        _expect_quant_outputs(out, m, k, f)
+    if gmode not in ("dynamic", "static"):
+        raise ValueError("gmode must be 'dynamic' or 'static'")
     gm = RQ_SCALE_DYNAMIC if gmode == "dynamic" else RQ_SCALE_STATIC
+    if gscale is not None:
+        _expect_bytes(gscale, 4, "gscale")
+        if gscale.dtype != torch.float32:
+            raise ValueError("gscale must be torch.float32")
+    if workspace is not None:
+        _expect_bytes(workspace, workspace_bytes(f), "workspace")
+    if f == RQ_NVFP4 and gscale is None and gm == RQ_SCALE_STATIC:
+        raise ValueError("static NVFP4 scaling needs gscale")
+    _require_cuda(x, signs, gscale, workspace, *(out or ()))
+    codes, scales = out if out is not None else _alloc_quant_outputs(m, k, f, x.device)
     if f == RQ_NVFP4:
         if gscale is None:
             gscale = torch.empty((1,), dtype=torch.float32, device=x.device)
@@ -146,9 +226,15 @@ def rotate_quantize(x, signs, block=128, fmt="int4", gmode="dynamic", gscale=Non
 
 def prepare_weights(w, signs, block=128, fmt="int4", out=None, workspace=None):
     """W [N, K] bf16 -> (codes, scales, gscale), the offline weight side."""
-    _require_cuda(w, signs)
     f = _fmt(fmt)
+    _expect_matrix_bf16(w, "w")
     n, k = w.shape
+    _expect_signs(signs, k)
+    if out is not None:
+        _expect_quant_outputs(out, n, k, f)
+    if workspace is not None:
+        _expect_bytes(workspace, workspace_bytes(f), "workspace")
+    _require_cuda(w, signs, workspace, *(out or ()))
     codes, scales = out if out is not None else _alloc_quant_outputs(n, k, f, w.device)
     gscale = torch.empty((1,), dtype=torch.float32, device=w.device) if f == RQ_NVFP4 else None
     if f == RQ_NVFP4 and workspace is None:
@@ -162,13 +248,23 @@ def w4a4_gemm(xq, wq, fmt="int4", out="f32", y=None):
     """Y = deq(xq) . deq(wq)^T with xq / wq the (codes, scales, gscale) triples."""
     xc, xs, xg = xq
     wc, ws, wg = wq
-    _require_cuda(xc, xs, wc, ws)
     f = _fmt(fmt)
+    if f not in (RQ_INT4, RQ_NVFP4, RQ_MXFP4):
+        raise ValueError("w4a4_gemm takes int4, nvfp4 or mxfp4 codes")
     o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16, "i32": RQ_OUT_I32_ACC}[out]
+    if xc.dim() != 2 or wc.dim() != 2:
+        raise ValueError("codes must be 2-D")
     m, kh = xc.shape
     n = wc.shape[0]
+    if wc.shape[1] != kh:
+        raise ValueError("X and W codes disagree on K: %d vs %d" % (2 * kh, 2 * wc.shape[1]))
+    _expect_quantized(xq, m, 2 * kh, f, "xq")
+    _expect_quantized(wq, n, 2 * kh, f, "wq")
+    dt = {RQ_OUT_F32: torch.float32, RQ_OUT_BF16: torch.bfloat16, RQ_OUT_I32_ACC: torch.int32}[o]
+    if y is not None:
+        _expect_output_matrix(y, m, n, dt)
+    _require_cuda(xc, xs, xg, wc, ws, wg, y)
     if y is None:
-        dt = {RQ_OUT_F32: torch.float32, RQ_OUT_BF16: torch.bfloat16, RQ_OUT_I32_ACC: torch.int32}[o]
         y = torch.empty((m, n), dtype=dt, device=xc.device)
     _check(lib.rq_w4a4_gemm(_ptr(xc), _ptr(xs), _ptr(xg), _ptr(wc), _ptr(ws), _ptr(wg), m, n, 2 * kh, f, _ptr(y),
                             y.stride(0), o, _stream(xc)), "rq_w4a4_gemm")
@@ -181,13 +277,25 @@ def int_gemm(xq, xfmt, wq, wfmt, out="f32", y=None):
     prepare_weights with formats xfmt / wfmt in {"int4", "int6", "int8"}."""
     xc, xs = xq[0], xq[1]
     wc, ws = wq[0], wq[1]
-    _require_cuda(xc, xs, wc, ws)
     fx, fw = _fmt(xfmt), _fmt(wfmt)
+    for f in (fx, fw):
+        if f not in (RQ_INT4, RQ_INT6, RQ_INT8):
+            raise ValueError("int_gemm takes int4, int6 or int8 codes")
     o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16, "i32": RQ_OUT_I32_ACC}[out]
+    if xc.dim() != 2 or wc.dim() != 2:
+        raise ValueError("codes must be 2-D")
     m, n = xc.shape[0], wc.shape[0]
     k = xc.shape[1] * (2 if fx == RQ_INT4 else 1)
+    kw = wc.shape[1] * (2 if fw == RQ_INT4 else 1)
+    if kw != k:
+        raise ValueError("X and W codes disagree on K: %d vs %d" % (k, kw))
+    _expect_quant_outputs((xc, xs), m, k, fx)
+    _expect_quant_outputs((wc, ws), n, k, fw)
+    dt = {RQ_OUT_F32: torch.float32, RQ_OUT_BF16: torch.bfloat16, RQ_OUT_I32_ACC: torch.int32}[o]
+    if y is not None:
+        _expect_output_matrix(y, m, n, dt)
+    _require_cuda(xc, xs, wc, ws, y)
     if y is None:
-        dt = {RQ_OUT_F32: torch.float32, RQ_OUT_BF16: torch.bfloat16, RQ_OUT_I32_ACC: torch.int32}[o]
         y = torch.empty((m, n), dtype=dt, device=xc.device)
     _check(lib.rq_int_gemm(_ptr(xc), _ptr(xs), fx, _ptr(wc), _ptr(ws), fw, m, n, k, _ptr(y), y.stride(0), o,
                            _stream(xc)), "rq_int_gemm")
@@ -196,10 +304,19 @@ def int_gemm(xq, xfmt, wq, wfmt, out="f32", y=None):
 
 def kv_rotate_quantize(kv, signs, out=None):
     """K or V [B, H, S, 128] bf16 (head_dim contiguous) -> (codes [B,H,S,64], scale fp16 [B,H,S], zero fp16 [B,H,S])."""
-    _require_cuda(kv, signs)
+    if kv.dim() != 4 or kv.dtype != torch.bfloat16:
+        raise ValueError("kv must be bf16 [B, H, S, 128]")
     b, h, s, d = kv.shape
+    if d != 128:
+        raise ValueError("head_dim must be 128")
     if kv.stride(3) != 1:
         raise ValueError("head_dim must be contiguous")
+    _expect_signs(signs, d)
+    if out is not None:
+        _expect(out[0], (b, h, s, d // 2), torch.uint8, "codes")
+        _expect(out[1], (b, h, s), torch.float16, "scale")
+        _expect(out[2], (b, h, s), torch.float16, "zero")
+    _require_cuda(kv, signs, *(out or ()))
     if out is None:
         codes = torch.empty((b, h, s, d // 2), dtype=torch.uint8, device=kv.device)
         scale = torch.empty((b, h, s), dtype=torch.float16, device=kv.device)
@@ -214,8 +331,14 @@ def kv_rotate_quantize(kv, signs, out=None):
 
 def rotate_f32(x, signs, block=128, out=None):
     """X.Q as fp32 [M, K]."""
-    _require_cuda(x, signs)
+    _expect_matrix_bf16(x, "x")
     m, k = x.shape
+    _expect_signs(signs, k)
+    if out is not None:
+        if out.dtype != torch.float32 or out.dim() != 2 or out.shape[0] != m or out.shape[1] < k or (
+                m > 0 and out.stride(1) != 1):
+            raise ValueError("out must be fp32 [M, >= K] with contiguous rows")
+    _require_cuda(x, signs, out)
     if out is None:
         out = torch.empty((m, k), dtype=torch.float32, device=x.device)
     _check(lib.rq_rotate_f32(_ptr(x), m, k, x.stride(0), _ptr(signs), int(block), _ptr(out), out.stride(0),
@@ -227,8 +350,14 @@ def rotate_quantize_nvfp4_noalloc(x, signs, out=None, gscale=None):
     """NVFP4 (128-wide blocks, dynamic per-tensor scale) without any device
     workspace: for callers that cannot allocate device memory.  Returns
     (codes, scales, gscale) like rotate_quantize; outputs may be passed in."""
-    _require_cuda(x, signs)
+    _expect_matrix_bf16(x, "x")
     m, k = x.shape
+    _expect_signs(signs, k)
+    if out is not None:
+        _expect_quant_outputs(out, m, k, RQ_NVFP4)
+    if gscale is not None:
+        _expect_bytes(gscale, 4, "gscale")
+    _require_cuda(x, signs, gscale, *(out or ()))
     codes, scales = out if out is not None else _alloc_quant_outputs(m, k, RQ_NVFP4, x.device)
     if gscale is None:
         gscale = torch.empty((1,), dtype=torch.float32, device=x.device)
@@ -244,14 +373,27 @@ def kv4_decode_attention(q, kcache, vcache, signs, softmax_scale=0.0, out_dtype=
     basis."""
     kc, ks, kz = kcache
     vc, vs, vz = vcache
-    _require_cuda(q, kc, ks, kz, vc, vs, vz, signs)
+    if q.dim() != 3 or kc.dim() != 4:
+        raise ValueError("q must be [B, H, 128] and the cache codes [B, H, S, 64]")
     b, h, d = q.shape
     s = kc.shape[2]
+    _expect(q, (b, h, 128), torch.bfloat16, "q")
+    for c, sc, z, nm in ((kc, ks, kz, "k"), (vc, vs, vz, "v")):
+        _expect(c, (b, h, s, 64), torch.uint8, nm + " codes")
+        _expect(sc, (b, h, s), torch.float16, nm + " scale")
+        _expect(z, (b, h, s), torch.float16, nm + " zero")
+    _expect_signs(signs, 128)
     o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16}[out_dtype]
+    odt = torch.float32 if o == RQ_OUT_F32 else torch.bfloat16
+    if out is not None:
+        _expect(out, (b, h, d), odt, "out")
+    nb = int(lib.rq_kv4_attention_workspace_bytes(b, h, s))
+    if workspace is not None:
+        _expect_bytes(workspace, nb, "workspace")
+    _require_cuda(q, kc, ks, kz, vc, vs, vz, signs, out, workspace)
     if out is None:
-        out = torch.empty((b, h, d), dtype=torch.float32 if o == RQ_OUT_F32 else torch.bfloat16, device=q.device)
+        out = torch.empty((b, h, d), dtype=odt, device=q.device)
     if workspace is None:
-        nb = int(lib.rq_kv4_attention_workspace_bytes(b, h, s))
         workspace = torch.empty((max(nb, 16),), dtype=torch.uint8, device=q.device)
     _check(lib.rq_kv4_decode_attention(_ptr(q), b, h, s, _ptr(kc), _ptr(ks), _ptr(kz), _ptr(vc), _ptr(vs), _ptr(vz),
                                        _ptr(signs), float(softmax_scale), _ptr(out), o, _ptr(workspace), _stream(q)),

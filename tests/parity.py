@@ -99,6 +99,7 @@ def check_nvfp4_quant(codes_gpu, sc_gpu, g_gpu, xr, g_ref=None):
     excused = np.repeat(bad_blk, 16, axis=1)
     eg = quant.unpack_nibbles(codes_gpu, signed=False)
     n_e = check_codes(eg, e, tie_e, rank=e2m1_rank, excused=excused, what="e2m1 codes")
+    check_tie_budget(n_s, sc.size, int(excused.sum()) + n_e, e.size, "nvfp4")
     return n_s, n_e
 
 
@@ -114,7 +115,18 @@ def check_mxfp4_quant(codes_gpu, sc_gpu, xr):
     excused = np.repeat(bad, 32, axis=1)
     eg = quant.unpack_nibbles(codes_gpu, signed=False)
     n_e = check_codes(eg, e, tie_e, rank=e2m1_rank, excused=excused, what="e2m1 codes")
+    check_tie_budget(int(bad.sum()), bad.size, int(excused.sum()) + n_e, e.size, "mxfp4")
     return int(bad.sum()), n_e
+
+
+def check_tie_budget(n_scales, total_scales, n_codes, total_codes, what):
+    """Rounding-boundary ties may affect at most TIE_FRACTION of the
+    elements: of the scale (or scale/zero) elements, and of the code elements,
+    where n_codes counts the code mismatches at ties plus every code of a
+    block or vector excused by a scale tie."""
+    assert n_scales <= TIE_FRACTION * total_scales, "%s: %d of %d scales at ties" % (what, n_scales, total_scales)
+    assert n_codes <= TIE_FRACTION * total_codes, "%s: %d of %d codes at or excused by ties" % (
+        what, n_codes, total_codes)
 
 
 def mxfp4_tie_bounds(e, sc, tie_e, tie_s):
@@ -149,6 +161,8 @@ def check_kv4(codes_gpu, scale_gpu, zero_gpu, xr):
     qg = quant.unpack_nibbles(codes_gpu, signed=False)
     excused = np.repeat(bad_sz[..., None], xr.shape[-1], axis=-1)
     n_codes = check_codes(qg, q, tie, excused=excused, what="kv4 codes")
+    n_sz = int((sg != s_h).sum() + (zg != z_h).sum())
+    check_tie_budget(n_sz, 2 * bad_sz.size, int(excused.sum()) + n_codes, q.size, "kv4")
     return n_codes, int(bad_sz.sum())
 
 

@@ -199,3 +199,93 @@ def test_rotate_quantize_format_rules():
     assert rotq(fmt=3, block=64) == SHAPE          # blocks of 16, 32, 128 or the full width
     assert rotq(fmt=3, m=0) == 0 and rotq(fmt=4, m=0) == 0 and rotq(fmt=5, m=0) == 0
     assert rotq(fmt=3, scales=P(0x10002)) == ALIGN  # fp32 scales
+
+
+# ---------------------------------------------------------------- the binding's own checks
+# The Python binding checks what the C ABI cannot see -- dtypes, inner strides
+# and the sizes of caller-passed buffers -- and raises ValueError before any
+# library call.  These run on CPU tensors: the checks come before the
+# CUDA-tensor check, so each message names the real problem.
+import torch  # noqa: E402
+
+
+def _bf16(m, k):
+    return torch.zeros((m, k), dtype=torch.bfloat16)
+
+
+def _s(k):
+    return torch.ones(k, dtype=torch.int8)
+
+
+def _raises(match, fn, *a, **kw):
+    with pytest.raises(ValueError, match=match):
+        fn(*a, **kw)
+
+
+def test_binding_checks_rotate_quantize_inputs():
+    _raises("bfloat16", rq.rotate_quantize, torch.zeros((4, 512)), _s(512))              # fp32 X
+    _raises("stride", rq.rotate_quantize, _bf16(512, 4).t(), _s(512))                   # column-strided X
+    _raises("2-D", rq.rotate_quantize, torch.zeros((2, 4, 512), dtype=torch.bfloat16), _s(512))
+    _raises("signs", rq.rotate_quantize, _bf16(4, 512), _s(256))                        # short signs
+    _raises("signs", rq.rotate_quantize, _bf16(4, 512), torch.ones(512, dtype=torch.int32))
+    _raises("CUDA", rq.rotate_quantize, _bf16(4, 512), _s(512))                         # all right but on the host
+
+
+def test_binding_checks_rotate_quantize_outputs():
+    x, s = _bf16(4, 512), _s(512)
+    ok_codes = torch.empty((4, 256), dtype=torch.uint8)
+    _raises("codes", rq.rotate_quantize, x, s, out=(torch.empty((4, 255), dtype=torch.uint8),
+                                                    torch.empty(4, dtype=torch.float32)))
+    _raises("scales", rq.rotate_quantize, x, s, out=(ok_codes, torch.empty(3, dtype=torch.float32)))
+    _raises("scales", rq.rotate_quantize, x, s, fmt="nvfp4", out=(ok_codes, torch.empty((4, 16), dtype=torch.uint8)))
+    _raises("codes", rq.rotate_quantize, x, s, fmt="int8", out=(ok_codes, torch.empty(4, dtype=torch.float32)))
+    _raises("workspace", rq.rotate_quantize, x, s, fmt="nvfp4", workspace=torch.empty(8, dtype=torch.uint8))
+    _raises("gscale", rq.rotate_quantize, x, s, fmt="nvfp4", gscale=torch.empty(1, dtype=torch.float64))
+    _raises("gscale", rq.rotate_quantize, x, s, fmt="nvfp4", gmode="static")
+    _raises("codes", rq.prepare_weights, x, s, out=(torch.empty((256, 4), dtype=torch.uint8).t(),
+                                                    torch.empty(4, dtype=torch.float32)))
+
+
+def test_binding_checks_gemm_operands():
+    xq = (torch.empty((8, 256), dtype=torch.uint8), torch.empty(8, dtype=torch.float32), None)
+    wq = (torch.empty((16, 256), dtype=torch.uint8), torch.empty(16, dtype=torch.float32), None)
+    wq_k = (torch.empty((16, 128), dtype=torch.uint8), torch.empty(16, dtype=torch.float32), None)
+    _raises("disagree on K", rq.w4a4_gemm, xq, wq_k, "int4")
+    _raises("scales", rq.w4a4_gemm, xq, (wq[0], torch.empty(15, dtype=torch.float32), None), "int4")
+    _raises("scales", rq.w4a4_gemm, xq, wq, "nvfp4")                                    # INT4 scales as NVFP4
+    _raises("gscale", rq.w4a4_gemm, (xq[0], torch.empty((8, 32), dtype=torch.uint8), None),
+            (wq[0], torch.empty((16, 32), dtype=torch.uint8), None), "nvfp4")
+    _raises("y must be", rq.w4a4_gemm, xq, wq, "int4", "f32", y=torch.empty((8, 15), dtype=torch.float32))
+    _raises("y must be", rq.w4a4_gemm, xq, wq, "int4", "bf16", y=torch.empty((8, 16), dtype=torch.float32))
+    _raises("int4, nvfp4 or mxfp4", rq.w4a4_gemm, xq, wq, "int8")
+    _raises("CUDA", rq.w4a4_gemm, xq, wq, "int4")
+    x8 = (torch.empty((8, 512), dtype=torch.int8), torch.empty(8, dtype=torch.float32))
+    _raises("disagree on K", rq.int_gemm, x8, "int8", wq_k, "int4")
+    _raises("codes", rq.int_gemm, (torch.empty((8, 512), dtype=torch.uint8), x8[1]), "int8", wq, "int4")
+    _raises("CUDA", rq.int_gemm, x8, "int8", wq, "int4")
+
+
+def test_binding_checks_kv_and_attention():
+    kv = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    _raises("head_dim", rq.kv_rotate_quantize, torch.zeros((1, 2, 8, 64), dtype=torch.bfloat16), _s(64))
+    _raises("bf16", rq.kv_rotate_quantize, kv.float(), _s(128))
+    _raises("signs", rq.kv_rotate_quantize, kv, _s(64))
+    _raises("scale", rq.kv_rotate_quantize, kv, _s(128), out=(torch.empty((1, 2, 8, 64), dtype=torch.uint8),
+                                                              torch.empty((1, 2, 7), dtype=torch.float16),
+                                                              torch.empty((1, 2, 8), dtype=torch.float16)))
+    cache = (torch.empty((1, 2, 8, 64), dtype=torch.uint8), torch.empty((1, 2, 8), dtype=torch.float16),
+             torch.empty((1, 2, 8), dtype=torch.float16))
+    q = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
+    _raises("q", rq.kv4_decode_attention, q.float(), cache, cache, _s(128))
+    _raises("v codes", rq.kv4_decode_attention, q, cache, (cache[0][:, :, :4], cache[1], cache[2]), _s(128))
+    _raises("workspace", rq.kv4_decode_attention, q, cache, cache, _s(128), workspace=torch.empty(16, dtype=torch.uint8))
+    _raises("out", rq.kv4_decode_attention, q, cache, cache, _s(128), out=torch.empty((1, 2, 128), dtype=torch.bfloat16))
+    _raises("CUDA", rq.kv4_decode_attention, q, cache, cache, _s(128))
+
+
+def test_binding_checks_rotate_f32_and_noalloc():
+    _raises("out", rq.rotate_f32, _bf16(4, 512), _s(512), out=torch.empty((4, 500), dtype=torch.float32))
+    _raises("signs", rq.rotate_f32, _bf16(4, 512), _s(128))
+    _raises("scales", rq.rotate_quantize_nvfp4_noalloc, _bf16(4, 512), _s(512),
+            out=(torch.empty((4, 256), dtype=torch.uint8), torch.empty((4, 16), dtype=torch.uint8)))
+    _raises("CUDA", rq.rotate_quantize_nvfp4_noalloc, _bf16(4, 512), _s(512))

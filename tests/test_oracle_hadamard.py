@@ -124,3 +124,13 @@ def test_sign_flip_changes_result():
     x = rng.standard_normal((2, 128))
     s = rng.choice([-1, 1], size=128)
     assert not np.allclose(hadamard.rotate(x, s, 128), hadamard.rotate(x, np.ones(128), 128))
+
+
+def test_block_of_one_is_the_sign_diagonal():
+    """block = 1 (the unrotated arm): H_1 = [1], so Q = diag(s) and X.Q flips
+    the signs of the channels and nothing else."""
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((5, 64))
+    s = rng.choice([-1, 1], size=64)
+    assert np.array_equal(hadamard.rotate(x, s, 1), x * s)
+    assert np.array_equal(hadamard.rotate(x, np.ones(64, dtype=np.int64), 1), x)

@@ -337,3 +337,64 @@ def test_asym_int4_groups_equal_kv4_per_group():
         qg, sg, zg, _, _ = quant.kv4_vectors(x[:, 128 * g:128 * (g + 1)])
         assert np.array_equal(q[:, 128 * g:128 * (g + 1)], qg)
         assert np.array_equal(s_h[:, g], sg) and np.array_equal(z_h[:, g], zg)
+
+
+# ---------------------------------------------------------------- NVFP4 worked by hand
+def _nvfp4_golden(golden):
+    """Parse tests/golden/nvfp4_block.txt: the per-tensor scale cases and a
+    2 x 32 tensor with its E4M3 block scales and E2M1 codes."""
+    gcases, x, e, s = [], np.zeros((2, 32)), np.zeros((2, 32), dtype=np.int64), np.zeros((2, 2), dtype=np.int64)
+    for line in golden("nvfp4_block.txt"):
+        t = line.split()
+        if t[0] == "g":
+            gcases.append((float(t[1]), int(t[2], 16)))
+            continue
+        r, b = int(t[1]), int(t[2])
+        sl = slice(16 * b, 16 * b + 16)
+        if t[0] == "x":
+            x[r, sl] = [float(v) for v in t[3:]]
+        elif t[0] == "e":
+            e[r, sl] = [int(v) for v in t[3:]]
+        elif t[0] == "s":
+            s[r, b] = int(t[3], 16)
+    return gcases, x, e, s
+
+
+def test_nvfp4_global_scale_golden(golden):
+    gcases, _, _, _ = _nvfp4_golden(golden)
+    assert len(gcases) == 4
+    for amax, bits in gcases:
+        x = np.array([[0.25 * amax, -amax, 0.0, 0.5 * amax]])     # the max is taken over |x|
+        g = quant.nvfp4_global_scale(x)
+        assert g.dtype == np.float32
+        assert int(np.asarray(g).view(np.uint32)) == bits, (amax, hex(int(np.asarray(g).view(np.uint32))))
+
+
+def test_nvfp4_block_golden(golden):
+    """Every block scale and code of the hand-worked tensor (two saturating,
+    one subnormal-scale and two in-between blocks' worth of rounding cases,
+    ties resolved to the even code, -0 written as +0)."""
+    _, x, e_ref, s_ref = _nvfp4_golden(golden)
+    # the fixture's values are exact in bf16, so the same tensor can feed the GPU path
+    import torch
+    assert np.array_equal(torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy(), x)
+    g = quant.nvfp4_global_scale(x)
+    assert g == np.float32(0.0625)
+    e, sc, tie_e, tie_s = quant.nvfp4_rows(x, g)
+    assert np.array_equal(sc, s_ref), (sc, s_ref)
+    assert np.array_equal(e, e_ref), np.argwhere(e != e_ref)
+    assert not tie_s.any()
+    # exact midpoints are flagged as ties (and resolved to the even code above)
+    assert tie_e[0, 3] and tie_e[0, 4] and tie_e[0, 5] and tie_e[1, 16 + 2] and not tie_e[0, 0]
+    xh = quant.nvfp4_dequant(e, sc, g)
+    assert xh[1, 16] == 6 * 2.0 ** -13                               # 8 * 2^-13 saturates to 6 * S g
+
+
+def test_nvfp4_block_golden_catches_a_wrong_scale_divisor(golden, monkeypatch):
+    """A planted mistake in the oracle -- the block scale's divisor 6 g taken
+    as 4 g -- changes three of the four golden block scales."""
+    _, x, _, s_ref = _nvfp4_golden(golden)
+    g = quant.nvfp4_global_scale(x)
+    monkeypatch.setattr(quant, "E2M1_MAX", 4.0)
+    _, sc, _, _ = quant.nvfp4_rows(x, g)
+    assert (sc != s_ref).sum() == 3

@@ -7,7 +7,10 @@ librq.  This file runs last so that a failure here leaves every other test's
 result standing.  It calls the C ABI directly and compares the outputs with
 rq_rotate_quantize's (same kernels, so the match must be exact) on two calls
 in a row, the second with a smaller per-tensor maximum so that a scratch word
-left over from the first call would show.
+left over from the first call would show; a third call, again with a smaller
+maximum, has more rows than the SMs' shared memory holds, so the scratch goes
+through the two-pass path (a max pass that gathers into it, then a quantize
+pass that reads it).
 """
 
 import ctypes
@@ -34,7 +37,7 @@ def _call_noalloc(rq, x, s):
     return codes, scales, g
 
 
-def test_noalloc_matches_regular_entry_point_twice():
+def test_noalloc_matches_regular_entry_point_in_a_row():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     from rotation_w4a4_quantization_b200 import rq
     from rotation_w4a4_quantization_b200 import synthetic as syn
@@ -44,7 +47,8 @@ def test_noalloc_matches_regular_entry_point_twice():
     gen = torch.Generator().manual_seed(92)
     x1 = (torch.randn((333, k), generator=gen) * 3.0).to(torch.bfloat16).cuda()
     x2 = (torch.randn((2048, k), generator=gen) * 0.5).to(torch.bfloat16).cuda()   # smaller max than x1
-    for x in (x1, x2):
+    x3 = (torch.randn((4100, k), generator=gen) * 0.25).to(torch.bfloat16).cuda()  # two-pass, smaller again
+    for x in (x1, x2, x3):
         got = _call_noalloc(rq, x, s)
         ref = rq.rotate_quantize(x, s, 128, "nvfp4", "dynamic")
         torch.cuda.synchronize()
