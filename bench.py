@@ -37,7 +37,14 @@ from rotation_w4a4_quantization_b200 import synthetic as syn  # noqa: E402
 METRIC = "fused Hadamard+quant GB/s vs HBM peak; W4A4 GEMM TOPS vs tensor peak"
 L2_BYTES = 126 << 20      # B200 L2 (nominal)
 RING_MAX = 16
-DEFAULT_WORKLOAD = "q_proj_int4"
+# The default run measures every timed configuration of the metric in one
+# invocation: the headline is down_proj (the largest one carrying both halves
+# of the metric, rotate+quantize and the W4A4 GEMM); q_proj INT4 (full-width
+# rotation), q_proj NVFP4 and the KV4 cache are reported beside it.  The tiny
+# 64 x 512 case is a parity case (launch-bound), not a bench line.
+DEFAULT_WORKLOAD = "all"
+HEADLINE = "down_proj_int4"
+ALSO_MEASURED = ("q_proj_int4", "q_proj_nvfp4", "kv4")
 
 
 def parse():
@@ -45,7 +52,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=["all"] + sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--y-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -526,7 +533,54 @@ def main():
 
     from rotation_w4a4_quantization_b200 import rq
     rq.init(local)
-    wl = Workload(args.workload, rq, dev, seed_offset=rank, y_dtype=args.y_dtype)
+    if args.workload == "all":
+        # every rank measures the same configurations in the same order
+        head = run_workload(HEADLINE, args, rq, dev, dist, world, rank, local, cpu_scale=0.5)
+        head["config"] = workload_config(args, HEADLINE)
+        head["configs"] = {}
+        for name in ALSO_MEASURED:
+            sub = run_workload(name, args, rq, dev, dist, world, rank, local, cpu_scale=0.4)
+            for key in ("metric", "n_gpus", "warmup", "higher_is_better", "scaling", "vs_baseline", "data"):
+                sub.pop(key, None)
+            head["configs"][name] = sub
+        out = head
+    else:
+        out = run_workload(args.workload, args, rq, dev, dist, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def product_errors(name, wl, rq, rows=256):
+    """Relative product error ||X W^T - Y|| / ||X W^T|| of the library's own Y
+    on the first `rows` rows of the workload's X (all N outputs), for the
+    rotated arm (the workload's block and signs) and the unrotated arm
+    (block = 1, all signs +1: the same quantizers on X and W themselves).
+    X W^T is formed in fp64 on the host from the bf16 inputs."""
+    c = wl.cfg
+    dev = wl.x.device
+    x = wl.xs[0][:rows]
+    w = syn.weights(name, device=dev)
+    y_true = x.double().cpu().numpy() @ w.double().cpu().numpy().T
+    ones = torch.ones_like(wl.signs)
+    out = {"rows": int(rows), "outputs": int(c["N"]), "reference": "fp64 X.W^T on the host from the bf16 inputs"}
+    for arm, block, sg in (("rotated", c["block"], wl.signs), ("unrotated", 1, ones)):
+        wq = rq.prepare_weights(w, sg, block, wl.wfmt)
+        xq = rq.rotate_quantize(x.contiguous(), sg, block, wl.fmt)
+        y = rq.w4a4_gemm(xq, wq, wl.fmt, "f32")
+        yh = y.double().cpu().numpy()
+        out[arm] = round(float(np.linalg.norm(yh - y_true) / np.linalg.norm(y_true)), 5)
+        del wq, xq, y
+    out["arms"] = "rotated: block %s with the workload's random signs; unrotated: block 1, signs +1" % (
+        "full" if c["block"] == 0 else c["block"])
+    return out
+
+
+def run_workload(name, args, rq, dev, dist, world, rank, local, cpu_scale=1.0):
+    """Build one workload, time it, and return its JSON object."""
+    wl = Workload(name, rq, dev, seed_offset=rank, y_dtype=args.y_dtype)
     stream = torch.cuda.current_stream(dev)
     K = args.steps
 
@@ -557,18 +611,17 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    torch.cuda.nvtx.range_push("timed steps")
+    torch.cuda.nvtx.range_push("timed steps " + name)
     ev_step = timed(step)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    clk = clocks.stop()
-    rq.get_device_error()
     # per-kernel averages for the roofline: each kernel alone, K launches the same way
     ev_q = timed(lambda i: wl.quant(i))
     ev_g = timed(lambda i: wl.gemm(wl.slot_codes(i), i)) if wl.gemm_launches() else None
     torch.cuda.synchronize()
+    clk = clocks.stop()
     rq.get_device_error()
     step_tot = ev_step[0].elapsed_time(ev_step[1])
     q_tot = ev_q[0].elapsed_time(ev_q[1])
@@ -599,12 +652,12 @@ def main():
         "vs_baseline": None,
         "dtype": wl.cfg.get("fmt", "int4"),
         "data": "synthetic (seeded, shaped like the article's Qwen3-8B layer inputs)",
-        "config": workload_config(args, wl),
+        "config": workload_config(args, name),
         "gpu_launches": K * (wl.quant_launches() + wl.gemm_launches()),
     }
     q_launch_ms = q_mean_ms / wl.quant_launches()
     roof_q = {"bound": "hbm", "achieved": round(wl.quant_bytes / wl.quant_launches() / (q_launch_ms * 1e-3) / 1e9, 1),
-              "peak": peaks["hbm"], "unit": "GB/s", "traffic": traffic("hadamard_quant", args.workload),
+              "peak": peaks["hbm"], "unit": "GB/s", "traffic": traffic("hadamard_quant", name),
               "kernel": wl.quant_kernel(),
               "peak_source": peaks["src"]}
     roof_q["frac"] = round(roof_q["achieved"] / roof_q["peak"], 4)
@@ -616,7 +669,7 @@ def main():
         peak_t = peaks["bf16"] * ratio
         two_sm = wl.cfg["M"] > 128
         roof_g = {"bound": "tensor", "achieved": round(wl.gemm_ops / (g_mean_ms * 1e-3) / 1e12, 1), "peak": peak_t,
-                  "unit": "TFLOP/s", "traffic": traffic("gemm", args.workload),
+                  "unit": "TFLOP/s", "traffic": traffic("gemm", name),
                   "kernel": gemm_kernel_name(wl, two_sm),
                   "peak_source": "%s bf16 x %g (nominal %s/bf16 ratio)" % (peaks["src"], ratio,
                                                                            "int8" if ratio == 2 else "fp4")}
@@ -632,17 +685,19 @@ def main():
     out["hadamard_quant_ms"] = round(q_mean_ms, 5)
     out["e2e"] = e2e
     out["clocks"] = clk
+    if wl.gemm_launches() and wl.fmt in ("int4", "nvfp4"):
+        out["product_error"] = product_errors(name, wl, rq)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, tops_cpu, secs, desc = oracle_sample(args.workload, sample_rows(args.workload))
+        rows = max(min_rows(name), int(sample_rows(name) * cpu_scale))
+        gbs, tops_cpu, secs, desc = oracle_sample(name, rows)
         out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
                                "sample": desc, "seconds": round(secs, 2), "host_cpus": os.cpu_count()}
         if tops_cpu is not None:
             out["cpu_baseline"]["gemm_tops"] = round(tops_cpu, 5)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    del wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_e2e(wl, rq, dev, stream, K):
@@ -712,25 +767,28 @@ def measure_e2e(wl, rq, dev, stream, K):
     return e2e_result(t0.elapsed_time(t1) / K, h2d, d2h)
 
 
-def workload_config(args, wl=None):
-    """The `config` object of both arms (the reference arm passes no Workload)."""
-    c = dict(syn.WORKLOADS[args.workload])
+def workload_config(args, name):
+    """The `config` object of both arms for workload `name`; with the default
+    --workload all, the headline's config also lists the other measured ones."""
+    c = dict(syn.WORKLOADS[name])
     c.pop("index", None)
-    cfg = {"workload": args.workload}
+    cfg = {"workload": name}
     cfg.update(c)
-    if args.workload not in ("kv4", "kv4_decode"):
+    if name not in ("kv4", "kv4_decode"):
         cfg["block"] = "full" if c["block"] == 0 else c["block"]
         cfg["y_dtype"] = args.y_dtype
         cfg["weights"] = "rotated+quantized once before timing (offline side)"
-    r = ring_slots(args.workload)
+    r = ring_slots(name)
     if r > 1:
         cfg["l2"] = ("inputs larger than L2: %d distinct input sets (activations and weight codes, %d MB) "
-                     "cycled step to step, steps back to back, no flush" % (r, ring_bytes(args.workload) // 10**6))
+                     "cycled step to step, steps back to back, no flush" % (r, ring_bytes(name) // 10**6))
     else:
         cfg["l2"] = ("inputs larger than L2 (%d MB read per step), steps back to back, no flush"
-                     % (ring_bytes(args.workload) // 10**6))
+                     % (ring_bytes(name) // 10**6))
     cfg["timing"] = ("K steps between one event pair (max over ranks); per-kernel averages from K launches "
                      "of each kernel alone over the same inputs")
+    if args.workload == "all" and name == HEADLINE:
+        cfg["also_measured"] = list(ALSO_MEASURED)
     return cfg
 
 
@@ -739,14 +797,15 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     K = args.steps
+    name = HEADLINE if args.workload == "all" else args.workload
     # each step a bounded sample: about sample_rows() rows in all, split over
     # the K steps, so that the whole run stays within a few minutes
-    rows = max(min_rows(args.workload), sample_rows(args.workload) // max(K, 1))
+    rows = max(min_rows(name), sample_rows(name) // max(K, 1))
     for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample(args.workload, rows)
+        oracle_sample(name, rows)
     rates, secs = [], 0.0
     for _ in range(K):
-        gbs, tops, s, desc = oracle_sample(args.workload, rows)
+        gbs, tops, s, desc = oracle_sample(name, rows)
         rates.append(gbs)
         secs += s
     v = float(len(rates) / np.sum(1.0 / np.array(rates)))  # the rate over all steps' bytes (equal per step)
@@ -754,7 +813,7 @@ def run_reference(args, world, rank):
         "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(1e3 * secs / K, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
-        "config": workload_config(args),
+        "config": workload_config(args, name),
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -132,14 +132,19 @@ rq_status launch_block(RotParams p, cudaStream_t st, bool pdl = true) {
   return launch_rotate<MODE, 0, 7>(p, st, pdl);
 }
 
-// K = 4096: the 64 x 64 two-pass kernel, two CTAs of four row teams per SM.
+// K = 4096: the 64 x 64 two-pass kernel, two CTAs of four row teams per SM,
+// each CTA's rows staged in up to kF4kSlots shared-memory slots (all of them
+// when they fit, else a ring whose depth is a multiple of the team count).
 template <int MODE>
 rq_status launch_full4096(RotParams p, cudaStream_t st) {
-  const int64_t ctas = (p.rows + kR64Teams - 1) / kR64Teams;
   const int64_t cap = 2 * (int64_t)num_sms_of_current_device();
-  const int64_t grid = ctas < cap ? ctas : cap;
-  if (!ensure_smem(reinterpret_cast<const void*>(rotate_full4096_kernel<MODE>), (int)kR64Smem)) return RQ_ERR_CUDA;
-  (void)launch_pdl(rotate_full4096_kernel<MODE>, dim3((unsigned)grid), dim3(kR64Threads), kR64Smem, st, p);
+  const int64_t grid = p.rows < cap ? p.rows : cap;
+  const int64_t rpc = (p.rows + grid - 1) / grid;  // the most rows any CTA takes
+  const int slots = rpc <= kF4kSlots ? (int)rpc : kF4kSlots;
+  if (!ensure_smem(reinterpret_cast<const void*>(rotate_full4096_kernel<MODE>), (int)f4k_smem_bytes(kF4kSlots)))
+    return RQ_ERR_CUDA;
+  (void)launch_pdl(rotate_full4096_kernel<MODE>, dim3((unsigned)grid), dim3(kR64Threads), f4k_smem_bytes(slots), st,
+                   p, slots);
   return last_launch_status();
 }
 

@@ -355,6 +355,71 @@ __device__ __forceinline__ void quant_int4_store(const float (&v)[128], float c,
   (void)out;
 }
 
+// Per-row symmetric quantization without a rotation (blocks of one channel:
+// v holds the sign-flipped inputs themselves, exact bf16 values), codes
+// rint(x / s) with s = fp32(amax / qmax) the stored scale.  bf16 inputs often
+// sit exactly on, or within fp32 rounding of, a midpoint k + 1/2 of x / s, where
+// a product with the reciprocal may round either way; there the quotient is
+// formed in fp64 (x / s exactly as the plain definition divides).  BITS = 4
+// packs two codes per byte (64 bytes per 128 values), BITS = 8 stores one
+// code per byte (128 bytes).
+template <bool PERM, int BITS>
+__device__ __forceinline__ void quant_int_exact_store(const float (&v)[128], float amax_true, float qmax, int mo,
+                                                      uint8_t* dst) {
+  const float s = __fdiv_rn(amax_true, qmax);
+  const float r = amax_true > 0.f ? __fdiv_rn(qmax, amax_true) : 0.0f;
+  const int qlo = -(int)qmax - 1, qhi = (int)qmax;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    int q[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = v[8 * j + e];
+      const float t = x * r;
+      int qi = __float2int_rn(t);
+      const float d = fabsf(t - floorf(t) - 0.5f);
+      if (d <= 0x1p-18f * fmaxf(1.0f, fabsf(t)) && s > 0.f) qi = __double2int_rn((double)x / (double)s);
+      q[e] = min(max(qi, qlo), qhi);
+    }
+    const int d = PERM ? (j ^ mo) : j;
+    if (BITS == 4) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w |= ((uint32_t)q[e] & 0xFu) << (4 * e);
+      *reinterpret_cast<uint32_t*>(dst + 4 * d) = w;
+    } else {
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w0 |= ((uint32_t)q[e] & 0xFFu) << (8 * e);
+        w1 |= ((uint32_t)q[e + 4] & 0xFFu) << (8 * e);
+      }
+      *reinterpret_cast<uint2*>(dst + 8 * d) = make_uint2(w0, w1);
+    }
+  }
+}
+
+// The E2M1 code (sign in bit 3, magnitude code 0..7 for 0, .5, 1, 1.5, 2, 3,
+// 4, 6) of an fp64 value, rounded to nearest with ties to the even code and
+// saturating at 6; a value that rounds to magnitude 0 gives +0.  Each
+// comparison is against a midpoint of the grid: ">" where the lower neighbour
+// has the even code, ">=" where the upper one has.
+__device__ __forceinline__ uint32_t e2m1_code_f64(double x) {
+  const double a = fabs(x);
+  const uint32_t m = (uint32_t)(a > 0.25) + (uint32_t)(a >= 0.75) + (uint32_t)(a > 1.25) + (uint32_t)(a >= 1.75) +
+                     (uint32_t)(a > 2.5) + (uint32_t)(a >= 3.5) + (uint32_t)(a > 5.0);
+  return (x < 0.0 && m != 0) ? (m | 8u) : m;
+}
+
+// True when the fp32 value t (a quotient x / (S g)) lies within a relative
+// 2^-18 of an E2M1 rounding midpoint (0.25, 0.75, 1.25, 1.75 below 2; 2.5,
+// 3.5 below 4; 5 below 6; the test also fires, harmlessly, at 7 and above).
+__device__ __forceinline__ bool near_e2m1_midpoint(float t) {
+  const float a = fabsf(t);
+  const float u = a < 2.0f ? 2.0f * a : (a < 4.0f ? a : 0.5f * a);
+  return fabsf(u - floorf(u) - 0.5f) <= 0x1p-18f * fmaxf(1.0f, u);
+}
+
 // 6- / 8-bit per-row quantization of v (true value = v * c * chi): codes
 // rint(x * qmax / amax) in [-qmax, qmax], one two's-complement byte each.
 // Writes 128 bytes at dst.
@@ -392,8 +457,11 @@ __device__ __forceinline__ void quant_int8_store(const float (&v)[128], float c,
 }
 
 // NVFP4 quantization of v (true value = v * c * chi): 8 groups of 16.
-// Writes 64 bytes of codes and 8 bytes of E4M3 scales.
-template <bool PERM = false>
+// Writes 64 bytes of codes and 8 bytes of E4M3 scales.  EXACT (the unrotated
+// arm, v = the sign-flipped bf16 inputs, c = 1, chi = +1): a code whose fp32
+// quotient lies near an E2M1 midpoint is decided again from the fp64 quotient
+// x / (S g), the plain definition (bf16 inputs hit such midpoints often).
+template <bool PERM = false, bool EXACT = false>
 __device__ __forceinline__ void quant_nvfp4_store(const float (&v)[128], float c, float g, float inv6g, int m,
                                                   int mo, uint8_t* dst_codes, uint8_t* dst_scales) {
   uint32_t words[16];
@@ -419,6 +487,15 @@ __device__ __forceinline__ void quant_nvfp4_store(const float (&v)[128], float c
       const float* s = &v[8 * j];
       words[j] = pack8_e2m1(s[0] * mul, s[1] * mul, s[2] * mul, s[3] * mul, s[4] * mul, s[5] * mul, s[6] * mul,
                             s[7] * mul);
+      if (EXACT && denom > 0.f) {
+        const double dd = (double)sdec * (double)g;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (near_e2m1_midpoint(s[e] * mul)) {
+            const uint32_t code = e2m1_code_f64((double)s[e] / dd);
+            words[j] = (words[j] & ~(0xFu << (4 * e))) | (code << (4 * e));
+          }
+      }
     }
     if (PERM) {
       dst_scales[gi ^ (mo >> 1)] = (uint8_t)scode;  // group gi = chunks 2 gi, 2 gi + 1
@@ -500,21 +577,25 @@ __device__ __forceinline__ double inv_sqrt_block_f64() {
   else return 0.0625 * 1.4142135623730951;                            // 2^-3.5 = 2^-4 sqrt(2)
 }
 
-// The rotated min and max of one group of 128 channels, in fp64, by the whole
-// warp: lane l takes channels 4l .. 4l+3 of the group's bf16 inputs at `src`
-// (global memory) and of its sign masks, and the fast Walsh-Hadamard
-// butterflies of the 2^LOGB-wide blocks run in fp64 (the first two stages
-// within a lane, the others across lanes), scaled by 1/sqrt(2^LOGB).  The sum
-// of a block's +-x is exact in fp64 for any inputs whose magnitudes span less
-// than 2^45, so the result is the true min / max to within one fp64 rounding.
+// One group of 128 channels rotated in fp64 by the whole warp: lane l takes
+// channels 4l .. 4l+3 of the group's bf16 inputs at `src` (global memory) and
+// of its sign masks, and the fast Walsh-Hadamard butterflies of the
+// 2^LOGB-wide blocks run in fp64 (the first two stages within a lane, the
+// others across lanes), scaled by 1/sqrt(2^LOGB).  On return y[e] is rotated
+// channel 4 lane + e, and lo / hi are the group's min / max (the same in every
+// lane).  The sum of a block's +-x is exact in fp64 for inputs whose
+// magnitudes span less than 2^45, so y is the true rotation to within one
+// fp64 rounding.
 template <int LOGB>
-__device__ __forceinline__ void rotated_minmax_f64(const uint8_t* src, const uint32_t* smask_grp, int lane, double& lo,
-                                                   double& hi) {
+__device__ __forceinline__ void rotated_group_f64(const uint8_t* src, const uint32_t* smask_grp, int lane,
+                                                  double (&v)[4], double& lo, double& hi) {
   const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src) + lane);
   const uint2 mk = *reinterpret_cast<const uint2*>(smask_grp + 2 * lane);
   const uint32_t a = raw.x ^ mk.x, b = raw.y ^ mk.y;
-  double v[4] = {(double)__uint_as_float(a << 16), (double)__uint_as_float(a & 0xFFFF0000u),
-                 (double)__uint_as_float(b << 16), (double)__uint_as_float(b & 0xFFFF0000u)};
+  v[0] = (double)__uint_as_float(a << 16);
+  v[1] = (double)__uint_as_float(a & 0xFFFF0000u);
+  v[2] = (double)__uint_as_float(b << 16);
+  v[3] = (double)__uint_as_float(b & 0xFFFF0000u);
   if constexpr (LOGB >= 1) {  // h = 1
     const double t0 = v[0], t2 = v[2];
     v[0] = t0 + v[1];
@@ -538,6 +619,9 @@ __device__ __forceinline__ void rotated_minmax_f64(const uint8_t* src, const uin
       v[e] = upper ? o - v[e] : v[e] + o;
     }
   }
+  const double c = inv_sqrt_block_f64<LOGB>();
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] *= c;
   double mn = fmin(fmin(v[0], v[1]), fmin(v[2], v[3]));
   double mx = fmax(fmax(v[0], v[1]), fmax(v[2], v[3]));
 #pragma unroll
@@ -545,9 +629,8 @@ __device__ __forceinline__ void rotated_minmax_f64(const uint8_t* src, const uin
     mn = fmin(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
     mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
   }
-  const double c = inv_sqrt_block_f64<LOGB>();
-  lo = mn * c;
-  hi = mx * c;
+  lo = mn;
+  hi = mx;
 }
 
 // KV4 and per-group asymmetric INT4: asymmetric quantization of one group of
@@ -557,14 +640,16 @@ __device__ __forceinline__ void rotated_minmax_f64(const uint8_t* src, const uin
 // The fp32 butterflies leave the group's min and max within about 2^-23 of
 // its largest magnitude (measured; the bound of a 7-level summation is a few
 // times that), which can decide the fp16 rounding of z or s when either lies
-// that close to a midpoint between two fp16 values.  The lanes for which that
-// is possible (a band of 2^-20 of the largest magnitude around z, 2^-22 around
-// s: about 1 % of groups) have their group's min and max re-evaluated in fp64
-// by the whole warp (rotated_minmax_f64), so z and s are the fp16 roundings of
-// the exact values.  Every lane of the warp must call this function together;
+// that close to a midpoint between two fp16 values.  So after the group is
+// stored, the lanes for which that is possible (a band of 2^-20 of the
+// largest magnitude around z, 2^-22 around s: about 1 % of groups) have their
+// group rotated again in fp64 by the whole warp (rotated_group_f64); where the
+// fp16 roundings of the exact min and scale differ from the stored ones (about
+// 2 groups in 10^4), the warp rewrites the group's z, s and codes from the
+// fp64 values.  Every lane of the warp must call this function together;
 // `valid` marks lanes that hold a real group (only they store), and `src_of()`
 // gives the group's global input address (called only by lanes that need the
-// re-evaluation).
+// second look).
 template <bool PERM, int LOGB, typename SrcFn>
 __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, int m, int mo, bool valid,
                                                 SrcFn src_of, const uint32_t* smask_grp, uint8_t* dst_codes,
@@ -589,31 +674,8 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
   lo *= c;
   hi *= c;
   const float s = __fdiv_rn(hi - lo, 15.0f);
-  __half s_h = __float2half_rn(s);
-  __half z_h = __float2half_rn(lo);
-  {
-    const float am = fmaxf(fabsf(lo), fabsf(hi));
-    const bool unsure = valid && (near_fp16_midpoint(lo, am * 0x1p-20f) || near_fp16_midpoint(s, am * 0x1p-22f));
-    unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
-    if (pending) {
-      const int lane = threadIdx.x & 31;
-      const uint8_t* src = unsure ? src_of() : nullptr;
-      while (pending) {
-        const int L = __ffs(pending) - 1;
-        pending &= pending - 1;
-        const uint8_t* srcL =
-            reinterpret_cast<const uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(src), L));
-        const uint32_t* mskL = reinterpret_cast<const uint32_t*>(
-            __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(smask_grp), L));
-        double dlo, dhi;
-        rotated_minmax_f64<LOGB>(srcL, mskL, lane, dlo, dhi);
-        if (lane == L) {
-          z_h = __double2half(dlo);
-          s_h = __double2half((dhi - dlo) / 15.0);
-        }
-      }
-    }
-  }
+  const __half s_h = __float2half_rn(s);
+  const __half z_h = __float2half_rn(lo);
   const float sf = __half2float(s_h);
   const float zf = __half2float(z_h);
   const float inv = sf > 0.f ? __frcp_rn(sf) : 0.0f;
@@ -650,6 +712,48 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
   if (valid) {
     *dst_scale = s_h;
     *dst_zero = z_h;
+  }
+  // the second look at groups whose z or s lies near an fp16 midpoint
+  const float am = fmaxf(fabsf(lo), fabsf(hi));
+  const bool unsure = valid && (near_fp16_midpoint(lo, am * 0x1p-20f) || near_fp16_midpoint(s, am * 0x1p-22f));
+  unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
+  if (pending) {
+    const int lane = threadIdx.x & 31;
+    const uint8_t* src = unsure ? src_of() : nullptr;
+    const uint32_t szbits = ((uint32_t)__half_as_ushort(s_h) << 16) | __half_as_ushort(z_h);
+    __syncwarp();  // this warp's stores above come before any rewrite below
+    while (pending) {
+      const int L = __ffs(pending) - 1;
+      pending &= pending - 1;
+      const auto bcast = [&](const void* ptr) {
+        return (uintptr_t)__shfl_sync(0xFFFFFFFFu, (unsigned long long)reinterpret_cast<uintptr_t>(ptr), L);
+      };
+      const uint8_t* srcL = reinterpret_cast<const uint8_t*>(bcast(src));
+      const uint32_t* mskL = reinterpret_cast<const uint32_t*>(bcast(smask_grp));
+      double y[4], dlo, dhi;
+      rotated_group_f64<LOGB>(srcL, mskL, lane, y, dlo, dhi);
+      const __half zx = __double2half(dlo);
+      const __half sx = __double2half((dhi - dlo) / 15.0);
+      const uint32_t xbits = ((uint32_t)__half_as_ushort(sx) << 16) | __half_as_ushort(zx);
+      if (xbits != __shfl_sync(0xFFFFFFFFu, szbits, L)) {  // the same in every lane
+        uint8_t* dstL = reinterpret_cast<uint8_t*>(bcast(dst_codes));
+        const double sd = (double)__half2float(sx), zd = (double)__half2float(zx);
+        uint32_t nib = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int q = 0;
+          if (sd > 0.0) q = min(max(__double2int_rn((y[e] - zd) / sd), 0), 15);
+          nib |= (uint32_t)q << (4 * e);
+        }
+        *reinterpret_cast<uint16_t*>(dstL + 2 * lane) = (uint16_t)nib;  // channels 4 lane .. 4 lane + 3
+        __half* dsL = reinterpret_cast<__half*>(bcast(dst_scale));
+        __half* dzL = reinterpret_cast<__half*>(bcast(dst_zero));
+        if (lane == 0) {
+          *dsL = sx;
+          *dzL = zx;
+        }
+      }
+    }
   }
 }
 
@@ -940,20 +1044,26 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
         const float a = valid ? absmax128(v) * c : 0.f;
         const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
         if (valid) {
-          quant_int4_store<PERM>(v, c, amax_row, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64);
+          if constexpr (LOGB == 0)
+            quant_int_exact_store<PERM, 4>(v, amax_row, 7.0f, mo, p.codes + row * (p.K / 2) + (size_t)b * 64);
+          else
+            quant_int4_store<PERM>(v, c, amax_row, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64);
           if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, 7.0f);
         }
       } else if (MODE == kModeInt8) {
         const float a = valid ? absmax128(v) * c : 0.f;
         const float amax_row = row_max(a, RPS, nb, G, grp, wig, slots);
         if (valid) {
-          quant_int8_store<PERM>(v, c, amax_row, p.qmax, mchi, mo, p.codes + row * p.K + (size_t)b * 128);
+          if constexpr (LOGB == 0)
+            quant_int_exact_store<PERM, 8>(v, amax_row, p.qmax, mo, p.codes + row * p.K + (size_t)b * 128);
+          else
+            quant_int8_store<PERM>(v, c, amax_row, p.qmax, mchi, mo, p.codes + row * p.K + (size_t)b * 128);
           if (b == 0) p.scales_f32[row] = __fdiv_rn(amax_row, p.qmax);
         }
       } else if (MODE == kModeNvfp4) {
         if (valid)
-          quant_nvfp4_store<PERM>(v, c, g, inv6g, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                                  p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+          quant_nvfp4_store<PERM, LOGB == 0>(v, c, g, inv6g, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                                             p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
       } else if (MODE == kModeMxfp4) {
         if (valid)
           quant_mxfp4_store<PERM>(v, c, mchi, mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
@@ -1029,31 +1139,61 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
 }
 
 // ---------------------------------------------------------------------------
-// Full-width rotation of K = 4096 as a 64 x 64 two-pass transform.
+// Full-width rotation of K = 4096 as a 64 x 64 two-pass transform, with the
+// rows staged in shared memory.
 //
 // Sylvester's H_4096 is the Kronecker product of twelve H_2, one per bit of
 // the element index n, so the bits can be transformed in any grouping.  The
 // row is read as a 64 x 64 matrix X[a][b] with a = bits 3..8 of n and
 // b = bits 0..2 and 9..11: H_64 along b in every matrix row, then H_64 along a
 // in every column.  A team of 64 threads (two warps) owns one row at a time.
-// Thread a loads matrix row a -- eight 16-byte pieces at elements
-// 8 a + 512 i, so each warp load instruction reads 512 contiguous bytes --
-// signs and transforms it (the next row's loads are issued before this row's
-// arithmetic), writes it to shared memory and, after a team barrier,
-// transforms column b = a.  The codes of its outputs (a = 0..63, b) go back
-// through shared memory as bytes, and thread t stores the codes of outputs
-// 64 t .. 64 t + 63 with 16-byte stores.  Four teams per CTA, two CTAs per SM;
-// a team synchronises on its own named barrier (1..4).  Shared-memory
-// granules are XOR-swizzled so that the row writes, column reads and code
-// transposes are free of bank conflicts (the code reads: two-way).
+//
+// Staging: each CTA takes a contiguous run of rows (M / grid, rounded down or
+// up) and, at kernel start, issues one bulk copy (cp.async.bulk, local memory,
+// no multicast) per row into a slot of shared memory -- as many rows as fit,
+// up to kF4kSlots -- and builds its sign table while they are in flight; so
+// every CTA's reads are in the memory system from the start instead of one
+// row per team at a time.  Rows go to the CTA's four teams in turn; with more
+// rows than slots the slots form a ring (kF4kSlots is a multiple of the team
+// count, so a slot always serves the same team), and a team refills its slot
+// once it has finished with the row.
+//
+// Per row: thread a reads matrix row a (elements 8 a + 512 i + e) from the
+// slot, signs and transforms it; the slot then holds, in two halves of 32
+// matrix rows, the fp32 transpose, and thread b transforms column b; the codes
+// of its outputs (a = 0..63, b) go back through the slot as bytes, and thread t
+// stores the codes of outputs 64 t .. 64 t + 63 with 16-byte stores.
+// Shared-memory granules are XOR-swizzled so that the row writes, column reads
+// and code transposes are free of bank conflicts (the code reads: two-way).
+// Two CTAs of four teams per SM; a team synchronises on its own named barrier
+// (1..4).
 // ---------------------------------------------------------------------------
 constexpr int kR64Teams = 4;
 constexpr int kR64Threads = 64 * kR64Teams;
-constexpr size_t kR64TeamBytes = 64 * 64 * 4 + 64 * 64 + 16;  // fp32 transpose | code bytes | amax slots
-constexpr size_t kR64Smem = 2048 * 4 + kR64Teams * kR64TeamBytes;
+constexpr int kF4kSlots = 12;                      // row slots per CTA (a multiple of kR64Teams)
+constexpr size_t kF4kRowBytes = 4096 * 2;
+static_assert(kF4kSlots % kR64Teams == 0, "a slot must always serve the same team");
+__host__ __device__ constexpr size_t f4k_smem_bytes(int slots) {
+  // sign masks | row slots | mbarriers (one per slot) | per-slot issue counts | team max slots | abort flag
+  return 2048 * 4 + (size_t)slots * kF4kRowBytes + (size_t)slots * 8 + (size_t)slots * 4 + kR64Teams * 2 * 4 + 16;
+}
 
 __device__ __forceinline__ void team_sync(int team) {
   asm volatile("bar.sync %0, 64;" ::"r"(team + 1) : "memory");
+}
+
+// Team-wide AND of a predicate (every thread of the team gets the result).
+__device__ __forceinline__ bool team_all(bool v, int team) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 64, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(team + 1)
+      : "memory");
+  return out != 0;
 }
 
 // 64-point fast Walsh-Hadamard transform in registers (unnormalized).
@@ -1082,20 +1222,6 @@ __device__ __forceinline__ void fwht64(float (&v)[64]) {
   }
 }
 
-// Matrix row a of `row` -- elements 8 a + 512 i + e, i, e = 0..7 (bf16) -- into
-// registers, bypassing L1.
-__device__ __forceinline__ void load_row64(const RotParams& p, int64_t row, int a, uint4 (&raw)[8]) {
-  const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.sS) + a;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint4 w;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
-                 : "l"(src + 64 * i));
-    raw[i] = w;
-  }
-}
-
 // Four code bytes (two's complement, element order) -> two packed nibble bytes.
 __device__ __forceinline__ uint32_t nibbles_of(uint32_t w0, uint32_t w1) {
   const uint32_t a = w0 & 0x0F0F0F0Fu, b = w1 & 0x0F0F0F0Fu;
@@ -1103,110 +1229,156 @@ __device__ __forceinline__ uint32_t nibbles_of(uint32_t w0, uint32_t w1) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const RotParams p) {
+__global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const RotParams p, int slots) {
   griddep_wait();
   griddep_trigger();
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw);  // [2048] XOR masks, one per bf16 pair
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw);              // [2048] XOR masks, one per bf16 pair
+  uint8_t* rows = smem_raw + 2048 * 4;                                   // [slots][8 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rows + (size_t)slots * kF4kRowBytes);
+  unsigned* issued = reinterpret_cast<unsigned*>(bars + slots);         // copies issued per slot
+  float* tmax = reinterpret_cast<float*>(issued + slots);                // [team][2]
+  int* abort_flag = reinterpret_cast<int*>(tmax + 2 * kR64Teams);
   const int team = threadIdx.x >> 6, t = threadIdx.x & 63, lane = threadIdx.x & 31;
-  uint8_t* tb = smem_raw + 2048 * 4 + (size_t)team * kR64TeamBytes;
-  float* tr = reinterpret_cast<float*>(tb);             // [a][b] fp32, 16-byte granule g of row a at g ^ (a mod 16)
-  uint8_t* cb = tb + 64 * 64 * 4;                       // [a][b] code bytes, 8-byte group g of row a at g ^ (a / 8)
-  float* slots = reinterpret_cast<float*>(cb + 64 * 64);
-  // each CTA a contiguous run of M / grid rows (rounded down or up), dealt to
-  // its teams in turn: no SM carries a whole team-round more rows than another
-  const int64_t row_end = ((int64_t)blockIdx.x + 1) * p.rows / gridDim.x;
-  int64_t row = (int64_t)blockIdx.x * p.rows / gridDim.x + team;
-  uint4 raw[8];
-  // the sign table first, then the first row: issued together, the 4 KB of
-  // signs every CTA reads queue behind the whole grid's row loads
-  build_sign_table(p.signs, 32, smask, []() {});
-  if (row < row_end) load_row64(p, row, t, raw);
-  __syncthreads();
+  // each CTA a contiguous run of M / grid rows (rounded down or up)
+  const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
+  const int nloc = (int)(((int64_t)blockIdx.x + 1) * p.rows / gridDim.x - r_begin);
+  const int S = nloc < slots ? nloc : slots;  // slots in use (all rows when they fit)
 
-#pragma unroll 1
-  for (; row < row_end; row += kR64Teams) {
-    float v[64];
-    {
-      const uint4* sm = reinterpret_cast<const uint4*>(smask) + t;  // the pairs of elements 8 t + 512 i + e
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 w = raw[i];
-        const uint4 s = sm[64 * i];
-        w.x ^= s.x;
-        w.y ^= s.y;
-        w.z ^= s.z;
-        w.w ^= s.w;
-        v[8 * i + 0] = __uint_as_float(w.x << 16);
-        v[8 * i + 1] = __uint_as_float(w.x & 0xFFFF0000u);
-        v[8 * i + 2] = __uint_as_float(w.y << 16);
-        v[8 * i + 3] = __uint_as_float(w.y & 0xFFFF0000u);
-        v[8 * i + 4] = __uint_as_float(w.z << 16);
-        v[8 * i + 5] = __uint_as_float(w.z & 0xFFFF0000u);
-        v[8 * i + 6] = __uint_as_float(w.w << 16);
-        v[8 * i + 7] = __uint_as_float(w.w & 0xFFFF0000u);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&bars[i], 1);
+      issued[i] = 0;
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  build_sign_table(p.signs, 32, smask, [&]() {
+    if (threadIdx.x == 0) {  // the first S rows, one copy each
+      for (int i = 0; i < S; ++i) {
+        mbar_arrive_expect_tx(&bars[i], (unsigned)kF4kRowBytes);
+        bulk_g2s(rows + (size_t)i * kF4kRowBytes, p.x + (r_begin + i) * p.sS, (unsigned)kF4kRowBytes, &bars[i]);
+        issued[i] = 1;
       }
     }
-    if (row + kR64Teams < row_end) load_row64(p, row + kR64Teams, t, raw);
-    fwht64(v);
+  });
+  __syncthreads();
+
+  float* slot_max = tmax + 2 * team;
+#pragma unroll 1
+  for (int i = team; i < nloc; i += kR64Teams) {
+    const int sl = i % S;
+    const int64_t row = r_begin + i;
+    uint8_t* buf = rows + (size_t)sl * kF4kRowBytes;
+    if (!team_all(mbar_wait_bounded(&bars[sl], (unsigned)((i / S) & 1)), team)) {
+      if (t == 0) atomicOr(abort_flag, 1);
+      break;
+    }
+    float v[64];
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(buf) + t;        // elements 8 t + 512 i + e
+      const uint4* sm = reinterpret_cast<const uint4*>(smask) + t;
 #pragma unroll
-    for (int g = 0; g < 16; ++g)
-      *reinterpret_cast<float4*>(tr + 64 * t + 4 * (g ^ (t & 15))) =
-          make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-    team_sync(team);
-#pragma unroll
-    for (int k = 0; k < 64; ++k) v[k] = tr[64 * k + 4 * ((t >> 2) ^ (k & 15)) + (t & 3)];
+      for (int k = 0; k < 8; ++k) {
+        uint4 w = src[64 * k];
+        const uint4 sg = sm[64 * k];
+        w.x ^= sg.x;
+        w.y ^= sg.y;
+        w.z ^= sg.z;
+        w.w ^= sg.w;
+        v[8 * k + 0] = __uint_as_float(w.x << 16);
+        v[8 * k + 1] = __uint_as_float(w.x & 0xFFFF0000u);
+        v[8 * k + 2] = __uint_as_float(w.y << 16);
+        v[8 * k + 3] = __uint_as_float(w.y & 0xFFFF0000u);
+        v[8 * k + 4] = __uint_as_float(w.z << 16);
+        v[8 * k + 5] = __uint_as_float(w.z & 0xFFFF0000u);
+        v[8 * k + 6] = __uint_as_float(w.w << 16);
+        v[8 * k + 7] = __uint_as_float(w.w & 0xFFFF0000u);
+      }
+    }
     fwht64(v);
-    // v[k] is output n = (t mod 8) + 8 k + 512 (t / 8)
+    team_sync(team);  // every thread has read the row: the slot becomes the transpose buffer
+    float* tr = reinterpret_cast<float*>(buf);  // 32 matrix rows of 64 fp32, granule g of row a at g ^ (a mod 16)
+    float w[64];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if ((t >> 5) == h) {
+        const int a = t & 31;
+#pragma unroll
+        for (int g = 0; g < 16; ++g)
+          *reinterpret_cast<float4*>(tr + 64 * a + 4 * (g ^ (a & 15))) =
+              make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+      }
+      team_sync(team);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) w[32 * h + k] = tr[64 * k + 4 * ((t >> 2) ^ (k & 15)) + (t & 3)];
+      team_sync(team);
+    }
+    fwht64(w);
+    // w[k] is output n = (t mod 8) + 8 k + 512 (t / 8)
     if (MODE == kModeF32) {
       float* orow = p.out_f32 + row * p.ldo + (t & 7) + 512 * (t >> 3);
 #pragma unroll
-      for (int k = 0; k < 64; ++k) orow[8 * k] = v[k] * 0.015625f;
-      team_sync(team);  // every column read is done before the next row's writes
-      continue;
-    }
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 64; k += 4) {
-      a0 = fmaxf(a0, fabsf(v[k]));
-      a1 = fmaxf(a1, fabsf(v[k + 1]));
-      a2 = fmaxf(a2, fabsf(v[k + 2]));
-      a3 = fmaxf(a3, fabsf(v[k + 3]));
-    }
-    float a = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-    if (lane == 0) slots[t >> 5] = a;
-    team_sync(team);
-    const float amax = fmaxf(slots[0], slots[1]) * 0.015625f;  // max |x~| (x~ = H x / 64, exact scaling)
-    const float qmax = MODE == kModeInt4 ? 7.0f : p.qmax;
-    const float rr = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.0f;
-    const float cr = rr * 0.015625f;
-#pragma unroll
-    for (int k = 0; k < 64; k += 2) {
-      const float2 q = __ffma2_rn(make_float2(v[k], v[k + 1]), make_float2(cr, cr),
-                                  make_float2(kRoundMagic, kRoundMagic));
-      cb[64 * k + (t ^ (8 * (k >> 3)))] = (uint8_t)__float_as_uint(q.x);
-      cb[64 * (k + 1) + (t ^ (8 * ((k + 1) >> 3)))] = (uint8_t)__float_as_uint(q.y);
-    }
-    team_sync(team);
-    // outputs 64 t + 8 r + e sit at a = 8 (t mod 8) + r, b = 8 (t / 8) + e
-    uint2 c[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      c[r] = *reinterpret_cast<const uint2*>(cb + 64 * (8 * (t & 7) + r) + 8 * ((t >> 3) ^ (t & 7)));
-    if (MODE == kModeInt4) {
-      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 2048 + 32 * t);
-      dst[0] = make_uint4(nibbles_of(c[0].x, c[0].y), nibbles_of(c[1].x, c[1].y), nibbles_of(c[2].x, c[2].y),
-                          nibbles_of(c[3].x, c[3].y));
-      dst[1] = make_uint4(nibbles_of(c[4].x, c[4].y), nibbles_of(c[5].x, c[5].y), nibbles_of(c[6].x, c[6].y),
-                          nibbles_of(c[7].x, c[7].y));
+      for (int k = 0; k < 64; ++k) orow[8 * k] = w[k] * 0.015625f;
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 4096 + 64 * t);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(c[2 * i].x, c[2 * i].y, c[2 * i + 1].x, c[2 * i + 1].y);
+      for (int k = 0; k < 64; k += 4) {
+        a0 = fmaxf(a0, fabsf(w[k]));
+        a1 = fmaxf(a1, fabsf(w[k + 1]));
+        a2 = fmaxf(a2, fabsf(w[k + 2]));
+        a3 = fmaxf(a3, fabsf(w[k + 3]));
+      }
+      float am = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      if (lane == 0) slot_max[t >> 5] = am;
+      team_sync(team);
+      const float amax = fmaxf(slot_max[0], slot_max[1]) * 0.015625f;  // max |x~| (x~ = H x / 64, exact scaling)
+      const float qmax = MODE == kModeInt4 ? 7.0f : p.qmax;
+      const float rr = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.0f;
+      const float cr = rr * 0.015625f;
+      uint8_t* cb = buf;  // [a][b] code bytes, 8-byte group g of row a at g ^ (a / 8)
+#pragma unroll
+      for (int k = 0; k < 64; k += 2) {
+        const float2 q = __ffma2_rn(make_float2(w[k], w[k + 1]), make_float2(cr, cr),
+                                    make_float2(kRoundMagic, kRoundMagic));
+        cb[64 * k + (t ^ (8 * (k >> 3)))] = (uint8_t)__float_as_uint(q.x);
+        cb[64 * (k + 1) + (t ^ (8 * ((k + 1) >> 3)))] = (uint8_t)__float_as_uint(q.y);
+      }
+      team_sync(team);
+      // outputs 64 t + 8 r + e sit at a = 8 (t mod 8) + r, b = 8 (t / 8) + e
+      uint2 c[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        c[r] = *reinterpret_cast<const uint2*>(cb + 64 * (8 * (t & 7) + r) + 8 * ((t >> 3) ^ (t & 7)));
+      if (MODE == kModeInt4) {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 2048 + 32 * t);
+        dst[0] = make_uint4(nibbles_of(c[0].x, c[0].y), nibbles_of(c[1].x, c[1].y), nibbles_of(c[2].x, c[2].y),
+                            nibbles_of(c[3].x, c[3].y));
+        dst[1] = make_uint4(nibbles_of(c[4].x, c[4].y), nibbles_of(c[5].x, c[5].y), nibbles_of(c[6].x, c[6].y),
+                            nibbles_of(c[7].x, c[7].y));
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 4096 + 64 * t);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(c[2 * k].x, c[2 * k].y, c[2 * k + 1].x, c[2 * k + 1].y);
+      }
+      if (t == 0) p.scales_f32[row] = __fdiv_rn(amax, qmax);
     }
-    if (t == 0) p.scales_f32[row] = __fdiv_rn(amax, qmax);
+    team_sync(team);  // the slot and the team's max slots are free again
+    if (t == 0 && i + S < nloc) {  // refill: the next row this slot serves (the same team's)
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bars[sl], (unsigned)kF4kRowBytes);
+      bulk_g2s(buf, p.x + (row + S) * p.sS, (unsigned)kF4kRowBytes, &bars[sl]);
+      issued[sl] += 1;
+    }
+  }
+  __syncthreads();
+  // after a timed-out wait, let this CTA's own copies in flight land before it exits
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int sl = 0; sl < S; ++sl)
+      if (issued[sl] > 0) (void)mbar_wait_bounded(&bars[sl], (issued[sl] - 1) & 1);
   }
 }
 
@@ -1308,8 +1480,8 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
     float v[128];
     load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
     fwht_block_diag<LOGB>(v);
-    quant_nvfp4_store<PERM>(v, c, g, inv6g, ck.mchi, ck.mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                            p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+    quant_nvfp4_store<PERM, LOGB == 0>(v, c, g, inv6g, ck.mchi, ck.mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
+                                       p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
   }
 }
 

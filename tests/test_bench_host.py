@@ -68,3 +68,14 @@ def test_traffic_dropped_when_sources_changed(monkeypatch):
 def test_job_rate_and_rank_max():
     assert bench.job_rate(1000, 4, 2.0) == pytest.approx(2_000_000)
     assert list(bench.max_over_ranks([1.0, 3.0])) == [1.0, 3.0]
+
+
+def test_reference_arm_config_matches_the_default_run():
+    """With the default --workload all, both arms print the headline's config
+    (down_proj), including the list of the other measured configurations."""
+    import argparse
+    args = argparse.Namespace(workload="all", y_dtype="bf16")
+    cfg = bench.workload_config(args, bench.HEADLINE)
+    assert cfg["workload"] == "down_proj_int4"
+    assert cfg["also_measured"] == list(bench.ALSO_MEASURED)
+    assert "also_measured" not in bench.workload_config(args, "q_proj_int4")
