@@ -228,6 +228,14 @@ class Workload:
             self.wqs = [None if wq is None else tuple(None if t is None else t.clone() for t in wq)
                         for _ in range(self.R)]
             self.wq = self.wqs[0]
+            # INT4 weights also in the byte layout (the same codes one per byte), for the
+            # W4A4 GEMM that reads them without widening
+            self.wqs_bytes = None
+            if self.fmt == "int4":
+                w = syn.weights(name, device=device)
+                wb = rq.prepare_weights(w, self.signs, self.block, "int4_bytes")
+                del w
+                self.wqs_bytes = [tuple(None if t is None else t.clone() for t in wb) for _ in range(self.R)]
             m, k, n = c["M"], c["K"], c["N"]
             self.xq_outs = [rq._alloc_quant_outputs(m, k, rq._fmt(self.fmt), device) for _ in range(self.R)]
             self.xq_out = self.xq_outs[0]
@@ -301,6 +309,11 @@ class Workload:
         if self.fmt in ("int8", "int6"):
             return self.rq.int_gemm(xq, self.fmt, self.wqs[r], self.wfmt, self.y_dtype, y=self.ys[r])
         return self.rq.w4a4_gemm(xq, self.wqs[r], self.fmt, self.y_dtype, y=self.ys[r])
+
+    def gemm_bytes(self, xq, i=0):
+        """The same W4A4 product against the weights' INT4 codes in the byte layout."""
+        r = i % self.R
+        return self.rq.int_gemm(xq, "int4", self.wqs_bytes[r], "int4_bytes", self.y_dtype, y=self.ys[r])
 
     def result(self):
         if self.kvdec:
@@ -620,6 +633,7 @@ def run_workload(name, args, rq, dev, dist, world, rank, local, cpu_scale=1.0):
     # per-kernel averages for the roofline: each kernel alone, K launches the same way
     ev_q = timed(lambda i: wl.quant(i))
     ev_g = timed(lambda i: wl.gemm(wl.slot_codes(i), i)) if wl.gemm_launches() else None
+    ev_gb = timed(lambda i: wl.gemm_bytes(wl.slot_codes(i), i)) if getattr(wl, "wqs_bytes", None) else None
     torch.cuda.synchronize()
     clk = clocks.stop()
     rq.get_device_error()
@@ -676,6 +690,14 @@ def run_workload(name, args, rq, dev, dist, world, rank, local, cpu_scale=1.0):
         roof_g["frac"] = round(roof_g["achieved"] / peak_t, 4)
         out["gemm"] = {"value": round(tops, 2), "unit": "TOPS", "ms": round(g_mean_ms, 5),
                        "frac_of_peak": roof_g["frac"]}
+        if ev_gb is not None:
+            gb_ms = max_over_ranks([ev_gb[0].elapsed_time(ev_gb[1])], dist, dev)[0] / K
+            gb_tops = job_rate(wl.gemm_ops, world, gb_ms) / 1e12
+            out["gemm_int4_bytes"] = {
+                "value": round(gb_tops, 2), "unit": "TOPS", "ms": round(gb_ms, 5),
+                "frac_of_peak": round(wl.gemm_ops / (gb_ms * 1e-3) / 1e12 / peak_t, 4),
+                "kernel": "gemm_int_2sm_ts_kernel<A4, W8>",
+                "weights": "the same INT4 codes and scales, one code per byte (twice the packed weight memory)"}
         dominant = roof_g if g_mean_ms >= q_mean_ms else roof_q
         out["roofline"] = dominant
         out["roofline_hadamard_quant"] = roof_q

@@ -71,7 +71,8 @@ typedef enum {
   RQ_MXFP4 = 2, /* E2M1, one E8M0 (power-of-two) scale per 32 values */
   RQ_INT8 = 3,  /* symmetric 8-bit, one int8 code per byte, one fp32 scale per row */
   RQ_INT6 = 4,  /* symmetric 6-bit (codes in [-31, 31]), one int8 byte each, one fp32 scale per row */
-  RQ_INT4_ASYM = 5 /* asymmetric 4-bit per group of 128 along K: fp16 (scale, zero) per group */
+  RQ_INT4_ASYM = 5, /* asymmetric 4-bit per group of 128 along K: fp16 (scale, zero) per group */
+  RQ_INT4_BYTES = 6 /* the RQ_INT4 codes and scales, one int8 byte per code (the layout the integer MMA reads) */
 } rq_format;
 
 typedef enum {
@@ -143,6 +144,11 @@ RQ_API size_t rq_workspace_bytes(rq_format fmt);
  *               codes_dev  int8 [M, K], scales_dev float [M]:
  *               s = amax/qmax with qmax = 127 / 31; q = rint(x~/s).  gscale_dev
  *               and workspace_dev are unused (may be NULL).
+ *             RQ_INT4_BYTES (a weight layout for rq_int_gemm):
+ *               codes_dev  int8 [M, K], scales_dev float [M]: exactly the
+ *               RQ_INT4 codes and scales, one code per byte instead of two.
+ *               Twice the memory of packed INT4; the GEMM then reads the
+ *               codes as int8 MMA operands with no widening.
  *             RQ_INT4_ASYM (per-group asymmetric INT4, "SpinQuant", field
  *             "Activation scheme"; block 16, 32 or 128):
  *               codes_dev  uint8 [M, K/2], unsigned nibbles q in [0, 15],
@@ -207,8 +213,11 @@ RQ_API rq_status rq_w4a4_gemm(const uint8_t* xcodes_dev, const void* xscales_dev
  *        (xcodes int8 [M, K]); xscales float [M].
  *  wfmt  the same for W [N, K]; wscales float [N].
  *  Supported pairs (xfmt, wfmt): (INT4, INT4) -- the rq_w4a4_gemm INT4 path --
- *  (INT6/INT8, INT4) and (INT6/INT8, INT6/INT8).  (INT4, INT6/INT8) returns
- *  RQ_ERR_UNSUPPORTED_SHAPE.
+ *  (INT4, INT4_BYTES) -- the same W4A4 product with the weights' INT4 codes
+ *  stored one per byte (wcodes int8 [N, K], from rq_prepare_weights with
+ *  RQ_INT4_BYTES), which the two-SM kernel feeds to the tensor cores without
+ *  widening them --, (INT6/INT8, INT4) and (INT6/INT8, INT6/INT8).
+ *  (INT4, INT6/INT8) returns RQ_ERR_UNSUPPORTED_SHAPE.
  *  acc = sum_k qx[m,k] qw[n,k] exactly in int32 (|acc| < 2^31 for K <= 65536);
  *  Y = float(acc) * sx[m] * sw[n] (float(acc) rounds to nearest above 2^24).
  *  Codes 16-byte aligned, xscales 4-byte and wscales 16-byte aligned; K a

@@ -132,12 +132,11 @@ rq_status launch_block(RotParams p, cudaStream_t st, bool pdl = true) {
   return launch_rotate<MODE, 0, 7>(p, st, pdl);
 }
 
-// K = 4096: the 64 x 64 two-pass kernel, two CTAs of four row teams per SM,
-// each CTA's rows staged in up to kF4kSlots shared-memory slots (all of them
-// when they fit, else a ring whose depth is a multiple of the team count).
+// K = 4096: the 64 x 64 two-pass kernel, one CTA of eight row teams per SM,
+// each CTA's rows staged through a ring of up to kF4kSlots shared-memory slots.
 template <int MODE>
 rq_status launch_full4096(RotParams p, cudaStream_t st) {
-  const int64_t cap = 2 * (int64_t)num_sms_of_current_device();
+  const int64_t cap = (int64_t)num_sms_of_current_device();
   const int64_t grid = p.rows < cap ? p.rows : cap;
   const int64_t rpc = (p.rows + grid - 1) / grid;  // the most rows any CTA takes
   const int slots = rpc <= kF4kSlots ? (int)rpc : kF4kSlots;
@@ -171,21 +170,24 @@ rq_status launch_nvfp4_resident_b(RotParams p, cudaStream_t st) {
     return RQ_ERR_UNSUPPORTED_SHAPE;
   const int sms = num_sms_of_current_device();
   const int64_t rpc = (p.rows + sms - 1) / sms;
-  const size_t smem = (size_t)rpc * p.K * 2 + (size_t)p.nb * 64 * 4 + 32;
+  const size_t smem = (size_t)rpc * p.K * 2 + (size_t)p.nb * 64 * 4 + 48;
   if (smem > kSmemBudget) return RQ_ERR_UNSUPPORTED_SHAPE;
+  // the rotated values wait in tensor memory between the passes when a CTA's
+  // 128-value units fit its 512 columns x 128 lanes
+  int stash = rpc * p.nb <= kResStashUnits ? 1 : 0;
   const int grid = (int)((p.rows + rpc - 1) / rpc);
   if (!ensure_smem(reinterpret_cast<const void*>(rotate_nvfp4_resident_kernel<LOGB>))) return RQ_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_nvfp4_resident_kernel<LOGB>, 384, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_nvfp4_resident_kernel<LOGB>, kResThreads, smem) !=
           cudaSuccess ||
       per_sm < 1 || grid > per_sm * sms)
     return RQ_ERR_UNSUPPORTED_SHAPE;
   p.nvfp4_dynamic = 1;
   int rows_per_cta = (int)rpc;
-  void* args[] = {&p, &rows_per_cta};
+  void* args[] = {&p, &rows_per_cta, &stash};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(384);
+  cfg.blockDim = dim3(kResThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -249,10 +251,10 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
   rq_status s = check_rotation_args(X, M, K, ldx, signs, block);
   if (s != RQ_OK) return s;
   if (fmt != RQ_INT4 && fmt != RQ_NVFP4 && fmt != RQ_MXFP4 && fmt != RQ_INT8 && fmt != RQ_INT6 &&
-      fmt != RQ_INT4_ASYM)
+      fmt != RQ_INT4_ASYM && fmt != RQ_INT4_BYTES)
     return RQ_ERR_INVALID_ARG;
   if (gmode != RQ_SCALE_DYNAMIC && gmode != RQ_SCALE_STATIC) return RQ_ERR_INVALID_ARG;
-  const bool int_fmt = fmt == RQ_INT4 || fmt == RQ_INT8 || fmt == RQ_INT6;
+  const bool int_fmt = fmt == RQ_INT4 || fmt == RQ_INT8 || fmt == RQ_INT6 || fmt == RQ_INT4_BYTES;
   if (!int_fmt && block == 0) return RQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return RQ_OK;
   if (!codes || !scales) return RQ_ERR_INVALID_ARG;
@@ -279,9 +281,11 @@ rq_status rotate_quantize_impl(const void* X, int64_t M, int64_t K, int64_t ldx,
     p.kv_scale = static_cast<__half*>(scales);
     return launch_block<kModeAsym4>(p, st);
   }
-  if (fmt == RQ_INT8 || fmt == RQ_INT6) {
+  if (fmt == RQ_INT8 || fmt == RQ_INT6 || fmt == RQ_INT4_BYTES) {
+    // one code per byte; RQ_INT4_BYTES is the INT4 rule (qmax 7, the same
+    // reciprocal and rounding as the packed INT4 kernels) in this layout
     p.scales_f32 = static_cast<float*>(scales);
-    p.qmax = fmt == RQ_INT8 ? 127.0f : 31.0f;
+    p.qmax = fmt == RQ_INT8 ? 127.0f : (fmt == RQ_INT6 ? 31.0f : 7.0f);
     if (block == 0) return launch_full<kModeInt8>(p, st);
     return launch_block<kModeInt8>(p, st);
   }

@@ -852,9 +852,9 @@ struct I3 {
   static constexpr int StgA = A8 ? 128 * 128 : 128 * 64;  // A tile per k-tile: int8 or packed nibbles
   static constexpr int StgB = W8 ? 0 : 128 * 64;          // packed W (W8: straight into the operand ring)
   static constexpr int Stg = A8 ? 4 : 6;                  // staging depth within 227 KB
-  static constexpr int Ops = (A8 && W8) ? 6 : 4;           // operand ring: B in smem, A in TMEM (32 columns each)
+  static constexpr int Ops = W8 ? 6 : 4;                   // operand ring: B in smem, A in TMEM (32 columns each)
   static constexpr int BArr = W8 ? 0 : kI3BWarps;         // B converter arrivals per k-tile and CTA
-  static constexpr int Shift = A8 ? (W8 ? 0 : 4) : 8;
+  static constexpr int Shift = A8 ? (W8 ? 0 : 4) : (W8 ? 4 : 8);  // A4 x W8: 16 qx against the int8 codes of W
   static constexpr size_t Smem = 1024 + (size_t)Ops * kI3OpB + (size_t)Stg * (StgA + StgB) + 2 * kEpiStage + 256;
   static_assert(Smem <= 232448, "fits the 227 KB of shared memory a CTA may use");
 };
@@ -1357,10 +1357,11 @@ inline rq_status int_gemm_dispatch(const uint8_t* xc, const float* xs, rq_format
                                    const float* ws, rq_format wfmt, int64_t M, int64_t N, int64_t K, void* Y,
                                    int64_t ldy, rq_out out, cudaStream_t st) {
   auto is_int = [](rq_format f) { return f == RQ_INT4 || f == RQ_INT6 || f == RQ_INT8; };
-  if (!is_int(xfmt) || !is_int(wfmt)) return RQ_ERR_INVALID_ARG;
+  const bool a4w8 = xfmt == RQ_INT4 && wfmt == RQ_INT4_BYTES;  // W4A4 with the weight codes one per byte
+  if (!a4w8 && (!is_int(xfmt) || !is_int(wfmt))) return RQ_ERR_INVALID_ARG;
   if (xfmt == RQ_INT4 && wfmt == RQ_INT4)
     return gemm_dispatch(xc, xs, nullptr, wc, ws, nullptr, M, N, K, RQ_INT4, Y, ldy, out, st);
-  if (xfmt == RQ_INT4) return RQ_ERR_UNSUPPORTED_SHAPE;  // 4-bit activations with wider weights
+  if (xfmt == RQ_INT4 && !a4w8) return RQ_ERR_UNSUPPORTED_SHAPE;  // 4-bit activations with wider weights
   const bool w8 = wfmt != RQ_INT4;
   if (M < 0 || N < 0 || K <= 0 || ldy < N) return RQ_ERR_INVALID_ARG;
   if (out != RQ_OUT_F32 && out != RQ_OUT_BF16 && out != RQ_OUT_I32_ACC) return RQ_ERR_INVALID_ARG;
@@ -1384,7 +1385,7 @@ inline rq_status int_gemm_dispatch(const uint8_t* xc, const float* xs, rq_format
   p.ldy = ldy;
   p.out = (int)out;
   p.vec_ok = ((reinterpret_cast<uintptr_t>(Y) % 16) == 0 && (ldy * (int64_t)esz) % 16 == 0) ? 1 : 0;
-  p.acc_shift = w8 ? I3<true, true>::Shift : I3<true, false>::Shift;
+  p.acc_shift = a4w8 ? I3<false, true>::Shift : (w8 ? I3<true, true>::Shift : I3<true, false>::Shift);
   p.tiles_m = (int)((M + 255) / 256);
   p.tiles_n = (int)((N + kBN - 1) / kBN);
   p.num_tiles = p.tiles_m * p.tiles_n;
@@ -1393,7 +1394,11 @@ inline rq_status int_gemm_dispatch(const uint8_t* xc, const float* xs, rq_format
 
   CUtensorMap tx, tw, ty;
   std::memset(&ty, 0, sizeof(ty));
-  if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return RQ_ERR_CUDA;
+  if (a4w8) {  // packed X nibbles, staged 64B-swizzled for the A converters
+    if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return RQ_ERR_CUDA;
+  } else if (!make_tmap_u8(&tx, xc, (uint64_t)M, (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    return RQ_ERR_CUDA;
+  }
   if (w8) {
     if (!make_tmap_u8(&tw, wc, (uint64_t)N, (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return RQ_ERR_CUDA;
   } else {
@@ -1401,7 +1406,13 @@ inline rq_status int_gemm_dispatch(const uint8_t* xc, const float* xs, rq_format
   }
   p.tma_store = (out == RQ_OUT_BF16 && p.vec_ok) ? 1 : 0;
   if (p.tma_store && !make_tmap_y_bf16(&ty, Y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy)) return RQ_ERR_CUDA;
-  if (w8) {
+  if (a4w8) {
+    if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<false, true>),
+                          (int)I3<false, true>::Smem))
+      return RQ_ERR_CUDA;
+    (void)launch_pdl(gemm_int_2sm_ts_kernel<false, true>, dim3(grid2), dim3(kI3Threads), I3<false, true>::Smem, st, tx,
+                     tw, ty, p);
+  } else if (w8) {
     if (!gemm_ensure_smem(reinterpret_cast<const void*>(gemm_int_2sm_ts_kernel<true, true>),
                           (int)I3<true, true>::Smem))
       return RQ_ERR_CUDA;

@@ -562,10 +562,21 @@ __device__ __forceinline__ const uint8_t* row_src(const RotParams& p, int64_t ro
   return p.x + (bh / p.H) * p.sB + (bh % p.H) * p.sH + t * p.sS;
 }
 
-// True when the fp16 rounding of v could change within +-band, i.e. v lies
-// that close to the midpoint between two neighbouring fp16 values.
-__device__ __forceinline__ bool near_fp16_midpoint(float v, float band) {
-  return __half2float(__float2half_rn(v - band)) != __half2float(__float2half_rn(v + band));
+// True when v may lie within 2^-LOG2BAND of `am` (am >= |v| > 0 in practice)
+// of a midpoint between two neighbouring fp16 values, so that an error of that
+// size could change its fp16 rounding.  Integer arithmetic on the fp32 bits:
+// in the fp16 normal range a midpoint is where the 13 fraction bits fp16 drops
+// read 0x1000, and 2^-LOG2BAND am is at most 2^(23 - LOG2BAND + 1 + ea - ev)
+// units in the last place of v (ea, ev the exponent fields).  Values outside
+// the fp16 normal range are reported as near (the caller then decides exactly).
+template <int LOG2BAND>
+__device__ __forceinline__ bool near_fp16_midpoint(float v, float am) {
+  const uint32_t b = __float_as_uint(v) & 0x7FFFFFFFu;
+  const int ev = (int)(b >> 23), ea = (int)((__float_as_uint(am) >> 23) & 0xFFu);
+  if (ev < 127 - 14 || ev > 127 + 15) return true;
+  const int d = (int)(b & 0x1FFFu) - 0x1000;
+  const int span = ea - ev;  // >= 0 when am >= |v|
+  return span > 10 || (d < 0 ? -d : d) <= ((1 << (24 - LOG2BAND)) << (span > 0 ? span : 0));
 }
 
 // 1 / sqrt(2^LOGB) in fp64 (LOGB = 0, 4, 5, 7).
@@ -633,27 +644,77 @@ __device__ __forceinline__ void rotated_group_f64(const uint8_t* src, const uint
   hi = mx;
 }
 
+// Where one group of 128 channels lives: its bf16 inputs (global), its sign
+// masks (shared) and its stored codes, scale and zero (global).
+struct KvGroup {
+  const uint8_t* src;
+  const uint32_t* smask;
+  uint8_t* codes;
+  __half* scale;
+  __half* zero;
+};
+
+// The second look of quant_kv4_store: for each lane L in `pending` the warp
+// rotates L's group in fp64 (rotated_group_f64) and, where the fp16 roundings
+// of the exact min and (max - min)/15 differ from the ones stored for that
+// group, rewrites its scale, zero and codes from the fp64 values.  Called by
+// every lane of the warp; group_of(L) gives lane L's group and is evaluated
+// (by the whole warp) only for the pending lanes, so none of its address
+// arithmetic runs in the common case.
+template <int LOGB, typename GroupFn>
+__device__ __forceinline__ void kv4_second_look(unsigned pending, GroupFn group_of) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();  // this warp's stores of its groups come before any rewrite below
+  while (pending) {
+    const int L = __ffs(pending) - 1;
+    pending &= pending - 1;
+    const KvGroup gr = group_of(L);
+    const uint32_t szbits = ((uint32_t)__half_as_ushort(*gr.scale) << 16) | __half_as_ushort(*gr.zero);
+    double y[4], dlo, dhi;
+    rotated_group_f64<LOGB>(gr.src, gr.smask, lane, y, dlo, dhi);
+    const __half zx = __double2half(dlo);
+    const __half sx = __double2half((dhi - dlo) / 15.0);
+    const uint32_t xbits = ((uint32_t)__half_as_ushort(sx) << 16) | __half_as_ushort(zx);
+    if (xbits != szbits) {  // the same in every lane
+      const double sd = (double)__half2float(sx), zd = (double)__half2float(zx);
+      uint32_t nib = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int q = 0;
+        if (sd > 0.0) q = min(max(__double2int_rn((y[e] - zd) / sd), 0), 15);
+        nib |= (uint32_t)q << (4 * e);
+      }
+      __syncwarp();  // every lane has read the stored scale and zero
+      *reinterpret_cast<uint16_t*>(gr.codes + 2 * lane) = (uint16_t)nib;  // channels 4 lane .. 4 lane + 3
+      if (lane == 0) {
+        *gr.scale = sx;
+        *gr.zero = zx;
+      }
+    }
+  }
+}
+
 // KV4 and per-group asymmetric INT4: asymmetric quantization of one group of
 // 128 channels (true value = v * c * chi): z = min, s = (max - min)/15, both
 // stored as fp16, q = clamp(rint((x - z)/s), 0, 15).
 //
-// The fp32 butterflies leave the group's min and max within about 2^-23 of
-// its largest magnitude (measured; the bound of a 7-level summation is a few
-// times that), which can decide the fp16 rounding of z or s when either lies
-// that close to a midpoint between two fp16 values.  So after the group is
-// stored, the lanes for which that is possible (a band of 2^-20 of the
-// largest magnitude around z, 2^-22 around s: about 1 % of groups) have their
+// The fp32 butterflies leave the group's min within about 2^-23 of its
+// largest magnitude and (max - min)/15 within about 2^-25 (the largest errors
+// seen over 6e5 Gaussian and outlier groups; the bound of a 7-level summation
+// is a few times that), which can decide the fp16 rounding of z or s when
+// either lies that close to a midpoint between two fp16 values.  So after
+// the group is stored, the lanes for which that is possible (a band of at
+// least 2^-22 of the largest magnitude around z, 2^-24 around s, found from
+// the fp32 bits alone: about 0.3 % of groups) have their
 // group rotated again in fp64 by the whole warp (rotated_group_f64); where the
 // fp16 roundings of the exact min and scale differ from the stored ones (about
 // 2 groups in 10^4), the warp rewrites the group's z, s and codes from the
-// fp64 values.  Every lane of the warp must call this function together;
-// `valid` marks lanes that hold a real group (only they store), and `src_of()`
-// gives the group's global input address (called only by lanes that need the
-// second look).
-template <bool PERM, int LOGB, typename SrcFn>
-__device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, int m, int mo, bool valid,
-                                                SrcFn src_of, const uint32_t* smask_grp, uint8_t* dst_codes,
-                                                __half* dst_scale, __half* dst_zero) {
+// fp64 values (kv4_second_look).  This function stores the group (only where
+// `valid`) and returns whether this lane's group needs the second look; the
+// caller then runs kv4_second_look with the whole warp.
+template <bool PERM>
+__device__ __forceinline__ bool quant_kv4_store(const float (&v)[128], float c, int m, int mo, bool valid,
+                                                uint8_t* dst_codes, __half* dst_scale, __half* dst_zero) {
   float lo = 3.0e38f, hi = -3.0e38f;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -685,6 +746,13 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
   // whether clamping to [0, 15] can be needed for this vector.
   const float tlo = fmaf(lo, inv, off), thi = fmaf(hi, inv, off);
   const bool need_clamp = !(tlo > -0.5f && thi < 15.5f);
+  // whether z or s lies near an fp16 midpoint (the second look, after the stores)
+  const float am = fmaxf(fabsf(lo), fabsf(hi));
+  const bool unsure = valid && (near_fp16_midpoint<22>(lo, am) || near_fp16_midpoint<24>(s, am));
+  if (valid) {
+    *dst_scale = s_h;
+    *dst_zero = z_h;
+  }
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
     uint32_t w[4];
@@ -709,52 +777,7 @@ __device__ __forceinline__ void quant_kv4_store(const float (&v)[128], float c, 
     }
     if (valid) store_words4<PERM>(dst_codes, j4, mo, w[0], w[1], w[2], w[3]);
   }
-  if (valid) {
-    *dst_scale = s_h;
-    *dst_zero = z_h;
-  }
-  // the second look at groups whose z or s lies near an fp16 midpoint
-  const float am = fmaxf(fabsf(lo), fabsf(hi));
-  const bool unsure = valid && (near_fp16_midpoint(lo, am * 0x1p-20f) || near_fp16_midpoint(s, am * 0x1p-22f));
-  unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
-  if (pending) {
-    const int lane = threadIdx.x & 31;
-    const uint8_t* src = unsure ? src_of() : nullptr;
-    const uint32_t szbits = ((uint32_t)__half_as_ushort(s_h) << 16) | __half_as_ushort(z_h);
-    __syncwarp();  // this warp's stores above come before any rewrite below
-    while (pending) {
-      const int L = __ffs(pending) - 1;
-      pending &= pending - 1;
-      const auto bcast = [&](const void* ptr) {
-        return (uintptr_t)__shfl_sync(0xFFFFFFFFu, (unsigned long long)reinterpret_cast<uintptr_t>(ptr), L);
-      };
-      const uint8_t* srcL = reinterpret_cast<const uint8_t*>(bcast(src));
-      const uint32_t* mskL = reinterpret_cast<const uint32_t*>(bcast(smask_grp));
-      double y[4], dlo, dhi;
-      rotated_group_f64<LOGB>(srcL, mskL, lane, y, dlo, dhi);
-      const __half zx = __double2half(dlo);
-      const __half sx = __double2half((dhi - dlo) / 15.0);
-      const uint32_t xbits = ((uint32_t)__half_as_ushort(sx) << 16) | __half_as_ushort(zx);
-      if (xbits != __shfl_sync(0xFFFFFFFFu, szbits, L)) {  // the same in every lane
-        uint8_t* dstL = reinterpret_cast<uint8_t*>(bcast(dst_codes));
-        const double sd = (double)__half2float(sx), zd = (double)__half2float(zx);
-        uint32_t nib = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int q = 0;
-          if (sd > 0.0) q = min(max(__double2int_rn((y[e] - zd) / sd), 0), 15);
-          nib |= (uint32_t)q << (4 * e);
-        }
-        *reinterpret_cast<uint16_t*>(dstL + 2 * lane) = (uint16_t)nib;  // channels 4 lane .. 4 lane + 3
-        __half* dsL = reinterpret_cast<__half*>(bcast(dst_scale));
-        __half* dzL = reinterpret_cast<__half*>(bcast(dst_zero));
-        if (lane == 0) {
-          *dsL = sx;
-          *dzL = zx;
-        }
-      }
-    }
-  }
+  return unsure;
 }
 
 template <bool PERM = false>
@@ -1072,13 +1095,34 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
         if (valid) store_f32_block<PERM>(v, c, mchi, mo, p.out_f32 + row * p.ldo + (size_t)b * 128);
       } else if (MODE == kModeAmax) {
         if (valid) amax_acc = fmaxf(amax_acc, absmax128(v) * c);
-      } else if (MODE == kModeKv4) {
-        quant_kv4_store<false, 7>(v, c, m, 0, valid, [&]() { return row_src(p, row); }, smask, p.codes + row * 64,
-                                  p.kv_scale + row, p.kv_zero + row);
-      } else if (MODE == kModeAsym4) {
-        __half* sz = p.kv_scale + 2 * (row * nb + b);
-        quant_kv4_store<PERM, LOGB>(v, c, mchi, mo, valid, [&]() { return row_src(p, row) + (size_t)b * 256; },
-                                    smask + bl * 64, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
+      } else if (MODE == kModeKv4 || MODE == kModeAsym4) {
+        constexpr bool KV = MODE == kModeKv4;
+        __half* sz = KV ? p.kv_scale + row : p.kv_scale + 2 * (row * nb + b);
+        const bool unsure = KV ? quant_kv4_store<false>(v, c, m, 0, valid, p.codes + row * 64, sz, p.kv_zero + row)
+                               : quant_kv4_store<PERM>(v, c, mchi, mo, valid,
+                                                       p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
+        const unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
+        if (pending) {
+          // lane L's row and block, by the same mapping as this thread's
+          kv4_second_look<KV ? 7 : LOGB>(pending, [&](int L) {
+            const int rL = RPS > 1 ? L / nb : 0;
+            const int bL = RPS > 1 ? L - rL * nb : wig * 32 + L;
+            const int64_t rowL = r0 + rL;
+            KvGroup gr;
+            gr.src = row_src(p, rowL) + (size_t)bL * 256;
+            gr.smask = smask + bL * 64;
+            if (KV) {
+              gr.codes = p.codes + rowL * 64;
+              gr.scale = p.kv_scale + rowL;
+              gr.zero = p.kv_zero + rowL;
+            } else {
+              gr.codes = p.codes + rowL * (p.K / 2) + (size_t)bL * 64;
+              gr.scale = p.kv_scale + 2 * (rowL * nb + bL);
+              gr.zero = gr.scale + 1;
+            }
+            return gr;
+          });
+        }
       }
     } else {
       constexpr int NB = NBF ? NBF : 1;
@@ -1146,36 +1190,37 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
 // the element index n, so the bits can be transformed in any grouping.  The
 // row is read as a 64 x 64 matrix X[a][b] with a = bits 3..8 of n and
 // b = bits 0..2 and 9..11: H_64 along b in every matrix row, then H_64 along a
-// in every column.  A team of 64 threads (two warps) owns one row at a time.
+// in every column.  A team of 64 threads (two warps) owns one row at a time;
+// eight teams per CTA, one CTA per SM.
 //
 // Staging: each CTA takes a contiguous run of rows (M / grid, rounded down or
 // up) and, at kernel start, issues one bulk copy (cp.async.bulk, local memory,
-// no multicast) per row into a slot of shared memory -- as many rows as fit,
-// up to kF4kSlots -- and builds its sign table while they are in flight; so
-// every CTA's reads are in the memory system from the start instead of one
-// row per team at a time.  Rows go to the CTA's four teams in turn; with more
-// rows than slots the slots form a ring (kF4kSlots is a multiple of the team
-// count, so a slot always serves the same team), and a team refills its slot
-// once it has finished with the row.
+// no multicast) per row into a ring of up to kF4kSlots shared-memory slots,
+// building its sign table while they are in flight; so every CTA's reads are
+// in the memory system from the start instead of one row per team at a time.
+// Local row i goes to team i mod 8 and slot i mod S; once its team has read
+// it into registers, the slot is refilled with row i + S (whichever team
+// takes that one waits on the slot's mbarrier).
 //
 // Per row: thread a reads matrix row a (elements 8 a + 512 i + e) from the
-// slot, signs and transforms it; the slot then holds, in two halves of 32
-// matrix rows, the fp32 transpose, and thread b transforms column b; the codes
-// of its outputs (a = 0..63, b) go back through the slot as bytes, and thread t
-// stores the codes of outputs 64 t .. 64 t + 63 with 16-byte stores.
-// Shared-memory granules are XOR-swizzled so that the row writes, column reads
-// and code transposes are free of bank conflicts (the code reads: two-way).
-// Two CTAs of four teams per SM; a team synchronises on its own named barrier
-// (1..4).
+// slot, signs and transforms it, and writes it to the team's fp32 transpose
+// buffer; after a team barrier, thread b transforms column b.  The codes of
+// its outputs (a = 0..63, b) go back through the team's code buffer as bytes,
+// and thread t stores the codes of outputs 64 t .. 64 t + 63 with 16-byte
+// stores.  Three team barriers per row (transpose, row max, codes).
+// Shared-memory granules are XOR-swizzled so that the row writes, column
+// reads and code transposes are free of bank conflicts (the code reads:
+// two-way).  A team synchronises on its own named barrier (1..8).
 // ---------------------------------------------------------------------------
-constexpr int kR64Teams = 4;
+constexpr int kR64Teams = 8;
 constexpr int kR64Threads = 64 * kR64Teams;
-constexpr int kF4kSlots = 12;                      // row slots per CTA (a multiple of kR64Teams)
+constexpr int kF4kSlots = 7;                        // row slots per CTA
 constexpr size_t kF4kRowBytes = 4096 * 2;
-static_assert(kF4kSlots % kR64Teams == 0, "a slot must always serve the same team");
+constexpr size_t kR64TeamBytes = 64 * 64 * 4 + 64 * 64 + 16;  // fp32 transpose | code bytes | row max slots
 __host__ __device__ constexpr size_t f4k_smem_bytes(int slots) {
-  // sign masks | row slots | mbarriers (one per slot) | per-slot issue counts | team max slots | abort flag
-  return 2048 * 4 + (size_t)slots * kF4kRowBytes + (size_t)slots * 8 + (size_t)slots * 4 + kR64Teams * 2 * 4 + 16;
+  // sign masks | team buffers | row slots | mbarriers (one per slot) | per-slot row tags | abort flag
+  return 2048 * 4 + kR64Teams * kR64TeamBytes + (size_t)slots * kF4kRowBytes + (size_t)slots * 8 +
+         (size_t)slots * 4 + 16;
 }
 
 __device__ __forceinline__ void team_sync(int team) {
@@ -1229,17 +1274,25 @@ __device__ __forceinline__ uint32_t nibbles_of(uint32_t w0, uint32_t w1) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const RotParams p, int slots) {
+__global__ void __launch_bounds__(kR64Threads, 1) rotate_full4096_kernel(const RotParams p, int slots) {
   griddep_wait();
   griddep_trigger();
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw);              // [2048] XOR masks, one per bf16 pair
-  uint8_t* rows = smem_raw + 2048 * 4;                                   // [slots][8 KB]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rows + (size_t)slots * kF4kRowBytes);
-  unsigned* issued = reinterpret_cast<unsigned*>(bars + slots);         // copies issued per slot
-  float* tmax = reinterpret_cast<float*>(issued + slots);                // [team][2]
-  int* abort_flag = reinterpret_cast<int*>(tmax + 2 * kR64Teams);
   const int team = threadIdx.x >> 6, t = threadIdx.x & 63, lane = threadIdx.x & 31;
+  uint8_t* tb = smem_raw + 2048 * 4 + (size_t)team * kR64TeamBytes;
+  float* tr = reinterpret_cast<float*>(tb);             // [a][b] fp32, 16-byte granule g of row a at g ^ (a mod 16)
+  uint8_t* cb = tb + 64 * 64 * 4;                       // [a][b] code bytes, 8-byte group g of row a at g ^ (a / 8)
+  float* slot_max = reinterpret_cast<float*>(cb + 64 * 64);
+  uint8_t* rows = smem_raw + 2048 * 4 + kR64Teams * kR64TeamBytes;  // [slots][8 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rows + (size_t)slots * kF4kRowBytes);
+  // the local row most recently issued into each slot.  Consecutive fills of a
+  // slot go to different teams, so an mbarrier parity alone cannot tell a team
+  // waiting for fill f from fill f - 2: a team first waits until the slot's
+  // tag names its row -- the copy is issued, so fill f - 1 has completed (its
+  // consumer issued this one) -- and only then for the fill's parity.
+  int* tags = reinterpret_cast<int*>(bars + slots);
+  int* abort_flag = tags + slots;
   // each CTA a contiguous run of M / grid rows (rounded down or up)
   const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
   const int nloc = (int)(((int64_t)blockIdx.x + 1) * p.rows / gridDim.x - r_begin);
@@ -1248,7 +1301,7 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&bars[i], 1);
-      issued[i] = 0;
+      tags[i] = i;
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -1259,19 +1312,29 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
       for (int i = 0; i < S; ++i) {
         mbar_arrive_expect_tx(&bars[i], (unsigned)kF4kRowBytes);
         bulk_g2s(rows + (size_t)i * kF4kRowBytes, p.x + (r_begin + i) * p.sS, (unsigned)kF4kRowBytes, &bars[i]);
-        issued[i] = 1;
       }
     }
   });
   __syncthreads();
 
-  float* slot_max = tmax + 2 * team;
 #pragma unroll 1
   for (int i = team; i < nloc; i += kR64Teams) {
     const int sl = i % S;
     const int64_t row = r_begin + i;
     uint8_t* buf = rows + (size_t)sl * kF4kRowBytes;
-    if (!team_all(mbar_wait_bounded(&bars[sl], (unsigned)((i / S) & 1)), team)) {
+    bool ok = true;
+    {
+      const long long t0 = clock64();
+      while (((volatile int*)tags)[sl] != i) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+          atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+          ok = false;
+          break;
+        }
+      }
+    }
+    ok = ok && mbar_wait_bounded(&bars[sl], (unsigned)((i / S) & 1));
+    if (!team_all(ok, team)) {
       if (t == 0) atomicOr(abort_flag, 1);
       break;
     }
@@ -1298,102 +1361,144 @@ __global__ void __launch_bounds__(kR64Threads, 2) rotate_full4096_kernel(const R
       }
     }
     fwht64(v);
-    team_sync(team);  // every thread has read the row: the slot becomes the transpose buffer
-    float* tr = reinterpret_cast<float*>(buf);  // 32 matrix rows of 64 fp32, granule g of row a at g ^ (a mod 16)
-    float w[64];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if ((t >> 5) == h) {
-        const int a = t & 31;
-#pragma unroll
-        for (int g = 0; g < 16; ++g)
-          *reinterpret_cast<float4*>(tr + 64 * a + 4 * (g ^ (a & 15))) =
-              make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-      }
-      team_sync(team);
-#pragma unroll
-      for (int k = 0; k < 32; ++k) w[32 * h + k] = tr[64 * k + 4 * ((t >> 2) ^ (k & 15)) + (t & 3)];
-      team_sync(team);
-    }
-    fwht64(w);
-    // w[k] is output n = (t mod 8) + 8 k + 512 (t / 8)
-    if (MODE == kModeF32) {
-      float* orow = p.out_f32 + row * p.ldo + (t & 7) + 512 * (t >> 3);
-#pragma unroll
-      for (int k = 0; k < 64; ++k) orow[8 * k] = w[k] * 0.015625f;
-    } else {
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int k = 0; k < 64; k += 4) {
-        a0 = fmaxf(a0, fabsf(w[k]));
-        a1 = fmaxf(a1, fabsf(w[k + 1]));
-        a2 = fmaxf(a2, fabsf(w[k + 2]));
-        a3 = fmaxf(a3, fabsf(w[k + 3]));
-      }
-      float am = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-      if (lane == 0) slot_max[t >> 5] = am;
-      team_sync(team);
-      const float amax = fmaxf(slot_max[0], slot_max[1]) * 0.015625f;  // max |x~| (x~ = H x / 64, exact scaling)
-      const float qmax = MODE == kModeInt4 ? 7.0f : p.qmax;
-      const float rr = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.0f;
-      const float cr = rr * 0.015625f;
-      uint8_t* cb = buf;  // [a][b] code bytes, 8-byte group g of row a at g ^ (a / 8)
-#pragma unroll
-      for (int k = 0; k < 64; k += 2) {
-        const float2 q = __ffma2_rn(make_float2(w[k], w[k + 1]), make_float2(cr, cr),
-                                    make_float2(kRoundMagic, kRoundMagic));
-        cb[64 * k + (t ^ (8 * (k >> 3)))] = (uint8_t)__float_as_uint(q.x);
-        cb[64 * (k + 1) + (t ^ (8 * ((k + 1) >> 3)))] = (uint8_t)__float_as_uint(q.y);
-      }
-      team_sync(team);
-      // outputs 64 t + 8 r + e sit at a = 8 (t mod 8) + r, b = 8 (t / 8) + e
-      uint2 c[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        c[r] = *reinterpret_cast<const uint2*>(cb + 64 * (8 * (t & 7) + r) + 8 * ((t >> 3) ^ (t & 7)));
-      if (MODE == kModeInt4) {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 2048 + 32 * t);
-        dst[0] = make_uint4(nibbles_of(c[0].x, c[0].y), nibbles_of(c[1].x, c[1].y), nibbles_of(c[2].x, c[2].y),
-                            nibbles_of(c[3].x, c[3].y));
-        dst[1] = make_uint4(nibbles_of(c[4].x, c[4].y), nibbles_of(c[5].x, c[5].y), nibbles_of(c[6].x, c[6].y),
-                            nibbles_of(c[7].x, c[7].y));
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 4096 + 64 * t);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(c[2 * k].x, c[2 * k].y, c[2 * k + 1].x, c[2 * k + 1].y);
-      }
-      if (t == 0) p.scales_f32[row] = __fdiv_rn(amax, qmax);
-    }
-    team_sync(team);  // the slot and the team's max slots are free again
-    if (t == 0 && i + S < nloc) {  // refill: the next row this slot serves (the same team's)
+    for (int g = 0; g < 16; ++g)
+      *reinterpret_cast<float4*>(tr + 64 * t + 4 * (g ^ (t & 15))) =
+          make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    team_sync(team);  // the transpose is written, and every thread has read the row out of its slot
+    if (t == 0 && i + S < nloc) {  // refill the slot with row i + S
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(&bars[sl], (unsigned)kF4kRowBytes);
       bulk_g2s(buf, p.x + (row + S) * p.sS, (unsigned)kF4kRowBytes, &bars[sl]);
-      issued[sl] += 1;
+      ((volatile int*)tags)[sl] = i + S;
     }
+#pragma unroll
+    for (int k = 0; k < 64; ++k) v[k] = tr[64 * k + 4 * ((t >> 2) ^ (k & 15)) + (t & 3)];
+    fwht64(v);
+    // v[k] is output n = (t mod 8) + 8 k + 512 (t / 8)
+    if (MODE == kModeF32) {
+      float* orow = p.out_f32 + row * p.ldo + (t & 7) + 512 * (t >> 3);
+#pragma unroll
+      for (int k = 0; k < 64; ++k) orow[8 * k] = v[k] * 0.015625f;
+      team_sync(team);  // every column read is done before the next row's writes
+      continue;
+    }
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; k += 4) {
+      a0 = fmaxf(a0, fabsf(v[k]));
+      a1 = fmaxf(a1, fabsf(v[k + 1]));
+      a2 = fmaxf(a2, fabsf(v[k + 2]));
+      a3 = fmaxf(a3, fabsf(v[k + 3]));
+    }
+    float am = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+    if (lane == 0) slot_max[t >> 5] = am;
+    team_sync(team);
+    const float amax = fmaxf(slot_max[0], slot_max[1]) * 0.015625f;  // max |x~| (x~ = H x / 64, exact scaling)
+    const float qmax = MODE == kModeInt4 ? 7.0f : p.qmax;
+    const float rr = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.0f;
+    const float cr = rr * 0.015625f;
+#pragma unroll
+    for (int k = 0; k < 64; k += 2) {
+      const float2 q = __ffma2_rn(make_float2(v[k], v[k + 1]), make_float2(cr, cr),
+                                  make_float2(kRoundMagic, kRoundMagic));
+      cb[64 * k + (t ^ (8 * (k >> 3)))] = (uint8_t)__float_as_uint(q.x);
+      cb[64 * (k + 1) + (t ^ (8 * ((k + 1) >> 3)))] = (uint8_t)__float_as_uint(q.y);
+    }
+    team_sync(team);
+    // outputs 64 t + 8 r + e sit at a = 8 (t mod 8) + r, b = 8 (t / 8) + e
+    uint2 c[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      c[r] = *reinterpret_cast<const uint2*>(cb + 64 * (8 * (t & 7) + r) + 8 * ((t >> 3) ^ (t & 7)));
+    if (MODE == kModeInt4) {
+      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 2048 + 32 * t);
+      dst[0] = make_uint4(nibbles_of(c[0].x, c[0].y), nibbles_of(c[1].x, c[1].y), nibbles_of(c[2].x, c[2].y),
+                          nibbles_of(c[3].x, c[3].y));
+      dst[1] = make_uint4(nibbles_of(c[4].x, c[4].y), nibbles_of(c[5].x, c[5].y), nibbles_of(c[6].x, c[6].y),
+                          nibbles_of(c[7].x, c[7].y));
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 4096 + 64 * t);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dst[k] = make_uint4(c[2 * k].x, c[2 * k].y, c[2 * k + 1].x, c[2 * k + 1].y);
+    }
+    if (t == 0) p.scales_f32[row] = __fdiv_rn(amax, qmax);
   }
   __syncthreads();
   // after a timed-out wait, let this CTA's own copies in flight land before it exits
   if (*abort_flag && threadIdx.x == 0) {
-    for (int sl = 0; sl < S; ++sl)
-      if (issued[sl] > 0) (void)mbar_wait_bounded(&bars[sl], (issued[sl] - 1) & 1);
+    for (int sl = 0; sl < S; ++sl) (void)mbar_wait_bounded(&bars[sl], (unsigned)((tags[sl] / S) & 1));
   }
 }
 
 // ---------------------------------------------------------------------------
 // NVFP4 with the dynamic per-tensor scale in ONE pass over HBM, for tensors that
 // fit in the SMs' combined shared memory: a cooperative launch (all CTAs
-// resident) where each CTA copies its rows into shared memory once, computes
-// the max |X~| of its rows, meets the other CTAs at a grid-wide barrier
-// (atomic counter, bounded spin), and then rotates its rows again from shared
-// memory and quantizes them with g = max/(6*448).
+// resident) where each CTA copies its rows into shared memory once, rotates
+// them and takes the max |X~| of its rows, meets the other CTAs at a grid-wide
+// barrier (atomic counter, bounded spin), and then quantizes its rotated rows
+// with g = max/(6*448).
+//
+// Between the two passes the rotated values wait in tensor memory when they
+// fit (stash = 1: at most 512 128-value units per CTA, i.e. 256 KB of fp32):
+// each thread writes its unit's 128 registers into its warp's TMEM lane
+// quadrant with tcgen05.st (column group warp / 4, or 3 for a second unit) and
+// reads them back after the barrier, so the rows are rotated once.  With more
+// units per CTA (stash = 0) the second pass rotates the rows again from
+// shared memory.
 // p.amax_word[0] gathers the max, p.amax_word[1] counts arrivals; both are
 // zeroed by the host before the launch.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc512(uint32_t* dst_smem) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(dst_smem))
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_free512(uint32_t taddr) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(taddr) : "memory");
+}
+// 128 fp32 registers of this thread to / from its lane, 128 consecutive columns
+// from `taddr` (the warp's lane-quadrant base and first column).
+__device__ __forceinline__ void tmem_store128(uint32_t taddr, const float (&v)[128]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float* q = &v[32 * k];
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr + 32u * (uint32_t)k),
+        "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]), "f"(q[8]),
+        "f"(q[9]), "f"(q[10]), "f"(q[11]), "f"(q[12]), "f"(q[13]), "f"(q[14]), "f"(q[15]), "f"(q[16]), "f"(q[17]),
+        "f"(q[18]), "f"(q[19]), "f"(q[20]), "f"(q[21]), "f"(q[22]), "f"(q[23]), "f"(q[24]), "f"(q[25]),
+        "f"(q[26]), "f"(q[27]), "f"(q[28]), "f"(q[29]), "f"(q[30]), "f"(q[31])
+        : "memory");
+  }
+}
+__device__ __forceinline__ void tmem_load128(uint32_t taddr, float (&v)[128]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float* q = &v[32 * k];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=f"(q[0]), "=f"(q[1]), "=f"(q[2]), "=f"(q[3]), "=f"(q[4]), "=f"(q[5]), "=f"(q[6]), "=f"(q[7]),
+          "=f"(q[8]), "=f"(q[9]), "=f"(q[10]), "=f"(q[11]), "=f"(q[12]), "=f"(q[13]), "=f"(q[14]), "=f"(q[15]),
+          "=f"(q[16]), "=f"(q[17]), "=f"(q[18]), "=f"(q[19]), "=f"(q[20]), "=f"(q[21]), "=f"(q[22]), "=f"(q[23]),
+          "=f"(q[24]), "=f"(q[25]), "=f"(q[26]), "=f"(q[27]), "=f"(q[28]), "=f"(q[29]), "=f"(q[30]), "=f"(q[31])
+        : "r"(taddr + 32u * (uint32_t)k)
+        : "memory");
+  }
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+constexpr int kResThreads = 384;
+constexpr int kResStashUnits = 512;  // 128 lanes x 4 column groups of 128
+
 template <int LOGB>
-__global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const RotParams p, int rows_per_cta) {
+__global__ void __launch_bounds__(kResThreads, 1) rotate_nvfp4_resident_kernel(const RotParams p, int rows_per_cta,
+                                                                              int stash) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int nb = p.nb;
   const int64_t r0 = (int64_t)blockIdx.x * rows_per_cta;
@@ -1404,7 +1509,8 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
   uint64_t* bar = reinterpret_cast<uint64_t*>(smask + nb * 64);
   unsigned* cta_max = reinterpret_cast<unsigned*>(bar + 1);
   int* flag = reinterpret_cast<int*>(cta_max + 1);
-  const int tid = threadIdx.x;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flag + 1);
+  const int tid = threadIdx.x, warp = tid >> 5;
   constexpr bool PERM = ChunkOrder<LOGB>::kPermuted;
   const ChunkKeys ck = chunk_keys<LOGB>(tid);
   const int m = ck.m;
@@ -1415,7 +1521,13 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
     fence_mbar_init();
     *cta_max = 0u;
   }
+  if (stash && warp == 0) tmem_alloc512(tmem_slot);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = stash ? *tmem_slot : 0u;
+  // this warp's lanes; column group of its first and second unit
+  const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   build_sign_table(p.signs, nb, smask, [&]() {
     if (tid == 0 && nrows > 0) {
       mbar_arrive_expect_tx(bar, (unsigned)(nrows * row_bytes));
@@ -1431,16 +1543,32 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
   __syncthreads();
   const bool loaded = *flag != 0;
 
-  // pass 1: max |X~| over this CTA's rows
+  // pass 1: rotate, max |X~| over this CTA's rows (and, stashing, park the values in TMEM)
   const int units = nrows * nb;
   float amax = 0.f;
   if (loaded) {
-    for (int u = tid; u < units; u += blockDim.x) {
-      const int r = u / nb, b = u - r * nb;
-      float v[128];
-      load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
-      fwht_block_diag<LOGB>(v);
-      amax = fmaxf(amax, absmax128(v) * c);
+    if (stash) {
+#pragma unroll 1
+      for (int i = 0; i < 2; ++i) {
+        if (32 * warp + kResThreads * i >= units) break;  // warp-uniform: no unit for any lane
+        const int u = tid + kResThreads * i;
+        const bool have = u < units;
+        const int r = have ? u / nb : 0, b = have ? u - r * nb : 0;
+        float v[128];
+        load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+        fwht_block_diag<LOGB>(v);
+        if (have) amax = fmaxf(amax, absmax128(v) * c);
+        tmem_store128(tq + 128u * (uint32_t)(i == 0 ? (warp >> 2) : 3), v);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    } else {
+      for (int u = tid; u < units; u += blockDim.x) {
+        const int r = u / nb, b = u - r * nb;
+        float v[128];
+        load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+        fwht_block_diag<LOGB>(v);
+        amax = fmaxf(amax, absmax128(v) * c);
+      }
     }
   }
   const unsigned wbits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
@@ -1468,20 +1596,47 @@ __global__ void __launch_bounds__(384, 1) rotate_nvfp4_resident_kernel(const Rot
     *flag = (ok && loaded) ? 1 : 0;
   }
   __syncthreads();
-  if (!*flag) return;
 
-  // pass 2: quantize with the tensor's scale
-  const float g = __fdiv_rn(__uint_as_float(*gmax), 2688.0f);
-  const float inv6g = g > 0.f ? __frcp_rn(6.0f * g) : 0.0f;
-  if (blockIdx.x == 0 && tid == 0 && p.g_out) *p.g_out = g;
-  for (int u = tid; u < units; u += blockDim.x) {
-    const int r = u / nb, b = u - r * nb;
-    const int64_t row = r0 + r;
-    float v[128];
-    load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
-    fwht_block_diag<LOGB>(v);
-    quant_nvfp4_store<PERM, LOGB == 0>(v, c, g, inv6g, ck.mchi, ck.mo, p.codes + row * (p.K / 2) + (size_t)b * 64,
-                                       p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+  // pass 2: quantize with the tensor's scale (skipped after a timed-out barrier)
+  if (*flag) {
+    const float g = __fdiv_rn(__uint_as_float(*gmax), 2688.0f);
+    const float inv6g = g > 0.f ? __frcp_rn(6.0f * g) : 0.0f;
+    if (blockIdx.x == 0 && tid == 0 && p.g_out) *p.g_out = g;
+    if (stash) {
+#pragma unroll 1
+      for (int i = 0; i < 2; ++i) {
+        if (32 * warp + kResThreads * i >= units) break;
+        const int u = tid + kResThreads * i;
+        float v[128];
+        tmem_load128(tq + 128u * (uint32_t)(i == 0 ? (warp >> 2) : 3), v);
+        if (u < units) {
+          const int r = u / nb, b = u - r * nb;
+          const int64_t row = r0 + r;
+          quant_nvfp4_store<PERM, LOGB == 0>(v, c, g, inv6g, ck.mchi, ck.mo,
+                                             p.codes + row * (p.K / 2) + (size_t)b * 64,
+                                             p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+        }
+      }
+    } else {
+      for (int u = tid; u < units; u += blockDim.x) {
+        const int r = u / nb, b = u - r * nb;
+        const int64_t row = r0 + r;
+        float v[128];
+        load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+        fwht_block_diag<LOGB>(v);
+        quant_nvfp4_store<PERM, LOGB == 0>(v, c, g, inv6g, ck.mchi, ck.mo,
+                                           p.codes + row * (p.K / 2) + (size_t)b * 64,
+                                           p.scales_e4m3 + row * (p.K / 16) + (size_t)b * 8);
+      }
+    }
+  }
+  if (stash) {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      tmem_free512(tmem);
+    }
   }
 }
 

@@ -15,7 +15,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librq.so")
 
-RQ_INT4, RQ_NVFP4, RQ_MXFP4, RQ_INT8, RQ_INT6, RQ_INT4_ASYM = 0, 1, 2, 3, 4, 5
+RQ_INT4, RQ_NVFP4, RQ_MXFP4, RQ_INT8, RQ_INT6, RQ_INT4_ASYM, RQ_INT4_BYTES = 0, 1, 2, 3, 4, 5, 6
 RQ_OUT_F32, RQ_OUT_BF16, RQ_OUT_I32_ACC = 0, 1, 2
 RQ_SCALE_DYNAMIC, RQ_SCALE_STATIC = 0, 1
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_INVALID_ARG", 2: "RQ_ERR_UNSUPPORTED_SHAPE", 3: "RQ_ERR_ALIGNMENT",
@@ -86,7 +86,7 @@ def _stream(t=None):
 def _fmt(fmt):
     if isinstance(fmt, str):
         return {"int4": RQ_INT4, "nvfp4": RQ_NVFP4, "mxfp4": RQ_MXFP4, "int8": RQ_INT8, "int6": RQ_INT6,
-                "int4_asym": RQ_INT4_ASYM}[fmt]
+                "int4_asym": RQ_INT4_ASYM, "int4_bytes": RQ_INT4_BYTES}[fmt]
     return int(fmt)
 
 
@@ -136,7 +136,7 @@ def _expect_bytes(t, nbytes, name):
 
 def _quant_shapes(rows, k, fmt):
     """(codes shape, codes dtype, scales shape, scales dtype) that a format writes."""
-    if fmt in (RQ_INT8, RQ_INT6):
+    if fmt in (RQ_INT8, RQ_INT6, RQ_INT4_BYTES):
         return (rows, k), torch.int8, (rows,), torch.float32
     if fmt == RQ_INT4_ASYM:
         return (rows, k // 2), torch.uint8, (rows, k // 128, 2), torch.float16
@@ -171,7 +171,7 @@ def _expect_output_matrix(y, m, n, dtype):
 
 
 def _alloc_quant_outputs(rows, k, fmt, device):
-    if fmt in (RQ_INT8, RQ_INT6):  # one int8 code per byte
+    if fmt in (RQ_INT8, RQ_INT6, RQ_INT4_BYTES):  # one int8 code per byte
         return (torch.empty((rows, k), dtype=torch.int8, device=device),
                 torch.empty((rows,), dtype=torch.float32, device=device))
     codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=device)
@@ -274,13 +274,13 @@ def w4a4_gemm(xq, wq, fmt="int4", out="f32", y=None):
 def int_gemm(xq, xfmt, wq, wfmt, out="f32", y=None):
     """Y = deq(xq) . deq(wq)^T for integer codes of different widths (W4A8, W6A6,
     W8A8, W4A4): xq / wq are (codes, scales, _) triples from rotate_quantize /
-    prepare_weights with formats xfmt / wfmt in {"int4", "int6", "int8"}."""
+    prepare_weights with formats xfmt / wfmt in {"int4", "int6", "int8"}; W4A4
+    also takes wfmt "int4_bytes" (the INT4 weight codes one per byte)."""
     xc, xs = xq[0], xq[1]
     wc, ws = wq[0], wq[1]
     fx, fw = _fmt(xfmt), _fmt(wfmt)
-    for f in (fx, fw):
-        if f not in (RQ_INT4, RQ_INT6, RQ_INT8):
-            raise ValueError("int_gemm takes int4, int6 or int8 codes")
+    if fx not in (RQ_INT4, RQ_INT6, RQ_INT8) or fw not in (RQ_INT4, RQ_INT6, RQ_INT8, RQ_INT4_BYTES):
+        raise ValueError("int_gemm takes int4, int6 or int8 codes (int4_bytes for the weights)")
     o = {"f32": RQ_OUT_F32, "bf16": RQ_OUT_BF16, "i32": RQ_OUT_I32_ACC}[out]
     if xc.dim() != 2 or wc.dim() != 2:
         raise ValueError("codes must be 2-D")

@@ -137,6 +137,9 @@ def test_int_gemm_rejections():
     assert igemm(xf=1) == INVALID                  # NVFP4 is not an integer format
     assert igemm(wf=5) == INVALID                  # per-group asymmetric codes have no GEMM
     assert igemm(xf=0, wf=3) == SHAPE              # 4-bit activations with wider weights
+    assert igemm(xf=3, wf=6) == INVALID            # the byte layout of INT4 weights pairs with INT4 activations
+    assert igemm(xf=0, wf=6, k=192) == SHAPE       # W4A4 with byte weights: K a multiple of 128
+    assert igemm(xf=0, wf=6, m=0) == 0
     assert igemm(xf=0, wf=0, k=192) == SHAPE       # W4A4 goes through the W4A4 GEMM's checks
     assert igemm(ldy=100) == INVALID
     assert igemm(out=9) == INVALID
@@ -193,7 +196,9 @@ def test_noalloc_and_selftest_rejections():
 
 
 def test_rotate_quantize_format_rules():
-    assert rotq(fmt=6) == INVALID                  # no such format
+    assert rotq(fmt=7) == INVALID                  # no such format
+    assert rotq(fmt=6, m=0) == 0                   # INT4 codes one per byte
+    assert rotq(fmt=6, scales=P(0x10002)) == ALIGN  # its fp32 scales
     assert rotq(fmt=2, block=0) == SHAPE           # MXFP4 needs block-diagonal rotation
     assert rotq(fmt=5, block=0) == SHAPE           # so do per-group asymmetric codes
     assert rotq(fmt=3, block=64) == SHAPE          # blocks of 16, 32, 128 or the full width
