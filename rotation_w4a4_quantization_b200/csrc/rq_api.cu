@@ -170,7 +170,7 @@ rq_status launch_nvfp4_resident_b(RotParams p, cudaStream_t st) {
     return RQ_ERR_UNSUPPORTED_SHAPE;
   const int sms = num_sms_of_current_device();
   const int64_t rpc = (p.rows + sms - 1) / sms;
-  const size_t smem = (size_t)rpc * p.K * 2 + (size_t)p.nb * 64 * 4 + 48;
+  const size_t smem = (size_t)rpc * p.K * 2 + (size_t)p.nb * 64 * 4 + (size_t)rpc * 8 + 48;
   if (smem > kSmemBudget) return RQ_ERR_UNSUPPORTED_SHAPE;
   // the rotated values wait in tensor memory between the passes when a CTA's
   // 128-value units fit its 512 columns x 128 lanes

@@ -694,6 +694,35 @@ __device__ __forceinline__ void kv4_second_look(unsigned pending, GroupFn group_
   }
 }
 
+// kv4_second_look out of line, for the rotate kernel: lane L's group follows
+// the kernel's thread mapping (rows of RPS per stage starting at r0; a group
+// is the lane's 128-wide block, or the vector itself for KV4).  Kept out of
+// line so that its code -- rarely run -- does not crowd the instruction cache
+// of the unrolled main loop.
+template <int LOGB, bool KV>
+__device__ __noinline__ void kv4_second_look_rows(unsigned pending, const RotParams p, int64_t r0, int wig,
+                                                  int RPS, const uint32_t* smask) {
+  const int nb = p.nb;
+  kv4_second_look<LOGB>(pending, [&](int L) {
+    const int rL = RPS > 1 ? L / nb : 0;
+    const int bL = RPS > 1 ? L - rL * nb : wig * 32 + L;
+    const int64_t rowL = r0 + rL;
+    KvGroup gr;
+    gr.src = row_src(p, rowL) + (size_t)bL * 256;
+    gr.smask = smask + bL * 64;
+    if (KV) {
+      gr.codes = p.codes + rowL * 64;
+      gr.scale = p.kv_scale + rowL;
+      gr.zero = p.kv_zero + rowL;
+    } else {
+      gr.codes = p.codes + rowL * (p.K / 2) + (size_t)bL * 64;
+      gr.scale = p.kv_scale + 2 * (rowL * nb + bL);
+      gr.zero = gr.scale + 1;
+    }
+    return gr;
+  });
+}
+
 // KV4 and per-group asymmetric INT4: asymmetric quantization of one group of
 // 128 channels (true value = v * c * chi): z = min, s = (max - min)/15, both
 // stored as fp16, q = clamp(rint((x - z)/s), 0, 15).
@@ -1102,27 +1131,7 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
                                : quant_kv4_store<PERM>(v, c, mchi, mo, valid,
                                                        p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
         const unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
-        if (pending) {
-          // lane L's row and block, by the same mapping as this thread's
-          kv4_second_look<KV ? 7 : LOGB>(pending, [&](int L) {
-            const int rL = RPS > 1 ? L / nb : 0;
-            const int bL = RPS > 1 ? L - rL * nb : wig * 32 + L;
-            const int64_t rowL = r0 + rL;
-            KvGroup gr;
-            gr.src = row_src(p, rowL) + (size_t)bL * 256;
-            gr.smask = smask + bL * 64;
-            if (KV) {
-              gr.codes = p.codes + rowL * 64;
-              gr.scale = p.kv_scale + rowL;
-              gr.zero = p.kv_zero + rowL;
-            } else {
-              gr.codes = p.codes + rowL * (p.K / 2) + (size_t)bL * 64;
-              gr.scale = p.kv_scale + 2 * (rowL * nb + bL);
-              gr.zero = gr.scale + 1;
-            }
-            return gr;
-          });
-        }
+        if (pending) kv4_second_look_rows<KV ? 7 : LOGB, KV>(pending, p, r0, wig, RPS, smask);
       }
     } else {
       constexpr int NB = NBF ? NBF : 1;
@@ -1506,8 +1515,8 @@ __global__ void __launch_bounds__(kResThreads, 1) rotate_nvfp4_resident_kernel(c
   const size_t row_bytes = (size_t)p.K * 2;
   uint8_t* rows = smem_raw;
   uint32_t* smask = reinterpret_cast<uint32_t*>(smem_raw + (size_t)rows_per_cta * row_bytes);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smask + nb * 64);
-  unsigned* cta_max = reinterpret_cast<unsigned*>(bar + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smask + nb * 64);  // one per row: a warp starts on its row once it lands
+  unsigned* cta_max = reinterpret_cast<unsigned*>(bars + rows_per_cta);
   int* flag = reinterpret_cast<int*>(cta_max + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flag + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -1517,7 +1526,7 @@ __global__ void __launch_bounds__(kResThreads, 1) rotate_nvfp4_resident_kernel(c
   const float c = LOGB == 7 ? 0.08838834764831845f : (LOGB == 0 ? 1.0f : p.cblk);  // 1/sqrt(block), rounded once
 
   if (tid == 0) {
-    mbar_init(bar, 1);
+    for (int rr = 0; rr < nrows; ++rr) mbar_init(&bars[rr], 1);
     fence_mbar_init();
     *cta_max = 0u;
   }
@@ -1529,51 +1538,48 @@ __global__ void __launch_bounds__(kResThreads, 1) rotate_nvfp4_resident_kernel(c
   // this warp's lanes; column group of its first and second unit
   const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   build_sign_table(p.signs, nb, smask, [&]() {
-    if (tid == 0 && nrows > 0) {
-      mbar_arrive_expect_tx(bar, (unsigned)(nrows * row_bytes));
-      if (p.contiguous) {  // the CTA's rows are one span of at most the shared-memory budget
-        bulk_g2s(rows, p.x + r0 * (int64_t)row_bytes, (unsigned)(nrows * row_bytes), bar);
-      } else {
-        for (int rr = 0; rr < nrows; ++rr)
-          bulk_g2s(rows + (size_t)rr * row_bytes, p.x + (r0 + rr) * p.sS, (unsigned)row_bytes, bar);
+    if (tid == 0) {  // one copy per row, in row order
+      for (int rr = 0; rr < nrows; ++rr) {
+        mbar_arrive_expect_tx(&bars[rr], (unsigned)row_bytes);
+        bulk_g2s(rows + (size_t)rr * row_bytes, p.x + (r0 + rr) * p.sS, (unsigned)row_bytes, &bars[rr]);
       }
     }
   });
-  if (tid == 0) *flag = (nrows == 0 || mbar_wait_bounded(bar, 0)) ? 1 : 0;
   __syncthreads();
-  const bool loaded = *flag != 0;
 
-  // pass 1: rotate, max |X~| over this CTA's rows (and, stashing, park the values in TMEM)
+  // pass 1: rotate, max |X~| over this CTA's rows (and, stashing, park the values
+  // in TMEM); each thread waits only for the row of its own unit
   const int units = nrows * nb;
   float amax = 0.f;
-  if (loaded) {
-    if (stash) {
+  bool ok = true;
+  if (stash) {
 #pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        if (32 * warp + kResThreads * i >= units) break;  // warp-uniform: no unit for any lane
-        const int u = tid + kResThreads * i;
-        const bool have = u < units;
-        const int r = have ? u / nb : 0, b = have ? u - r * nb : 0;
-        float v[128];
-        load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
-        fwht_block_diag<LOGB>(v);
-        if (have) amax = fmaxf(amax, absmax128(v) * c);
-        tmem_store128(tq + 128u * (uint32_t)(i == 0 ? (warp >> 2) : 3), v);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    } else {
-      for (int u = tid; u < units; u += blockDim.x) {
-        const int r = u / nb, b = u - r * nb;
-        float v[128];
-        load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
-        fwht_block_diag<LOGB>(v);
-        amax = fmaxf(amax, absmax128(v) * c);
-      }
+    for (int i = 0; i < 2; ++i) {
+      if (32 * warp + kResThreads * i >= units) break;  // warp-uniform: no unit for any lane
+      const int u = tid + kResThreads * i;
+      const bool have = u < units;
+      const int r = have ? u / nb : 0, b = have ? u - r * nb : 0;
+      if (have) ok = ok && mbar_wait_bounded(&bars[r], 0);
+      float v[128];
+      load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+      fwht_block_diag<LOGB>(v);
+      if (have) amax = fmaxf(amax, absmax128(v) * c);
+      tmem_store128(tq + 128u * (uint32_t)(i == 0 ? (warp >> 2) : 3), v);
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  } else {
+    for (int u = tid; u < units; u += blockDim.x) {
+      const int r = u / nb, b = u - r * nb;
+      ok = ok && mbar_wait_bounded(&bars[r], 0);
+      float v[128];
+      load_block(rows + (size_t)r * row_bytes + (size_t)b * 256, smask + b * 64, m, v);
+      fwht_block_diag<LOGB>(v);
+      amax = fmaxf(amax, absmax128(v) * c);
     }
   }
   const unsigned wbits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
   if ((tid & 31) == 0) atomicMax(cta_max, wbits);
-  __syncthreads();
+  const bool loaded = __syncthreads_and(ok) != 0;  // every row of this CTA landed
 
   // grid-wide barrier: publish this CTA's max, count arrivals, wait for all
   volatile unsigned* gmax = p.amax_word;
