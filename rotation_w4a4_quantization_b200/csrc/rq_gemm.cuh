@@ -65,6 +65,7 @@ struct GemmParams {
 
 // Bounded wait used by every role; on timeout the role stops issuing work.
 __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, unsigned parity, int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;  // the common case: one shared-memory round trip
   if (*((volatile int*)abort_flag)) return false;
   if (!mbar_wait_bounded(bar, parity)) {
     *((volatile int*)abort_flag) = 1;
@@ -626,7 +627,9 @@ done:
 // lane quadrants: SFA of its own 128 X rows, and SFB of ALL 256 W rows of the
 // tile (each SM's tensor core multiplies its rows by every column of the tile,
 // so it reads the scales of both W halves from its own tensor memory).  Then
-// they arrive on the even CTA's scales-ready barrier.
+// they arrive on the even CTA's operand barrier, which so completes once the
+// k-tile's operands have landed and its scales are in both CTAs' tensor
+// memory: the MMA thread waits on one barrier per k-tile.
 // ---------------------------------------------------------------------------
 constexpr int kN2St = 5;
 constexpr int kN2OpA = 128 * 128, kN2OpB = 128 * 128, kN2SfA = 128 * 16, kN2SfB = 256 * 16;
@@ -648,11 +651,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
   uint8_t* op = base;
   uint8_t* epi_stage = op + (size_t)kN2St * kN2Stage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + kEpiStage);
-  uint64_t* op_full = bars;                 // even CTA: both CTAs' X/W copies
+  uint64_t* op_full = bars;                 // even CTA: both CTAs' X/W copies and scales in TMEM
   uint64_t* op_empty = op_full + kN2St;     // both: multicast MMA commit
   uint64_t* sf_full = op_empty + kN2St;     // local: this CTA's scale copies
-  uint64_t* sf_ready = sf_full + kN2St;     // even CTA: both CTAs' scales in TMEM
-  uint64_t* acc_full = sf_ready + kN2St;
+  uint64_t* acc_full = sf_full + kN2St;
   uint64_t* acc_empty = acc_full + 1;       // even CTA: both epilogues
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -665,10 +667,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kN2St; ++i) {
-      mbar_init(&op_full[i], 1);
+      // the producer's arrival with the copies' bytes, and one per scale mover
+      // warp that wrote this k-tile's scales (4 quadrants x 2 CTAs)
+      mbar_init(&op_full[i], 1 + 8);
       mbar_init(&op_empty[i], 1);
       mbar_init(&sf_full[i], 1);
-      mbar_init(&sf_ready[i], 8);  // 4 quadrants x 2 CTAs (one mover warp per quadrant per k-tile)
     }
     mbar_init(&acc_full[0], 1);
     mbar_init(&acc_empty[0], 8);
@@ -721,8 +724,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
         if (!wait_or_fail(&acc_empty[0], (unsigned)(it & 1) ^ 1, abort_flag)) goto done;
         tc_fence_after();
         for (int kt = 0; kt < KT; ++kt) {
-          if (!wait_or_fail(&op_full[s], ph, abort_flag)) goto done;
-          if (!wait_or_fail(&sf_ready[s], ph, abort_flag)) goto done;
+          if (!wait_or_fail(&op_full[s], ph, abort_flag)) goto done;  // operands and scales
           tc_fence_after();
           const uint8_t* a = op + (size_t)s * kN2Stage;
           const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + kN2OpA);
@@ -781,7 +783,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kN2Threads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_u32(&sf_ready[s], 0));
+        if (lane == 0) mbar_arrive_cluster(mapa_u32(&op_full[s], 0));
         if (++s == kN2St) { s = 0; ph ^= 1; }
       }
     }
@@ -1025,16 +1027,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kI3Threads, 1)
       unsigned oph = 0;
       int it = 0;
       for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
-        if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&acc_empty[0], (unsigned)((it & 1) ^ 1))) {
-          *((volatile int*)abort_flag) = 1;
-          goto done;
-        }
+        if (!wait_or_fail(&acc_empty[0], (unsigned)((it & 1) ^ 1), abort_flag)) goto done;
         tc_fence_after();
         for (int kt = 0; kt < KT; ++kt) {
-          if (*((volatile int*)abort_flag) || !mbar_wait_bounded(&op_full[o], oph)) {
-            *((volatile int*)abort_flag) = 1;
-            goto done;
-          }
+          if (!wait_or_fail(&op_full[o], oph, abort_flag)) goto done;
           tc_fence_after();
           const uint64_t bd = smem_desc_sw128(opb + (size_t)o * kI3OpB);
           const uint32_t ta = tmem + kI3ACol0 + 32u * (uint32_t)o;

@@ -1031,8 +1031,12 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
   const bool producer = (wig == 0 && lane == 0);
   // 1/sqrt(block), rounded once; 1 without a rotation
   const float c = (NBF || LOGB == 7) ? 0.08838834764831845f : (LOGB == 0 ? 1.0f : p.cblk);
-  const int64_t TG = (int64_t)gridDim.x * p.GPC;
-  const int64_t gg = (int64_t)blockIdx.x * p.GPC + grp;
+  // each CTA a contiguous run of num_tiles / grid tiles (rounded down or up),
+  // dealt to its groups in turn, so that no SM gets a whole round more than
+  // another (tiles dealt grid-wide in turn left some SMs a whole round more)
+  const int64_t t_end = ((int64_t)blockIdx.x + 1) * p.num_tiles / gridDim.x;
+  const int64_t TG = p.GPC;
+  const int64_t gg = (int64_t)blockIdx.x * p.num_tiles / gridDim.x + grp;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.GPC * p.stages; ++i) mbar_init(&bars_all[i], 1);
@@ -1042,7 +1046,7 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
   build_sign_table(p.signs, nb, smask, [&]() {
     if (producer) {  // the first tile copies of this group
       int64_t tile = gg;
-      for (int st = 0; st < p.stages && tile < p.num_tiles; ++st, tile += TG)
+      for (int st = 0; st < p.stages && tile < t_end; ++st, tile += TG)
         issue_tile_load(p, tile, ring + st * sbytes, &full[st]);
     }
   });
@@ -1057,14 +1061,14 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
   float amax_acc = 0.f;
 
   int64_t i = 0;
-  for (int64_t tile = gg; tile < p.num_tiles; tile += TG, ++i) {
+  for (int64_t tile = gg; tile < t_end; tile += TG, ++i) {
     const int st = (int)(i % p.stages);
     const bool ok = group_all(mbar_wait_bounded(&full[st], (unsigned)((i / p.stages) & 1)), G, grp);
     if (!ok) {
       if (producer) {  // let the copies this group issued land before leaving
         for (int k = 1; k < p.stages; ++k) {
           const int64_t i2 = i + k;
-          if (gg + i2 * TG >= p.num_tiles) break;
+          if (gg + i2 * TG >= t_end) break;
           (void)mbar_wait_bounded(&full[i2 % p.stages], (unsigned)((i2 / p.stages) & 1));
         }
       }
@@ -1086,7 +1090,7 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
       group_sync(G, grp);  // stage consumed: refill it while this tile is computed
       if (producer) {
         const int64_t nt = tile + (int64_t)p.stages * TG;
-        if (nt < p.num_tiles) {
+        if (nt < t_end) {
           fence_proxy_async_smem();
           issue_tile_load(p, nt, stage, &full[st]);
         }
@@ -1144,7 +1148,7 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
       full_phase2<NB>(v, y[1], 1, zbuf, r, b, lane, m, p.cfull, valid);
       if (producer) {
         const int64_t nt = tile + (int64_t)p.stages * TG;
-        if (nt < p.num_tiles) {
+        if (nt < t_end) {
           fence_proxy_async_smem();
           issue_tile_load(p, nt, stage, &full[st]);
         }
