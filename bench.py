@@ -72,29 +72,31 @@ def load_peaks():
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
 ATTN_SOURCES = ("rq_common.cuh", "rq_attn.cuh")
-_ROT, _GEM, _ATT = "ca3beeb8c0e87f73", "bbf648be1c99fde4", "80b39046d2c3159b"
+_ROT, _GEM, _ATT = "6766e941b93707f2", "74cfd6dd085e3e33", "80b39046d2c3159b"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
 # ncu capture of the kernel (summarised in profiles/), with the fingerprint of
 # the sources it was taken on (reported as null once they change).  kv4 and
 # kv4_decode were captured at B = 4 and are scaled to the bench's B = 16 (traffic
 # grows with the vectors processed); kv4_decode is the partial + combine pair.
 TRAFFIC = {
-    ("hadamard_quant", "q_proj_int4"): (16809984, _ROT),
-    ("hadamard_quant", "down_proj_int4"): (105441792, _ROT),
-    ("hadamard_quant", "kv4"): (146989312 * 4, _ROT),
-    ("hadamard_quant", "q_proj_nvfp4"): (16830464, _ROT),
+    ("hadamard_quant", "q_proj_int4"): (16818176, _ROT),
+    ("hadamard_quant", "down_proj_int4"): (105203200, _ROT),
+    ("hadamard_quant", "kv4"): (145912576 * 4, _ROT),
+    ("hadamard_quant", "q_proj_nvfp4"): (16850944, _ROT),
     ("hadamard_quant", "q_proj_mxfp4"): (16832000, _ROT),
-    ("hadamard_quant", "q_proj_w4a8"): (16809216, _ROT),
-    ("hadamard_quant", "q_proj_w8a8"): (16809216, _ROT),
-    ("hadamard_quant", "q_proj_nvfp4_b16"): (16825600, _ROT),
-    ("hadamard_quant", "q_proj_int4_asym"): (16841216, _ROT),
-    ("hadamard_quant", "kv4_decode"): (72926720 * 4, _ATT),
-    ("gemm", "q_proj_int4"): (12649984, _GEM),
-    ("gemm", "down_proj_int4"): (59483904, _GEM),
-    ("gemm", "q_proj_nvfp4"): (14189568, _GEM),
-    ("gemm", "q_proj_mxfp4"): (13400320, _GEM),
-    ("gemm", "q_proj_w4a8"): (16844032, _GEM),
-    ("gemm", "q_proj_w8a8"): (25233920, _GEM),
+    ("hadamard_quant", "q_proj_w4a8"): (16817408, _ROT),
+    ("hadamard_quant", "q_proj_w8a8"): (16817408, _ROT),
+    ("hadamard_quant", "q_proj_nvfp4_b16"): (16850944, _ROT),
+    ("hadamard_quant", "q_proj_int4_asym"): (16849664, _ROT),
+    ("hadamard_quant", "kv4_decode"): (72226048 * 4, _ATT),
+    ("gemm", "q_proj_int4"): (12650496, _GEM),
+    ("gemm", "down_proj_int4"): (59438848, _GEM),
+    ("gemm", "q_proj_nvfp4"): (14189312, _GEM),
+    ("gemm", "q_proj_mxfp4"): (13400064, _GEM),
+    ("gemm", "q_proj_w4a8"): (16844544, _GEM),
+    ("gemm", "q_proj_w8a8"): (25230592, _GEM),
+    ("gemm_bytes", "q_proj_int4"): (21044480, _GEM),
+    ("gemm_bytes", "down_proj_int4"): (94283520, _GEM),
 }
 
 
@@ -696,7 +698,7 @@ def run_workload(name, args, rq, dev, dist, world, rank, local, cpu_scale=1.0):
             out["gemm_int4_bytes"] = {
                 "value": round(gb_tops, 2), "unit": "TOPS", "ms": round(gb_ms, 5),
                 "frac_of_peak": round(wl.gemm_ops / (gb_ms * 1e-3) / 1e12 / peak_t, 4),
-                "kernel": "gemm_int_2sm_ts_kernel<A4, W8>",
+                "kernel": "gemm_int_2sm_ts_kernel<A4, W8>", "traffic": traffic("gemm_bytes", name),
                 "weights": "the same INT4 codes and scales, one code per byte (twice the packed weight memory)"}
         dominant = roof_g if g_mean_ms >= q_mean_ms else roof_q
         out["roofline"] = dominant

@@ -2,12 +2,14 @@
 
     python -m rotation_w4a4_quantization_b200.launch_case rotate <workload> [reps]
     python -m rotation_w4a4_quantization_b200.launch_case gemm <workload> [reps]
+    python -m rotation_w4a4_quantization_b200.launch_case gemm_bytes <workload> [reps]
     python -m rotation_w4a4_quantization_b200.launch_case attention kv4_decode [reps]
 
 Each call builds the workload's inputs on cuda:0 (the rotations' inputs are
 made by the package's own kernels where a cache or codes are needed) and
 launches the named step `reps` times, so that a capture can skip the first
-launch (`-s 1 -c 1`).  The KV4 cases use a quarter of the batch (B = 4): each
+launch (`-s 1 -c 1`).  `gemm_bytes` is the INT4 workloads' GEMM with the
+weights' codes stored one per byte (RQ_INT4_BYTES).  The KV4 cases use a quarter of the batch (B = 4): each
 tensor is then still above the 126 MB L2 but the capture stays small.
 """
 
@@ -45,6 +47,14 @@ def main(argv):
                 rq.int_gemm(xq, c["fmt"], wq, wfmt, "bf16", y=y)
             else:
                 rq.w4a4_gemm(xq, wq, c["fmt"], "bf16", y=y)
+    elif kind == "gemm_bytes":
+        x = syn.activations(name, device="cuda")
+        w = syn.weights(name, device="cuda")
+        wq = rq.prepare_weights(w, s, c["block"], "int4_bytes")
+        xq = rq.rotate_quantize(x, s, c["block"], "int4")
+        y = torch.empty((c["M"], c["N"]), dtype=torch.bfloat16, device="cuda")
+        for _ in range(reps):
+            rq.int_gemm(xq, "int4", wq, "int4_bytes", "bf16", y=y)
     elif kind == "attention":
         kc = rq.kv_rotate_quantize(syn.kv(batch=4, device="cuda", which=0), s)
         vc = rq.kv_rotate_quantize(syn.kv(batch=4, device="cuda", which=1), s)
