@@ -589,8 +589,8 @@ __device__ __forceinline__ double inv_sqrt_block_f64() {
 }
 
 // One group of 128 channels rotated in fp64 by the whole warp: lane l takes
-// channels 4l .. 4l+3 of the group's bf16 inputs at `src` (global memory) and
-// of its sign masks, and the fast Walsh-Hadamard butterflies of the
+// channels 4l .. 4l+3 of the group's bf16 inputs at `src` (the tile's
+// shared-memory stage) and of its sign masks, and the fast Walsh-Hadamard butterflies of the
 // 2^LOGB-wide blocks run in fp64 (the first two stages within a lane, the
 // others across lanes), scaled by 1/sqrt(2^LOGB).  On return y[e] is rotated
 // channel 4 lane + e, and lo / hi are the group's min / max (the same in every
@@ -600,7 +600,7 @@ __device__ __forceinline__ double inv_sqrt_block_f64() {
 template <int LOGB>
 __device__ __forceinline__ void rotated_group_f64(const uint8_t* src, const uint32_t* smask_grp, int lane,
                                                   double (&v)[4], double& lo, double& hi) {
-  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src) + lane);
+  const uint2 raw = *(reinterpret_cast<const uint2*>(src) + lane);
   const uint2 mk = *reinterpret_cast<const uint2*>(smask_grp + 2 * lane);
   const uint32_t a = raw.x ^ mk.x, b = raw.y ^ mk.y;
   v[0] = (double)__uint_as_float(a << 16);
@@ -644,8 +644,8 @@ __device__ __forceinline__ void rotated_group_f64(const uint8_t* src, const uint
   hi = mx;
 }
 
-// Where one group of 128 channels lives: its bf16 inputs (global), its sign
-// masks (shared) and its stored codes, scale and zero (global).
+// Where one group of 128 channels lives: its bf16 inputs (the shared-memory
+// stage), its sign masks (shared) and its stored codes, scale and zero (global).
 struct KvGroup {
   const uint8_t* src;
   const uint32_t* smask;
@@ -656,20 +656,22 @@ struct KvGroup {
 
 // The second look of quant_kv4_store: for each lane L in `pending` the warp
 // rotates L's group in fp64 (rotated_group_f64) and, where the fp16 roundings
-// of the exact min and (max - min)/15 differ from the ones stored for that
-// group, rewrites its scale, zero and codes from the fp64 values.  Called by
-// every lane of the warp; group_of(L) gives lane L's group and is evaluated
-// (by the whole warp) only for the pending lanes, so none of its address
-// arithmetic runs in the common case.
+// of the exact min and (max - min)/15 differ from the ones lane L stored for
+// that group (`szb`: its fp16 scale bits << 16 | zero bits, taken from lane L
+// by a shuffle), rewrites its scale, zero and codes from the fp64 values.
+// Called by every lane of the warp; group_of(L) gives lane L's group and is
+// evaluated (by the whole warp) only for the pending lanes, so none of its
+// address arithmetic runs in the common case.  Nothing here reads global
+// memory: a look costs its arithmetic, not a round trip.
 template <int LOGB, typename GroupFn>
-__device__ __forceinline__ void kv4_second_look(unsigned pending, GroupFn group_of) {
+__device__ __forceinline__ void kv4_second_look(unsigned pending, uint32_t szb, GroupFn group_of) {
   const int lane = threadIdx.x & 31;
   __syncwarp();  // this warp's stores of its groups come before any rewrite below
   while (pending) {
     const int L = __ffs(pending) - 1;
     pending &= pending - 1;
     const KvGroup gr = group_of(L);
-    const uint32_t szbits = ((uint32_t)__half_as_ushort(*gr.scale) << 16) | __half_as_ushort(*gr.zero);
+    const uint32_t szbits = __shfl_sync(0xFFFFFFFFu, szb, L);
     double y[4], dlo, dhi;
     rotated_group_f64<LOGB>(gr.src, gr.smask, lane, y, dlo, dhi);
     const __half zx = __double2half(dlo);
@@ -684,7 +686,6 @@ __device__ __forceinline__ void kv4_second_look(unsigned pending, GroupFn group_
         if (sd > 0.0) q = min(max(__double2int_rn((y[e] - zd) / sd), 0), 15);
         nib |= (uint32_t)q << (4 * e);
       }
-      __syncwarp();  // every lane has read the stored scale and zero
       *reinterpret_cast<uint16_t*>(gr.codes + 2 * lane) = (uint16_t)nib;  // channels 4 lane .. 4 lane + 3
       if (lane == 0) {
         *gr.scale = sx;
@@ -700,15 +701,15 @@ __device__ __forceinline__ void kv4_second_look(unsigned pending, GroupFn group_
 // line so that its code -- rarely run -- does not crowd the instruction cache
 // of the unrolled main loop.
 template <int LOGB, bool KV>
-__device__ __noinline__ void kv4_second_look_rows(unsigned pending, const RotParams p, int64_t r0, int wig,
-                                                  int RPS, const uint32_t* smask) {
+__device__ __noinline__ void kv4_second_look_rows(unsigned pending, uint32_t szb, const RotParams p, int64_t r0,
+                                                  int wig, int RPS, const uint32_t* smask, const uint8_t* stage) {
   const int nb = p.nb;
-  kv4_second_look<LOGB>(pending, [&](int L) {
+  kv4_second_look<LOGB>(pending, szb, [&](int L) {
     const int rL = RPS > 1 ? L / nb : 0;
     const int bL = RPS > 1 ? L - rL * nb : wig * 32 + L;
     const int64_t rowL = r0 + rL;
     KvGroup gr;
-    gr.src = row_src(p, rowL) + (size_t)bL * 256;
+    gr.src = stage + (size_t)rL * p.K * 2 + (size_t)bL * 256;
     gr.smask = smask + bL * 64;
     if (KV) {
       gr.codes = p.codes + rowL * 64;
@@ -739,11 +740,13 @@ __device__ __noinline__ void kv4_second_look_rows(unsigned pending, const RotPar
 // fp16 roundings of the exact min and scale differ from the stored ones (about
 // 2 groups in 10^4), the warp rewrites the group's z, s and codes from the
 // fp64 values (kv4_second_look).  This function stores the group (only where
-// `valid`) and returns whether this lane's group needs the second look; the
-// caller then runs kv4_second_look with the whole warp.
+// `valid`), sets `szb` to the stored bits (scale << 16 | zero) and returns
+// whether this lane's group needs the second look; the caller then runs
+// kv4_second_look with the whole warp, from the tile's shared-memory stage.
 template <bool PERM>
 __device__ __forceinline__ bool quant_kv4_store(const float (&v)[128], float c, int m, int mo, bool valid,
-                                                uint8_t* dst_codes, __half* dst_scale, __half* dst_zero) {
+                                                uint8_t* dst_codes, __half* dst_scale, __half* dst_zero,
+                                                uint32_t& szb) {
   float lo = 3.0e38f, hi = -3.0e38f;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -778,6 +781,7 @@ __device__ __forceinline__ bool quant_kv4_store(const float (&v)[128], float c, 
   // whether z or s lies near an fp16 midpoint (the second look, after the stores)
   const float am = fmaxf(fabsf(lo), fabsf(hi));
   const bool unsure = valid && (near_fp16_midpoint<22>(lo, am) || near_fp16_midpoint<24>(s, am));
+  szb = ((uint32_t)__half_as_ushort(s_h) << 16) | __half_as_ushort(z_h);
   if (valid) {
     *dst_scale = s_h;
     *dst_zero = z_h;
@@ -1087,14 +1091,21 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
     load_block(stage + (size_t)(active ? r : 0) * p.K * 2 + (size_t)bl * 256, smask + bl * 64, m, v);
 
     if (NBF == 0) {
-      group_sync(G, grp);  // stage consumed: refill it while this tile is computed
-      if (producer) {
-        const int64_t nt = tile + (int64_t)p.stages * TG;
-        if (nt < t_end) {
-          fence_proxy_async_smem();
-          issue_tile_load(p, nt, stage, &full[st]);
+      // stage consumed: refill it while this tile is computed.  KV4 and
+      // per-group asymmetric INT4 keep it until after the tile's second look,
+      // which reads its inputs from there.
+      constexpr bool kKeepStage = MODE == kModeKv4 || MODE == kModeAsym4;
+      const auto refill = [&]() {
+        group_sync(G, grp);
+        if (producer) {
+          const int64_t nt = tile + (int64_t)p.stages * TG;
+          if (nt < t_end) {
+            fence_proxy_async_smem();
+            issue_tile_load(p, nt, stage, &full[st]);
+          }
         }
-      }
+      };
+      if (!kKeepStage) refill();
       fwht_block_diag<LOGB>(v);
       if (MODE == kModeInt4) {
         const float a = valid ? absmax128(v) * c : 0.f;
@@ -1131,11 +1142,14 @@ __global__ void __launch_bounds__(NBF ? RQ_FULL_WIDTH_THREADS : 384, 1) rotate_k
       } else if (MODE == kModeKv4 || MODE == kModeAsym4) {
         constexpr bool KV = MODE == kModeKv4;
         __half* sz = KV ? p.kv_scale + row : p.kv_scale + 2 * (row * nb + b);
-        const bool unsure = KV ? quant_kv4_store<false>(v, c, m, 0, valid, p.codes + row * 64, sz, p.kv_zero + row)
-                               : quant_kv4_store<PERM>(v, c, mchi, mo, valid,
-                                                       p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1);
+        uint32_t szb;
+        const bool unsure =
+            KV ? quant_kv4_store<false>(v, c, m, 0, valid, p.codes + row * 64, sz, p.kv_zero + row, szb)
+               : quant_kv4_store<PERM>(v, c, mchi, mo, valid, p.codes + row * (p.K / 2) + (size_t)b * 64, sz, sz + 1,
+                                       szb);
         const unsigned pending = __ballot_sync(0xFFFFFFFFu, unsure);
-        if (pending) kv4_second_look_rows<KV ? 7 : LOGB, KV>(pending, p, r0, wig, RPS, smask);
+        if (pending) kv4_second_look_rows<KV ? 7 : LOGB, KV>(pending, szb, p, r0, wig, RPS, smask, stage);
+        refill();
       }
     } else {
       constexpr int NB = NBF ? NBF : 1;
