@@ -72,22 +72,22 @@ def load_peaks():
 ROTATE_SOURCES = ("rq_common.cuh", "rq_rotate.cuh")
 GEMM_SOURCES = ("rq_common.cuh", "rq_tc.cuh", "rq_gemm.cuh")
 ATTN_SOURCES = ("rq_common.cuh", "rq_attn.cuh")
-_ROT, _GEM, _ATT = "6766e941b93707f2", "74cfd6dd085e3e33", "80b39046d2c3159b"
+_ROT, _GEM, _ATT = "121dbfcc644440af", "74cfd6dd085e3e33", "80b39046d2c3159b"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
 # ncu capture of the kernel (summarised in profiles/), with the fingerprint of
 # the sources it was taken on (reported as null once they change).  kv4 and
 # kv4_decode were captured at B = 4 and are scaled to the bench's B = 16 (traffic
 # grows with the vectors processed); kv4_decode is the partial + combine pair.
 TRAFFIC = {
-    ("hadamard_quant", "q_proj_int4"): (16818176, _ROT),
-    ("hadamard_quant", "down_proj_int4"): (105203200, _ROT),
-    ("hadamard_quant", "kv4"): (145912576 * 4, _ROT),
-    ("hadamard_quant", "q_proj_nvfp4"): (16850944, _ROT),
+    ("hadamard_quant", "q_proj_int4"): (16818432, _ROT),
+    ("hadamard_quant", "down_proj_int4"): (108285440, _ROT),
+    ("hadamard_quant", "kv4"): (149308928 * 4, _ROT),
+    ("hadamard_quant", "q_proj_nvfp4"): (16851200, _ROT),
     ("hadamard_quant", "q_proj_mxfp4"): (16832000, _ROT),
-    ("hadamard_quant", "q_proj_w4a8"): (16817408, _ROT),
-    ("hadamard_quant", "q_proj_w8a8"): (16817408, _ROT),
+    ("hadamard_quant", "q_proj_w4a8"): (16817920, _ROT),
+    ("hadamard_quant", "q_proj_w8a8"): (16817920, _ROT),
     ("hadamard_quant", "q_proj_nvfp4_b16"): (16850944, _ROT),
-    ("hadamard_quant", "q_proj_int4_asym"): (16849664, _ROT),
+    ("hadamard_quant", "q_proj_int4_asym"): (16847360, _ROT),
     ("hadamard_quant", "kv4_decode"): (72226048 * 4, _ATT),
     ("gemm", "q_proj_int4"): (12650496, _GEM),
     ("gemm", "down_proj_int4"): (59438848, _GEM),

@@ -705,8 +705,9 @@ __device__ __noinline__ void kv4_second_look_rows(unsigned pending, uint32_t szb
                                                   int wig, int RPS, const uint32_t* smask, const uint8_t* stage) {
   const int nb = p.nb;
   kv4_second_look<LOGB>(pending, szb, [&](int L) {
-    const int rL = RPS > 1 ? L / nb : 0;
-    const int bL = RPS > 1 ? L - rL * nb : wig * 32 + L;
+    // KV4: one head vector per lane (K = 128, 32 rows per stage)
+    const int rL = KV ? L : (RPS > 1 ? L / nb : 0);
+    const int bL = KV ? 0 : (RPS > 1 ? L - rL * nb : wig * 32 + L);
     const int64_t rowL = r0 + rL;
     KvGroup gr;
     gr.src = stage + (size_t)rL * p.K * 2 + (size_t)bL * 256;
