@@ -58,6 +58,75 @@ def test_kv4_constant_and_zero_vectors(rq):
     assert parity.to_np(scale)[0, 0, 0] == 0 and np.all(parity.to_np(codes)[0, 0, 0] == 0)
 
 
+def _near_fp16_midpoint_vectors(signs, n, seed):
+    """n head vectors whose exact rotated min (even rows) or (max - min)/15 (odd
+    rows) lies within 2^-22 of its size from an fp16 rounding midpoint, where an
+    fp32 rotation may round z or s to the wrong side: the kernels must take
+    those decisions from the exact values (their fp64 second look).
+
+    Each vector has three nonzero channels, 1, 2 and 4, holding a, b, c (times
+    the channel's sign): after diag(s) and H_128 / sqrt(128) its values are
+    (+-a +-b +-c) / sqrt(128), the min -(a + b + c) / sqrt(128) at channel 7
+    and the max at channel 0.  a + b + c, three bf16 values of falling size,
+    is chosen to put the target within 2^-22 of a midpoint; rows that miss are
+    redrawn.  Plain numpy on the pages' definitions; the expected values come
+    from the oracle."""
+    rng = np.random.default_rng(seed)
+    c = 2.0 ** -3.5
+
+    def bf16(v):
+        return float(torch.tensor(v, dtype=torch.float64).to(torch.bfloat16).to(torch.float64))
+
+    def midpoint(t):
+        ulp = np.ldexp(1.0, int(np.floor(np.log2(t))) - 10)
+        return (np.floor(t / ulp) + 0.5) * ulp
+
+    rows = []
+    while len(rows) < n:
+        scale_row = len(rows) % 2 == 1
+        m = midpoint(2.0 ** rng.uniform(-6, 6))
+        t = m * (1.0 + rng.uniform(-2.0 ** -24, 2.0 ** -24))
+        total = t * 15.0 / (2.0 * c) if scale_row else t / c
+        a = bf16(total * 0.99)
+        b = bf16(total - a)
+        cc = bf16(total - a - b)
+        got = (a + b + cc) * c * (2.0 / 15.0 if scale_row else 1.0)
+        if not (a > 0 and b > 0 and cc > 0) or abs(got - midpoint(got)) > 2.0 ** -22 * got:
+            continue
+        x = np.zeros(128)
+        x[1], x[2], x[4] = a * signs[1], b * signs[2], cc * signs[4]
+        rows.append(x)
+    return np.array(rows)
+
+
+def _check_exact_scale_zero(codes, scale, zero, xr):
+    q, s_h, z_h, tie, _ = quant.kv4_vectors(xr)
+    # no tie excuse for the fp16 decisions: they must be the exact ones
+    np.testing.assert_array_equal(np.asarray(scale, dtype=np.float64).reshape(s_h.shape), s_h)
+    np.testing.assert_array_equal(np.asarray(zero, dtype=np.float64).reshape(z_h.shape), z_h)
+    parity.check_codes(quant.unpack_nibbles(codes, signed=False).reshape(q.shape), q, tie, what="codes")
+
+
+def test_kv4_scale_zero_near_fp16_midpoints(rq):
+    sg = syn.workload_signs("kv4")
+    x = _near_fp16_midpoint_vectors(sg.numpy(), 512, 77)
+    kv = torch.from_numpy(x).to(torch.bfloat16).reshape(1, 1, -1, 128)
+    assert np.array_equal(parity.bf16_to_f64(kv).reshape(x.shape), x)   # the inputs are exactly these
+    codes, scale, zero = rq.kv_rotate_quantize(kv.cuda(), sg.cuda())
+    xr = hadamard.rotate(x, sg.numpy(), 128)
+    _check_exact_scale_zero(parity.to_np(codes).reshape(-1, 64), parity.to_np(scale), parity.to_np(zero), xr)
+
+
+def test_int4_asym_scale_zero_near_fp16_midpoints(rq):
+    sg = syn.workload_signs("kv4")
+    x = _near_fp16_midpoint_vectors(sg.numpy(), 384, 78)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    codes, sz, _ = rq.rotate_quantize(xb.cuda(), sg.cuda(), 128, "int4_asym")
+    sz = parity.to_np(sz).astype(np.float64).reshape(-1, 2)
+    xr = hadamard.rotate(x, sg.numpy(), 128)
+    _check_exact_scale_zero(parity.to_np(codes), sz[:, 0], sz[:, 1], xr)
+
+
 # ---------------------------------------------------------------- INT4 GEMM on identical codes
 def _rand_int4_operands(m, n, k, seed):
     rng = np.random.default_rng(seed)
