@@ -237,7 +237,8 @@ RQ_API rq_status rq_int_gemm(const uint8_t* xcodes_dev, const float* xscales_dev
  * q = clamp(rint((v~ - z_h)/s_h), 0, 15) (s_h = 0 gives q = 0).  z_h and s_h
  * are the fp16 roundings of the exact min and scale: the rotation runs in
  * fp32, and a vector whose fp32 min or scale lies near an fp16 rounding
- * midpoint has its min and max re-evaluated in fp64 (about 1 % of vectors).
+ * midpoint has its min and max re-evaluated in fp64 (about 0.3 % of
+ * vectors), within the same kernel.
  *  KV_dev      bf16, element (b,h,t,d) at KV_dev + b*strides_host[0] + h*strides_host[1]
  *              + t*strides_host[2] + d (strides in elements; d contiguous; each
  *              vector 16-byte aligned).
