@@ -40,6 +40,57 @@ def _gauss(m, k, seed, outliers=()):
     return x.to(torch.bfloat16)
 
 
+def _int_midpoint_rows(qmax, k, seed):
+    """Rows of k bf16 values whose quotients x / s, s = fp32(amax / qmax) the
+    row's stored scale, fall exactly on midpoints j + 1/2: amax is qmax * m *
+    2^e with m in {1, 1.25, 1.5, 1.75} (so s = m 2^e is exact in fp32) and the
+    row holds +-(j + 1/2) s for every j with that value exact in bf16, besides
+    amax itself; the rest of the row is small filler.  The plain definition
+    rounds them half to even, so every code is fixed; a product with the
+    reciprocal 1/s (inexact for m = 1.25, 1.5, 1.75) can land on either side."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    ms = (1.0, 1.25, 1.5, 1.75) if qmax == 7 else (1.0,)
+    for m in ms:
+        for e in (-3, 0, 2):
+            s = m * 2.0 ** e
+            amax = qmax * s
+            vals = [(j + 0.5) * s for j in range(qmax)]
+            vals = [v for v in vals if float(torch.tensor(v).to(torch.bfloat16)) == v]
+            row = np.zeros(k)
+            row[0] = amax if rng.random() < 0.5 else -amax
+            pos = rng.permutation(np.arange(1, k))
+            for n, v in enumerate(vals):
+                row[pos[2 * n]] = v
+                row[pos[2 * n + 1]] = -v
+            rest = pos[2 * len(vals):]
+            row[rest] = rng.uniform(-0.2, 0.2, len(rest)) * s
+            rows.append(row)
+    x = torch.from_numpy(np.array(rows)).to(torch.bfloat16)
+    return x
+
+
+@pytest.mark.parametrize("fmt,qmax", [("int4", 7), ("int8", 127)])
+def test_int_block1_exact_midpoints(rq, fmt, qmax):
+    """The unrotated arm takes its codes from x / s itself: on rows full of
+    exact midpoints every code must equal the plain definition's (half to
+    even), with no tie excused."""
+    k = 512
+    x = _int_midpoint_rows(qmax, k, 41 + qmax)
+    xd = parity.bf16_to_f64(x)
+    assert np.all(np.abs(xd).max(axis=1) == np.abs(xd[:, 0]))   # amax is where it was put
+    ones = torch.ones(k, dtype=torch.int8)
+    codes, sc, _ = rq.rotate_quantize(x.cuda(), ones.cuda(), 1, fmt)
+    torch.cuda.synchronize()
+    q, s_ref, tie = quant.int_sym_rows(xd, 4 if fmt == "int4" else 8)
+    assert tie.sum() >= 2 * 7 * x.shape[0] // 2      # the rows really sit on midpoints
+    np.testing.assert_array_equal(parity.to_np(sc), s_ref)
+    got = parity.to_np(codes)
+    got = quant.unpack_nibbles(got, signed=True) if fmt == "int4" else got.astype(np.int64)
+    np.testing.assert_array_equal(got, q)
+    rq.get_device_error()
+
+
 @pytest.mark.parametrize("m,k", [(37, 512), (300, 4096), (5, 12288)])
 def test_rotate_f32_block1_is_the_sign_flip(rq, m, k):
     x = _gauss(m, k, m + k, outliers=[(3, 50.0)])
