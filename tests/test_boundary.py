@@ -268,6 +268,14 @@ def test_binding_checks_gemm_operands():
     _raises("disagree on K", rq.int_gemm, x8, "int8", wq_k, "int4")
     _raises("codes", rq.int_gemm, (torch.empty((8, 512), dtype=torch.uint8), x8[1]), "int8", wq, "int4")
     _raises("CUDA", rq.int_gemm, x8, "int8", wq, "int4")
+    # INT4 weights in the byte layout: one int8 code per channel, K columns
+    x4 = (torch.empty((8, 256), dtype=torch.uint8), torch.empty(8, dtype=torch.float32))
+    wb = (torch.empty((16, 512), dtype=torch.int8), torch.empty(16, dtype=torch.float32))
+    _raises("disagree on K", rq.int_gemm, x4, "int4", (torch.empty((16, 256), dtype=torch.int8), wb[1]),
+            "int4_bytes")                                                            # packed width passed as bytes
+    _raises("codes", rq.int_gemm, x4, "int4", (torch.empty((16, 512), dtype=torch.uint8), wb[1]), "int4_bytes")
+    _raises("int4, int6 or int8", rq.int_gemm, wb, "int4_bytes", wb, "int4_bytes")     # activations never bytes
+    _raises("CUDA", rq.int_gemm, x4, "int4", wb, "int4_bytes")
 
 
 def test_binding_checks_kv_and_attention():
